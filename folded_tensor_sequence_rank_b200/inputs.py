@@ -1,0 +1,76 @@
+"""Seeded synthetic inputs shared by the CUDA path, the tests and the oracle.
+
+This module draws random numbers and nothing else: it holds none of the
+layer's arithmetic (no zigzag map, no shard split, no normalisation), so
+both sides of a parity check can take their inputs from it without sharing
+any of the computation under test.
+
+Recipe (one ``torch.Generator('cpu')`` stream per call, fp32 normal draws,
+each tensor rounded once to bf16 round-to-nearest-even):
+
+* ``layer_inputs``: X [T, h] ~ N(0, 1), then Wq, Wk, Wv, Wo [h, h],
+  W1 [h, F], W2 [F, h] ~ N(0, 0.02^2), all in the math orientation
+  ``y = x @ W`` ([in, out]).
+* ``rank_inputs``: the rank's own tokens x_local [L, h] ~ N(0, 1), the six
+  weights as above, then a stand-in for the all-gathered key/value tensors
+  K, V [T, h] ~ N(0, kv_std^2).  ``kv_std`` defaults to 0.02*sqrt(h), the
+  standard deviation of LayerNorm(x) @ W for such weights, so attention
+  logits have the spread the real projection gives.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+WEIGHT_STD = 0.02
+WEIGHT_NAMES = ("wq", "wk", "wv", "wo", "w1", "w2")
+
+
+def _draw(gen: torch.Generator, shape, std: float) -> torch.Tensor:
+    t = torch.randn(*shape, generator=gen, dtype=torch.float32)
+    if std != 1.0:
+        t.mul_(std)
+    return t.to(torch.bfloat16)
+
+
+def _weights(gen: torch.Generator, h: int, F: int) -> dict:
+    shapes = {"wq": (h, h), "wk": (h, h), "wv": (h, h), "wo": (h, h),
+              "w1": (h, F), "w2": (F, h)}
+    return {n: _draw(gen, shapes[n], WEIGHT_STD) for n in WEIGHT_NAMES}
+
+
+def layer_inputs(T: int, h: int, F: int, seed: int) -> dict:
+    """Full-sequence activations X [T, h] and the six layer weights (bf16, CPU)."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(seed)
+    out = {"x": _draw(gen, (T, h), 1.0)}
+    out.update(_weights(gen, h, F))
+    return out
+
+
+def rank_inputs(L: int, T: int, h: int, F: int, seed: int,
+                kv_std: float | None = None) -> dict:
+    """One rank's tokens, the weights and stand-in full-sequence K/V (bf16, CPU)."""
+    if kv_std is None:
+        kv_std = WEIGHT_STD * math.sqrt(h)
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(seed)
+    out = {"x_local": _draw(gen, (L, h), 1.0)}
+    out.update(_weights(gen, h, F))
+    out["k_full"] = _draw(gen, (T, h), kv_std)
+    out["v_full"] = _draw(gen, (T, h), kv_std)
+    return out
+
+
+def sample_rows(n_rows: int, n_sample: int, seed: int, must: tuple = ()) -> list:
+    """A deterministic sorted sample of row indices in [0, n_rows), including `must`."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(seed + 7919)
+    picked = set(int(m) for m in must if 0 <= int(m) < n_rows)
+    extra = torch.randperm(n_rows, generator=gen)[: max(0, n_sample)].tolist()
+    for e in extra:
+        if len(picked) >= len(set(must)) + n_sample:
+            break
+        picked.add(int(e))
+    return sorted(picked)

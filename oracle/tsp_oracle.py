@@ -1,0 +1,276 @@
+"""Oracle for the TSP per-rank dense-layer forward: plain, slow, CPU, fp64.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports, calls or
+executes this module: only the tests, the smoke check and the benchmark's
+CPU-baseline leg do.  It shares no code with the CUDA library and imports
+nothing from it.
+
+Source of the method: the zubnet.ai news item "Zyphra TSP folds TP+SP onto
+one GPU axis" (four paragraphs, cited below as [TSP ¶n]):
+
+* [TSP ¶1] Tensor and sequence parallelism are folded onto one device-mesh
+  axis of size D: every GPU holds 1/D of the weights *and* 1/D of the
+  sequence tokens.  The validated model is a dense decoder (h=4096, 32 Q/KV
+  heads, FFN = 4h, bf16) at 128K tokens with D=8.
+* [TSP ¶2] Attention: weight shards are broadcast one after another, each GPU
+  applies every shard to its own tokens, and K/V are all-gathered with a
+  zigzag sequence partition for load balance.  MLP: a ring passes the weight
+  shards point to point, which removes tensor parallelism's all-reduce.
+* [TSP ¶4] The MLP-without-all-reduce step stands on its own.
+
+The pages give no layer internals.  The layer form used here is the one the
+workload states: pre-LayerNorm (eps 1e-5, gamma=1, beta=0, biased variance),
+GELU with the tanh approximation, no biases, no positional encoding, causal
+softmax with scale 1/sqrt(head_dim), multi-head attention with as many K/V
+heads as Q heads.
+
+Because re-partitioning weights and tokens does not change what a layer
+computes, the per-rank TSP output is exactly (up to summation order) the
+rows, at that rank's token positions, of the plain unsharded layer.  So the
+reference for parity is that plain definition (``layer_forward`` and, given
+the all-gathered K/V, ``rank_rows_forward``).  ``rank_forward_sharded`` and
+``kv_all_gather_sharded`` restate the pages' shard-by-shard schedule; tests
+pin them to the plain definition (the sum over shards equals the unsharded
+contraction).
+
+Precision: every product and sum is fp64.  A bf16 layer stores the
+activations that feed its matmuls in bf16, so the oracle rounds exactly
+those to bf16 (round to nearest even): LN1 output, Q, K, V, the attention
+output, LN2 output and the GELU output H.  The residual stream (X + attn,
+and the layer output) stays fp64.  ``bf16_points=False`` gives the pure
+fp64 layer for diagnostics.
+
+Zigzag partition: the sequence is cut into 2D equal chunks of c = T/(2D)
+tokens, and rank r holds chunks r and 2D-1-r, in that order.
+
+Parity status: every function here is pinned by tests/test_oracle_pins.py
+(closed forms, invariants, brute force and independent library routines).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+LN_EPS = 1e-5
+
+
+# ----------------------------------------------------------------------------
+# bf16 storage rounding
+# ----------------------------------------------------------------------------
+def round_bf16(x) -> np.ndarray:
+    """Round each value to the nearest bf16 number (ties to even), kept as fp64.
+
+    bf16 keeps 8 significant bits.  frexp gives x = m * 2**e with
+    0.5 <= |m| < 1, so m*256 carries exactly 8 integer bits and rint (which
+    rounds half to even) performs the rounding; ldexp scales back.  Valid for
+    the normal range, which is all the layer produces.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)
+    return np.ldexp(np.rint(m * 256.0) / 256.0, e)
+
+
+def _maybe_round(x, on: bool):
+    return round_bf16(x) if on else x
+
+
+# ----------------------------------------------------------------------------
+# token partition  [TSP ¶2: "zigzag partition"]
+# ----------------------------------------------------------------------------
+def zigzag_index(T: int, D: int, rank: int) -> np.ndarray:
+    """Global positions of rank `rank`'s tokens, in rank-local order.
+
+    T tokens are cut into 2D chunks of c = T/(2D); rank r holds chunk r, then
+    chunk 2D-1-r.  Returned as int64 [2c].
+    """
+    if T % (2 * D) != 0:
+        raise ValueError("T must be a multiple of 2D")
+    if not 0 <= rank < D:
+        raise ValueError("rank out of range")
+    c = T // (2 * D)
+    first = np.arange(rank * c, (rank + 1) * c, dtype=np.int64)
+    second = np.arange((2 * D - 1 - rank) * c, (2 * D - rank) * c, dtype=np.int64)
+    return np.concatenate([first, second])
+
+
+# ----------------------------------------------------------------------------
+# elementwise pieces of the layer
+# ----------------------------------------------------------------------------
+def layer_norm(x, eps: float = LN_EPS) -> np.ndarray:
+    """Row-wise (x - mean) / sqrt(var + eps), biased variance, gamma=1, beta=0."""
+    x = np.asarray(x, dtype=np.float64)
+    mean = x.mean(axis=-1, keepdims=True)
+    centred = x - mean
+    var = (centred * centred).mean(axis=-1, keepdims=True)
+    return centred / np.sqrt(var + eps)
+
+
+def gelu_tanh(x) -> np.ndarray:
+    """GELU, tanh form: 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))."""
+    x = np.asarray(x, dtype=np.float64)
+    inner = np.sqrt(2.0 / np.pi) * (x + 0.044715 * x * x * x)
+    return 0.5 * x * (1.0 + np.tanh(inner))
+
+
+def causal_attention(q, k, v, q_pos, n_heads: int, scale: float,
+                     return_probs: bool = False):
+    """Multi-head causal attention of query rows at global positions `q_pos`.
+
+    q: [n, H*d] query rows; k, v: [T, H*d] full-sequence keys/values in
+    natural order, head j in columns j*d .. (j+1)*d.  Row i attends to the
+    keys at positions 0 .. q_pos[i] inclusive, with weights
+    softmax(scale * q.k).  Returns [n, H*d] (and the per-head probability
+    matrices when asked).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    q_pos = np.asarray(q_pos, dtype=np.int64)
+    n, hd = q.shape
+    d = hd // n_heads
+    kmax = int(q_pos.max()) + 1 if n else 0
+    out = np.zeros((n, hd), dtype=np.float64)
+    probs = []
+    if n == 0:
+        return (out, probs) if return_probs else out
+    key_pos = np.arange(kmax, dtype=np.int64)
+    allowed = key_pos[None, :] <= q_pos[:, None]            # [n, kmax]
+    for j in range(n_heads):
+        cols = slice(j * d, (j + 1) * d)
+        kj = np.asarray(k[:kmax, cols], dtype=np.float64)
+        vj = np.asarray(v[:kmax, cols], dtype=np.float64)
+        scores = scale * (q[:, cols] @ kj.T)                 # [n, kmax]
+        scores = np.where(allowed, scores, -np.inf)
+        scores -= scores.max(axis=1, keepdims=True)
+        w = np.exp(scores)
+        w /= w.sum(axis=1, keepdims=True)
+        out[:, cols] = w @ vj
+        if return_probs:
+            probs.append(w)
+    return (out, probs) if return_probs else out
+
+
+# ----------------------------------------------------------------------------
+# the plain (unsharded) layer
+# ----------------------------------------------------------------------------
+def _f64(w: dict) -> dict:
+    return {n: np.asarray(a, dtype=np.float64) for n, a in w.items()}
+
+
+def kv_project(x_rows, w: dict, eps: float = LN_EPS, bf16_points: bool = True):
+    """K and V rows of tokens `x_rows`: LN1(x) @ Wk and LN1(x) @ Wv."""
+    w = _f64(w)
+    xn = _maybe_round(layer_norm(x_rows, eps), bf16_points)
+    k = _maybe_round(xn @ w["wk"], bf16_points)
+    v = _maybe_round(xn @ w["wv"], bf16_points)
+    return k, v
+
+
+def rank_rows_forward(x_rows, q_pos, k_full, v_full, w: dict, n_heads: int,
+                      eps: float = LN_EPS, scale: float | None = None,
+                      bf16_points: bool = True) -> dict:
+    """Layer output for tokens `x_rows` at global positions `q_pos`.
+
+    `k_full`, `v_full` [T, h] are the keys and values of the whole sequence
+    (what every rank holds after the all-gather).  Every step is row-local
+    except attention, so any subset of a rank's rows can be computed alone.
+    Returns the output and the bf16-stored intermediates.
+    """
+    w = _f64(w)
+    x = np.asarray(x_rows, dtype=np.float64)
+    h = x.shape[1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(h // n_heads)
+    r = bf16_points
+    xn1 = _maybe_round(layer_norm(x, eps), r)
+    q = _maybe_round(xn1 @ w["wq"], r)
+    a = _maybe_round(causal_attention(q, k_full, v_full, q_pos, n_heads, scale), r)
+    y1 = x + a @ w["wo"]
+    xn2 = _maybe_round(layer_norm(y1, eps), r)
+    hh = _maybe_round(gelu_tanh(xn2 @ w["w1"]), r)
+    y = y1 + hh @ w["w2"]
+    return {"xn1": xn1, "q": q, "a": a, "y1": y1, "xn2": xn2, "h": hh, "y": y}
+
+
+def layer_forward(x, w: dict, n_heads: int, eps: float = LN_EPS,
+                  scale: float | None = None, bf16_points: bool = True) -> dict:
+    """The whole unsharded layer over a full sequence x [T, h] (natural order)."""
+    x = np.asarray(x, dtype=np.float64)
+    k, v = kv_project(x, w, eps, bf16_points)
+    out = rank_rows_forward(x, np.arange(x.shape[0]), k, v, w, n_heads, eps,
+                            scale, bf16_points)
+    out["k"], out["v"] = k, v
+    return out
+
+
+# ----------------------------------------------------------------------------
+# the pages' shard-by-shard schedule  [TSP ¶1, ¶2]
+# ----------------------------------------------------------------------------
+def kv_all_gather_sharded(x_full, D: int, w: dict, eps: float = LN_EPS,
+                          bf16_points: bool = True):
+    """Full-sequence K/V as TSP builds it.
+
+    Every rank r projects its own zigzag tokens with every attention shard
+    k (head group k = columns k*h/D .. (k+1)*h/D of Wk, Wv); the all-gather
+    places each rank's rows back at their global positions.
+    """
+    w = _f64(w)
+    x_full = np.asarray(x_full, dtype=np.float64)
+    T, h = x_full.shape
+    hs = h // D
+    K = np.zeros((T, h))
+    V = np.zeros((T, h))
+    for rank in range(D):
+        idx = zigzag_index(T, D, rank)
+        xn = _maybe_round(layer_norm(x_full[idx], eps), bf16_points)
+        for s in range(D):
+            cols = slice(s * hs, (s + 1) * hs)
+            K[idx, cols] = _maybe_round(xn @ w["wk"][:, cols], bf16_points)
+            V[idx, cols] = _maybe_round(xn @ w["wv"][:, cols], bf16_points)
+    return K, V
+
+
+def rank_forward_sharded(rank: int, D: int, x_local, k_full, v_full, w: dict,
+                         n_heads: int, eps: float = LN_EPS,
+                         scale: float | None = None,
+                         bf16_points: bool = True) -> np.ndarray:
+    """Rank `rank`'s output computed the way TSP schedules it.
+
+    Attention: shard k (heads k*H/D .. (k+1)*H/D of Wq and Wo) is applied to
+    the local tokens in turn and its output projection is accumulated.
+    MLP: at ring step s the rank holds W1/W2 shard (rank+s) mod D (FFN columns
+    of W1, rows of W2) and adds GELU(x W1_k) W2_k; the sum over shards is
+    local, so no all-reduce is needed.
+    """
+    w = _f64(w)
+    x = np.asarray(x_local, dtype=np.float64)
+    L, h = x.shape
+    T = np.asarray(k_full).shape[0]
+    F = w["w1"].shape[1]
+    hs, Fs, Hs = h // D, F // D, n_heads // D
+    if scale is None:
+        scale = 1.0 / np.sqrt(h // n_heads)
+    r = bf16_points
+    pos = zigzag_index(T, D, rank)
+    xn1 = _maybe_round(layer_norm(x, eps), r)
+    y1 = x.copy()
+    for s in range(D):
+        cols = slice(s * hs, (s + 1) * hs)
+        q_s = _maybe_round(xn1 @ w["wq"][:, cols], r)
+        a_s = _maybe_round(causal_attention(q_s, np.asarray(k_full)[:, cols],
+                                            np.asarray(v_full)[:, cols], pos,
+                                            Hs, scale), r)
+        y1 = y1 + a_s @ w["wo"][cols, :]
+    xn2 = _maybe_round(layer_norm(y1, eps), r)
+    y = y1.copy()
+    for step in range(D):
+        s = (rank + step) % D
+        cols = slice(s * Fs, (s + 1) * Fs)
+        h_s = _maybe_round(gelu_tanh(xn2 @ w["w1"][:, cols]), r)
+        y = y + h_s @ w["w2"][cols, :]
+    return y
+
+
+# ----------------------------------------------------------------------------
+# work accounting
+# ----------------------------------------------------------------------------
+def causal_pairs(T: int, D: int, rank: int) -> int:
+    """Number of (query, key) pairs rank `rank` scores: sum over its tokens of pos+1."""
+    return int((zigzag_index(T, D, rank) + 1).sum())
