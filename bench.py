@@ -1,0 +1,360 @@
+#!/usr/bin/env python
+"""Benchmark of one TSP rank step on B200: the rank projects its own K/V and
+runs its layer forward (LN1, QKV, causal zigzag attention, O + residual, LN2,
+W1 + GELU, W2 + residual) for the 7B dense layer at T = 131072, D = 8.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tsp|reference]
+
+One process per GPU (torchrun for N > 1); every GPU runs TSP rank
+(global rank mod D) on its own synthetic inputs: the per-rank work is
+independent, so the job scales weakly and needs no collective on the data
+path (the barrier and the max-over-ranks timing use NCCL).  Rank 0 prints one
+JSON line.  `--impl reference` times the CPU oracle on host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "TSP layer fwd tokens/s on 1 B200 (7B layer, 128K, D=8); % bf16 tensor peak"
+UNIT = "tokens/s"
+WORKLOADS = {
+    "7b-128k-d8": dict(T=131072, h=4096, H=32, F=16384, D=8, seed=2,
+                       desc="7B dense layer (h=4096, 32 heads x 128, FFN 16384, GELU-tanh, pre-LN), "
+                            "T=131072, D=8: one TSP rank step = own K/V projection + layer forward "
+                            "over 16384 local tokens (2 zigzag chunks of 8192) against 131072 keys"),
+    "7b-8k-d8": dict(T=8192, h=4096, H=32, F=16384, D=8, seed=1,
+                     desc="7B dense layer, T=8192, D=8, one TSP rank step"),
+    "7b-32k-d8": dict(T=32768, h=4096, H=32, F=16384, D=8, seed=4,
+                      desc="7B dense layer, T=32768, D=8, one TSP rank step"),
+}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            m = json.load(f)
+        return m, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def rank_flops(T, h, F, D, rank):
+    """Algorithmic FLOPs of one rank step (GEMMs + unmasked causal pairs)."""
+    c = T // (2 * D)
+    L = 2 * c
+    pairs = c * c * (2 * D - 1) + c * (c + 1)          # sum over local tokens of (pos + 1)
+    attn = 4 * h * pairs                               # QK^T and PV, all heads
+    qkv = 2 * L * h * 3 * h
+    o = 2 * L * h * h
+    mlp = 2 * 2 * L * h * F
+    return {"attention": attn, "qkv": qkv, "o": o, "mlp": mlp, "total": attn + qkv + o + mlp}
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = "index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active," \
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown," \
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(gpu_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------- dist
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus and world > 1:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    return world, rank, local
+
+
+def traffic_record(kernel_file):
+    """dram bytes per attention launch from the committed ncu summary, if it was
+    taken on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "attn_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    with open(kernel_file, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    if rec.get("source_sha") != sha:
+        return None
+    return rec
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+def oracle_sample(wl, n_rows, seed=0, cache={}):
+    """Times the oracle on `n_rows` of one rank's tokens (spread evenly over
+    both zigzag chunks): their K/V projection plus their layer output given
+    the full-sequence K/V.  Returns (seconds, rows, threads)."""
+    import numpy as np
+    from folded_tensor_sequence_rank_b200 import inputs
+    from oracle import tsp_oracle as O
+    T, h, F, D, H = wl["T"], wl["h"], wl["F"], wl["D"], wl["H"]
+    L = T // D
+    key = (T, h, F, D)
+    if key not in cache:
+        raw = inputs.rank_inputs(L, T, h, F, wl["seed"])
+        cache.clear()
+        cache[key] = dict(x=raw["x_local"].double().numpy(),
+                          w={n: raw[n].double().numpy() for n in inputs.WEIGHT_NAMES},
+                          K=raw["k_full"].float().numpy(), V=raw["v_full"].float().numpy())
+    st = cache[key]
+    c = L // 2
+    half = max(1, n_rows // 2)
+    offs = (np.arange(half) * c) // half + (seed % max(1, c // half))
+    rows = np.concatenate([offs, c + offs])[:max(1, n_rows)]
+    pos = O.zigzag_index(T, D, 0)[rows]
+    t0 = time.perf_counter()
+    O.kv_project(st["x"][rows], st["w"])
+    O.rank_rows_forward(st["x"][rows], pos, st["K"], st["V"], st["w"], H)
+    dt = time.perf_counter() - t0
+    return dt, len(rows)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def cpu_baseline(wl, budget_s=15.0):
+    dt, n = oracle_sample(wl, 4)                 # first call includes input generation
+    dt, n = oracle_sample(wl, 4, seed=1)
+    rows = max(2, min(64, int(4 * budget_s / max(dt, 1e-3))))
+    rows -= rows % 2
+    dt, n = oracle_sample(wl, rows, seed=2)
+    return {"value": n / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} of the rank's {wl['T'] // wl['D']} tokens (half in each zigzag chunk, evenly spaced): "
+                      f"their K/V projection and layer output in fp64 numpy given the full 131072-token K/V; "
+                      f"{dt:.1f} s"}
+
+
+def run_reference(args, wl):
+    world, rank, _ = dist_setup(args.gpus)
+    if rank != 0:
+        return
+    oracle_sample(wl, 2)                                   # inputs built once, untimed
+    dt1, _ = oracle_sample(wl, 2, seed=1)
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    rows = max(2, int(2 * budget / max(dt1, 1e-3)))
+    rows -= rows % 2
+    for i in range(args.warmup):
+        oracle_sample(wl, rows, seed=10 + i)
+    tot_t, tot_n = 0.0, 0
+    for i in range(args.steps):
+        dt, n = oracle_sample(wl, rows, seed=100 + i)
+        tot_t += dt
+        tot_n += n
+    value = tot_n / tot_t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * tot_t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl["desc"], "T": wl["T"], "D": wl["D"], "rank": 0},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"{rows} tokens per step (half per zigzag chunk)"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------- GPU arm
+def run_tsp(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    from folded_tensor_sequence_rank_b200 import tsp
+
+    world, grank, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    T, h, H, F, D = wl["T"], wl["h"], wl["H"], wl["F"], wl["D"]
+    trank = grank % D
+    L = T // D
+    dims = tsp.make_dims(T, h, H, F)
+    tsp.lib()
+
+    # synthetic inputs, drawn on the device (parity is the tests' job)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(wl["seed"] * 1000 + grank)
+    def rnd(*shape, std=1.0):
+        return (torch.randn(*shape, generator=g, device="cuda", dtype=torch.float32) * std).to(torch.bfloat16)
+    w_full = {"wq": rnd(h, h, std=0.02), "wk": rnd(h, h, std=0.02), "wv": rnd(h, h, std=0.02),
+              "wo": rnd(h, h, std=0.02), "w1": rnd(h, F, std=0.02), "w2": rnd(F, h, std=0.02)}
+    sw = tsp.pack_shards(dims, D, w_full)
+    del w_full
+    kv_std = 0.02 * math.sqrt(h)
+    x_local = rnd(L, h)
+    K = rnd(T, h, std=kv_std)
+    V = rnd(T, h, std=kv_std)
+    y = torch.empty(L, h, dtype=torch.bfloat16, device="cuda")
+    ws = tsp.alloc_workspace(dims, D)
+    stream = torch.cuda.current_stream()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(tsp.N_STEP_EVENTS)] for _ in range(args.steps)]
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        tsp.rank_step(dims, sw, trank, x_local, K, V, y, ws)
+    torch.cuda.synchronize()
+    assert tsp.get_device_status(ws) == tsp.TSP_OK, "device wait timed out during warm-up"
+
+    # --- device-timed steps, inputs resident in HBM
+    step_ms = {k: 0.0 for k in ("ln1", "qkv", "attention", "o", "ln2", "w1", "w2")}
+    barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    per_step = []
+    for i in range(args.steps):
+        tsp.rank_step(dims, sw, trank, x_local, K, V, y, ws, events=evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier()
+    ms = t0.elapsed_time(t1) / args.steps
+    names = list(step_ms)
+    for ev in evs:
+        for j, n in enumerate(names):
+            step_ms[n] += ev[j].elapsed_time(ev[j + 1]) / args.steps
+    kern_ms = sum(step_ms.values())
+
+    # --- end to end: host (pinned) tokens in, host result out, through the C ABI
+    hx = x_local.cpu().pin_memory()
+    hy = torch.empty(L, h, dtype=torch.bfloat16).pin_memory()
+    xs = torch.empty_like(x_local)
+    ys = torch.empty_like(y)
+    for _ in range(2):
+        tsp.rank_step_host(dims, sw, trank, hx, xs, K, V, ys, hy, ws)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        tsp.rank_step_host(dims, sw, trank, hx, xs, K, V, ys, hy, ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    assert tsp.get_device_status(ws) == tsp.TSP_OK, "device wait timed out"
+
+    if world > 1:
+        t = torch.tensor([ms, e2e_ms, step_ms["attention"]], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms, attn_ms = t.tolist()
+    else:
+        attn_ms = step_ms["attention"]
+
+    if grank == 0:
+        pk, src = peaks()
+        fl = rank_flops(T, h, F, D, trank)
+        peak_tf = pk["bf16_tflops_sustained"]
+        attn_tf = fl["attention"] / (attn_ms * 1e-3) / 1e12
+        traf = traffic_record(os.path.join(ROOT, "folded_tensor_sequence_rank_b200", "csrc", "attn_sm100.cuh"))
+        value = world * L / (ms * 1e-3)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl["desc"], "T": T, "D": D, "tsp_rank": trank, "local_tokens": L,
+                       "parallelism": f"{world} GPU(s), each an independent TSP rank (rank = gpu mod {D})",
+                       "l2": "inputs larger than L2 (K/V 2 x 1 GiB, weights 384 MiB); no flush"},
+            "roofline": {"bound": "tensor", "kernel": "attn_fwd_tcgen05<128>", "achieved": attn_tf,
+                         "peak": peak_tf, "unit": "TFLOP/s", "frac": attn_tf / peak_tf,
+                         "peak_source": f"{src} bf16_tflops_sustained (kernel timed inside a long step)",
+                         "algorithmic_per_launch": f"{fl['attention']:.4e} FLOP = 4 h x causal pairs",
+                         "traffic": (traf["bytes_per_launch"] if traf else None)},
+            "step_tflops": fl["total"] / (ms * 1e-3) / 1e12,
+            "step_frac_of_peak": fl["total"] / (ms * 1e-3) / 1e12 / peak_tf,
+            "kernel_ms": {k: round(v, 4) for k, v in step_ms.items()},
+            "kernel_ms_sum": kern_ms,
+            "gpu_launches": 7 * args.steps,
+            "e2e": {"value": world * L / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": L * h * 2,
+                    "d2h_bytes_per_step": L * h * 2},
+            "clocks": clk,
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="tsp", choices=["tsp", "reference"])
+    ap.add_argument("--workload", default="7b-128k-d8", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_tsp(args, wl)
+
+
+if __name__ == "__main__":
+    main()

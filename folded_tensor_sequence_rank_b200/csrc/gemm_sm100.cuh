@@ -1,0 +1,301 @@
+// gemm_sm100.cuh - persistent tcgen05 GEMM C = A * B^T for the TSP shard loops.
+//
+// A [M, K] bf16 K-major (one tensor map), B given as a list of per-shard
+// K-major tensor maps.  Two ways the shard list is walked, both without any
+// reduction kernel:
+//   N-split (Q/K/V and W1 shards: each shard owns a block of output columns):
+//     output column block n belongs to map n / shard_n.
+//   K-split (Wo and W2 shards: each shard owns a block of the reduction dim):
+//     k-block kb reads map (kb*64) / shard_k, so one TMEM accumulator sums the
+//     contributions of all D shards - the "no all-reduce" MLP sum of the
+//     TSP news item (zubnet.ai, paragraphs 2 and 4) done inside the K loop.
+//
+// Roles (192 threads, one CTA per SM, persistent over output tiles):
+//   warp 0     TMA producer: A and B tiles into a STAGES-deep shared ring
+//   warp 1     TMEM allocator + single-thread tcgen05.mma issuer
+//   warps 2-5  epilogue: tcgen05.ld the 128 x BN fp32 accumulator (thread =
+//              row), apply store / GELU / residual, write to global memory.
+// Two TMEM accumulators let the epilogue of tile i overlap the K loop of
+// tile i+1.
+#pragma once
+#include "ptx.cuh"
+
+namespace tsp {
+
+constexpr int kGemmBM = 128;
+constexpr int kGemmBK = 64;
+constexpr int kGemmThreads = 192;
+constexpr int kGemmMaxMaps = 48;  // 3 segments x 16 shards
+constexpr int kGemmGroupM = 16;   // M tiles per raster group (L2 reuse of A)
+
+enum GemmEpi : int { kEpiStoreBf16 = 0, kEpiGeluBf16 = 1, kEpiResidual = 2 };
+
+struct __align__(64) GemmParams {
+  CUtensorMap map_a;
+  CUtensorMap map_b[kGemmMaxMaps];
+  int M, N, K;
+  int ksplit;     // 0: N-split, 1: K-split
+  int shard_n;    // N-split: output columns per B map
+  int shard_k;    // K-split: reduction length per B map
+  int seg_n;      // N-split: output columns per output segment
+  int epi;        // GemmEpi
+  void* out[3];   // per segment (N-split) or out[0] (K-split)
+  int remap[3];   // per segment: 1 = write local row m at its global zigzag row
+  int64_t ldo;    // output row stride, elements
+  const void* resid;  // kEpiResidual: residual [M, N] (row stride ldo)
+  int resid_f32;      // residual dtype: 1 fp32, 0 bf16
+  int out_f32;        // kEpiResidual: output fp32 (1) or bf16 (0)
+  int c;              // zigzag: local rows [0,c) -> off0 + m, [c, 2c) -> off1 + m
+  int64_t off0, off1;
+  int* status;
+  uint64_t timeout_ns;
+};
+
+template <int BN>
+struct GemmShape {
+  static constexpr int kABytes = kGemmBM * kGemmBK * 2;
+  static constexpr int kBBytes = BN * kGemmBK * 2;
+  static constexpr int kStages = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);
+  static constexpr int kTmemCols = 2 * BN;  // two accumulators
+  static constexpr int kBarBytes = 256;
+  static constexpr int kSmemBytes = kStages * (kABytes + kBBytes) + kBarBytes + 1024;
+};
+
+__device__ __forceinline__ void gemm_tile_coords(int tile, int num_m, int num_n, int& mb, int& nb) {
+  const int per_group = kGemmGroupM * num_n;
+  const int group = tile / per_group;
+  const int first_m = group * kGemmGroupM;
+  const int gm = min(kGemmGroupM, num_m - first_m);
+  const int local = tile - group * per_group;
+  mb = first_m + local % gm;
+  nb = local / gm;
+}
+
+__device__ __forceinline__ float gelu_tanh_f(float x) {
+  const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
+  const float u = k0 * fmaf(0.044715f * x, x * x, x);
+  return 0.5f * x * (1.0f + tanh_approx(u));
+}
+
+// Bounded wait that ignores the abort flag: used only to drain copies and
+// MMAs this thread itself started, before the CTA exits.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(a, parity)) {
+    if (globaltimer_ns() - t0 > timeout_ns) break;
+  }
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1) gemm_bf16_tcgen05(const __grid_constant__ GemmParams p) {
+  using S = GemmShape<BN>;
+  constexpr int STAGES = S::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * S::kABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * S::kBBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, S::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
+
+  const int num_m = (p.M + kGemmBM - 1) / kGemmBM;
+  const int num_n = p.N / BN;
+  const int num_k = p.K / kGemmBK;
+  const int num_tiles = num_m * num_n;
+
+  if (warp == 0) {
+    if (elect_one()) {
+      tma_prefetch_desc(&p.map_a);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t used = 0, par = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        int mb, nb;
+        gemm_tile_coords(tile, num_m, num_n, mb, nb);
+        const int n0 = nb * BN;
+        for (int kb = 0; kb < num_k; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, ctl)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[stage], S::kABytes + S::kBBytes);
+          tma_load_2d(sA + stage * S::kABytes, &p.map_a, &full[stage], kb * kGemmBK, mb * kGemmBM);
+          const CUtensorMap* mb_map;
+          int bx, by;
+          if (p.ksplit) {
+            const int k0 = kb * kGemmBK;
+            mb_map = &p.map_b[k0 / p.shard_k];
+            bx = k0 % p.shard_k;
+            by = n0;
+          } else {
+            mb_map = &p.map_b[n0 / p.shard_n];
+            bx = kb * kGemmBK;
+            by = n0 % p.shard_n;
+          }
+          tma_load_2d(sB + stage * S::kBBytes, mb_map, &full[stage], bx, by);
+          used |= 1u << stage;
+          par = (par & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      // every copy this thread started lands before the CTA exits
+      for (int s = 0; s < STAGES; ++s)
+        if (used & (1u << s)) mbar_drain(&full[s], (par >> s) & 1, p.timeout_ns);
+    }
+  } else if (warp == 1) {
+    if (elect_one()) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kGemmBM, BN, 0, 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++acc) {
+        const int buf = acc & 1;
+        const uint32_t aph = (acc >> 1) & 1;
+        if (!mbar_wait(&tempty[buf], aph ^ 1, ctl)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * BN;
+        for (int kb = 0; kb < num_k; ++kb) {
+          if (!mbar_wait(&full[stage], phase, ctl)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * S::kABytes);
+          const uint32_t b0 = smem_u32(sB + stage * S::kBBytes);
+#pragma unroll
+          for (int kk = 0; kk < kGemmBK / 16; ++kk) {
+            const uint64_t ad = smem_desc_sw128(a0 + kk * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(b0 + kk * 32, 16, 1024);
+            mma_ss(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (ok) mma_commit(&tfull[buf]);
+      }
+      mma_commit(drain);
+      mbar_drain(drain, 0, p.timeout_ns);
+    }
+  } else {
+    // epilogue warps 2..5 -> TMEM lane quarters 2,3,0,1
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    int acc = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++acc) {
+      int mb, nb;
+      gemm_tile_coords(tile, num_m, num_n, mb, nb);
+      const int buf = acc & 1;
+      const uint32_t aph = (acc >> 1) & 1;
+      if (!mbar_wait(&tfull[buf], aph, ctl)) break;
+      tc_fence_after();
+      const int m = mb * kGemmBM + row;
+      const bool valid = m < p.M;
+      const int64_t grow = (m < p.c) ? (p.off0 + m) : (p.off1 + m);
+#pragma unroll 1
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        uint32_t r[32];
+        __syncwarp();
+        tmem_ld32(tmem_base + lane_off + buf * BN + ch * 32, r);
+        tmem_ld_wait();
+        const int n = nb * BN + ch * 32;
+        if (!valid) {
+        } else if (p.epi == kEpiResidual) {
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+          const int64_t off = static_cast<int64_t>(m) * p.ldo + n;
+          if (p.resid_f32) {
+            const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.resid) + off);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float4 q = src[i];
+              v[4 * i] += q.x; v[4 * i + 1] += q.y; v[4 * i + 2] += q.z; v[4 * i + 3] += q.w;
+            }
+          } else {
+            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.resid) + off);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint4 q = src[i];
+              const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&w[j]);
+                const float2 f = __bfloat1622float2(b2);
+                v[8 * i + 2 * j] += f.x;
+                v[8 * i + 2 * j + 1] += f.y;
+              }
+            }
+          }
+          if (p.out_f32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out[0]) + off);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out[0]) + off);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                                  pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+          }
+        } else {
+          const int seg = n / p.seg_n;
+          const int col = n - seg * p.seg_n;
+          const int64_t orow = p.remap[seg] ? grow : m;
+          uint32_t packed[16];
+          if (p.epi == kEpiGeluBf16) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              packed[i] = pack_bf16x2(gelu_tanh_f(__uint_as_float(r[2 * i])), gelu_tanh_f(__uint_as_float(r[2 * i + 1])));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              packed[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+          }
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out[seg]) + orow * p.ldo + col);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, S::kTmemCols);
+  }
+}
+
+}  // namespace tsp

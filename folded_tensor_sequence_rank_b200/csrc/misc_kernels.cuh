@@ -1,0 +1,138 @@
+// misc_kernels.cuh - the bandwidth-bound pieces of the TSP rank forward:
+// zigzag index map, pre-LayerNorm with bf16 output, weight shard packing, and
+// the bounded-wait self test.
+#pragma once
+#include "ptx.cuh"
+
+namespace tsp {
+
+// Zigzag partition (TSP news item, zubnet.ai, paragraph 2): local token i of
+// rank r sits at global position r*c + i (i < c) or (2D-1-r)*c + (i-c).
+__global__ void zigzag_index_kernel(int32_t* idx, int64_t c, int D, int rank) {
+  const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (i >= 2 * c) return;
+  idx[i] = static_cast<int32_t>(i < c ? rank * c + i : (2 * D - 1 - rank) * c + (i - c));
+}
+
+template <typename T>
+__device__ __forceinline__ void load8(const T* src, float (&v)[8]);
+
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* src, float (&v)[8]) {
+  const uint4 q = __ldg(reinterpret_cast<const uint4*>(src));
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+    v[2 * j] = f.x;
+    v[2 * j + 1] = f.y;
+  }
+}
+
+template <>
+__device__ __forceinline__ void load8<float>(const float* src, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(src));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(src) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// LayerNorm of one row per warp, gamma=1, beta=0:
+//   y = (x - mean) / sqrt(var + eps), var biased, statistics in fp32 over the
+//   row held in registers (two passes: mean, then centred sum of squares).
+// Output bf16 (round to nearest even).  MAXC = 8-element chunks per lane.
+template <typename Tin, int MAXC>
+__global__ void __launch_bounds__(256) layernorm_rows_kernel(const Tin* __restrict__ x, __nv_bfloat16* __restrict__ y,
+                                                             int64_t rows, int h, float eps) {
+  const int warps = blockDim.x >> 5;
+  const int64_t r = blockIdx.x * static_cast<int64_t>(warps) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const int nch = h >> 3;  // 8-element chunks in the row
+  const Tin* xr = x + r * h;
+  float v[MAXC][8];
+  float sum = 0.f;
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    const int ch = lane + 32 * c;
+    if (ch < nch) {
+      load8<Tin>(xr + ch * 8, v[c]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) sum += v[c][j];
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[c][j] = 0.f;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float mean = sum / h;
+  float sq = 0.f;
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    const int ch = lane + 32 * c;
+    if (ch < nch) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float d = v[c][j] - mean;
+        sq = fmaf(d, d, sq);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+  const float rstd = rsqrtf(sq / h + eps);
+  __nv_bfloat16* yr = y + r * h;
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    const int ch = lane + 32 * c;
+    if (ch < nch) {
+      uint4 o;
+      o.x = pack_bf16x2((v[c][0] - mean) * rstd, (v[c][1] - mean) * rstd);
+      o.y = pack_bf16x2((v[c][2] - mean) * rstd, (v[c][3] - mean) * rstd);
+      o.z = pack_bf16x2((v[c][4] - mean) * rstd, (v[c][5] - mean) * rstd);
+      o.w = pack_bf16x2((v[c][6] - mean) * rstd, (v[c][7] - mean) * rstd);
+      *reinterpret_cast<uint4*>(yr + ch * 8) = o;
+    }
+  }
+}
+
+// Shard packing: out[o][i] = w[(row0 + i) * ld + col0 + o] for o < n_out,
+// i < n_in; i.e. a transposed sub-block of the math-orientation weight, giving
+// the K-major [n_out, n_in] layout the GEMM's B operand uses.  32x32 tiles
+// staged through shared memory so both sides are coalesced.
+__global__ void pack_transpose_kernel(const __nv_bfloat16* __restrict__ w, int64_t ld, int64_t row0, int64_t col0,
+                                      __nv_bfloat16* __restrict__ out, int n_out, int n_in) {
+  __shared__ __nv_bfloat16 tile[32][33];
+  const int i0 = blockIdx.x * 32, o0 = blockIdx.y * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
+  for (int k = ty; k < 32; k += 8) {
+    const int i = i0 + k, o = o0 + tx;
+    if (i < n_in && o < n_out) tile[k][tx] = w[(row0 + i) * ld + col0 + o];
+  }
+  __syncthreads();
+  for (int k = ty; k < 32; k += 8) {
+    const int o = o0 + k, i = i0 + tx;
+    if (i < n_in && o < n_out) out[static_cast<int64_t>(o) * n_in + i] = tile[tx][k];
+  }
+}
+
+// Self test of the bounded waits: one thread waits on a barrier that expects
+// an arrival nobody makes.  The wait gives up after timeout_ns, records the
+// timeout in the status word and the kernel returns normally.
+__global__ void wait_timeout_selftest_kernel(int* status, uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const WaitCtl ctl{&abort_flag, status, timeout_ns};
+    mbar_wait(&bar, 0, ctl);
+  }
+}
+
+}  // namespace tsp

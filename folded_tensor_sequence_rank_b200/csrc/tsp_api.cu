@@ -1,0 +1,584 @@
+// tsp_api.cu - the C ABI (include/tsp.h): argument checks, workspace layout,
+// TMA tensor maps and the launch sequence of one TSP rank's layer forward.
+//
+// Launch sequence of tsp_rank_step (one stream, no host synchronisation):
+//   LN1(x_local) -> QKV GEMM (Q local; K, V to their global rows) ->
+//   attention -> O GEMM (+x, fp32 Y1) -> LN2(Y1) -> W1 GEMM (+GELU) ->
+//   W2 GEMM (+Y1) -> y_local.
+// The TSP exchanges (zubnet.ai news item, paragraph 2: shard broadcast, K/V
+// all-gather, MLP ring) are shard pointers already resident on this GPU.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/tsp.h"
+#include "attn_sm100.cuh"
+#include "gemm_sm100.cuh"
+#include "misc_kernels.cuh"
+
+namespace {
+
+using namespace tsp;
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
+constexpr size_t kAlign = 1024;
+
+thread_local char g_cuda_err[256] = "";
+
+int cuda_fail(cudaError_t e, const char* where) {
+  std::snprintf(g_cuda_err, sizeof(g_cuda_err), "%s: %s", where, cudaGetErrorString(e));
+  return TSP_ERR_CUDA;
+}
+
+#define TSP_CUDA(call)                                   \
+  do {                                                   \
+    cudaError_t e_ = (call);                             \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #call);  \
+  } while (0)
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// ---------------------------------------------------------------- tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 row-major [rows, cols] with row stride ld elements; box = 64
+// columns (128 bytes, 128B swizzle) x box_rows rows.
+int make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) {
+    std::snprintf(g_cuda_err, sizeof(g_cuda_err), "cuTensorMapEncodeTiled unavailable");
+    return TSP_ERR_CUDA;
+  }
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_cuda_err, sizeof(g_cuda_err), "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return TSP_ERR_CUDA;
+  }
+  return TSP_OK;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// ---------------------------------------------------------------- sizes
+struct Sizes {
+  int64_t T, c, L;
+  int h, H, d, F, D, hs, Fs;
+};
+
+Sizes sizes_of(const tsp_dims* dims, int D) {
+  Sizes s;
+  s.T = dims->T;
+  s.D = D;
+  s.c = dims->T / (2 * D);
+  s.L = 2 * s.c;
+  s.h = dims->h;
+  s.H = dims->n_heads;
+  s.d = dims->head_dim;
+  s.F = dims->ffn;
+  s.hs = dims->h / D;
+  s.Fs = dims->ffn / D;
+  return s;
+}
+
+struct WsLayout {
+  size_t status, xn, q, a, y1, hbuf, counters, total;
+};
+
+WsLayout ws_layout(const Sizes& s) {
+  WsLayout w;
+  size_t o = 0;
+  w.status = o; o += align_up(256);
+  w.counters = o; o += align_up(256);
+  w.xn = o; o += align_up(static_cast<size_t>(s.L) * s.h * 2);
+  w.q = o; o += align_up(static_cast<size_t>(s.L) * s.h * 2);
+  w.a = o; o += align_up(static_cast<size_t>(s.L) * s.h * 2);
+  w.y1 = o; o += align_up(static_cast<size_t>(s.L) * s.h * 4);
+  w.hbuf = o; o += align_up(static_cast<size_t>(s.L) * s.F * 2);
+  w.total = o;
+  return w;
+}
+
+int check_dims(const tsp_dims* dims, int D) {
+  if (!dims) return TSP_ERR_INVALID_ARG;
+  if (D < 1 || D > TSP_MAX_D) return D < 1 ? TSP_ERR_INVALID_ARG : TSP_ERR_UNSUPPORTED;
+  if (dims->T < 0 || dims->h <= 0 || dims->n_heads <= 0 || dims->head_dim <= 0 || dims->ffn <= 0)
+    return TSP_ERR_INVALID_ARG;
+  if (dims->T % (2 * D) != 0) return TSP_ERR_INVALID_ARG;
+  if (dims->n_heads % D != 0 || dims->ffn % D != 0) return TSP_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(dims->n_heads) * dims->head_dim != dims->h) return TSP_ERR_INVALID_ARG;
+  if (!(dims->ln_eps >= 0.f) || !(dims->softmax_scale > 0.f)) return TSP_ERR_INVALID_ARG;
+  if (dims->T >= (int64_t(1) << 31)) return TSP_ERR_UNSUPPORTED;
+  if (dims->head_dim != 64 && dims->head_dim != 128) return TSP_ERR_UNSUPPORTED;
+  if (dims->h % 64 != 0 || dims->h > 4096) return TSP_ERR_UNSUPPORTED;
+  if ((dims->h / D) % 64 != 0 || (dims->ffn / D) % 64 != 0) return TSP_ERR_UNSUPPORTED;
+  return TSP_OK;
+}
+
+int check_weights(const tsp_weights* w, int D) {
+  if (!w || w->D != D) return TSP_ERR_INVALID_ARG;
+  for (int k = 0; k < D; ++k) {
+    const void* ps[6] = {w->wq[k], w->wk[k], w->wv[k], w->wo[k], w->w1[k], w->w2[k]};
+    for (const void* p : ps)
+      if (!p || !aligned16(p)) return TSP_ERR_INVALID_ARG;
+  }
+  return TSP_OK;
+}
+
+// ---------------------------------------------------------------- launches
+template <typename Tin>
+int launch_layernorm(const Tin* x, __nv_bfloat16* y, int64_t rows, int h, float eps, cudaStream_t st) {
+  if (rows == 0) return TSP_OK;
+  const int warps = 8;
+  const dim3 grid(static_cast<unsigned>((rows + warps - 1) / warps));
+  const int nch = h / 8;
+  const int maxc = (nch + 31) / 32;
+  if (maxc <= 1) layernorm_rows_kernel<Tin, 1><<<grid, 256, 0, st>>>(x, y, rows, h, eps);
+  else if (maxc <= 2) layernorm_rows_kernel<Tin, 2><<<grid, 256, 0, st>>>(x, y, rows, h, eps);
+  else if (maxc <= 4) layernorm_rows_kernel<Tin, 4><<<grid, 256, 0, st>>>(x, y, rows, h, eps);
+  else if (maxc <= 8) layernorm_rows_kernel<Tin, 8><<<grid, 256, 0, st>>>(x, y, rows, h, eps);
+  else layernorm_rows_kernel<Tin, 16><<<grid, 256, 0, st>>>(x, y, rows, h, eps);
+  TSP_CUDA(cudaGetLastError());
+  return TSP_OK;
+}
+
+template <int BN>
+int launch_gemm_bn(GemmParams& p, cudaStream_t st) {
+  using S = GemmShape<BN>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(gemm_bf16_tcgen05<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes);
+  });
+  TSP_CUDA(attr_err);
+  const int tiles = ((p.M + kGemmBM - 1) / kGemmBM) * (p.N / BN);
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  gemm_bf16_tcgen05<BN><<<grid, kGemmThreads, S::kSmemBytes, st>>>(p);
+  TSP_CUDA(cudaGetLastError());
+  return TSP_OK;
+}
+
+int pick_bn(int n_block) {
+  if (n_block % 256 == 0) return 256;
+  if (n_block % 128 == 0) return 128;
+  return 64;
+}
+
+int launch_gemm(GemmParams& p, int bn, cudaStream_t st) {
+  if (p.M == 0) return TSP_OK;
+  switch (bn) {
+    case 256: return launch_gemm_bn<256>(p, st);
+    case 128: return launch_gemm_bn<128>(p, st);
+    default: return launch_gemm_bn<64>(p, st);
+  }
+}
+
+void gemm_common(GemmParams& p, const Sizes& s, int rank, int* status) {
+  p.c = static_cast<int>(s.c);
+  p.off0 = static_cast<int64_t>(rank) * s.c;                 // chunk r
+  p.off1 = static_cast<int64_t>(2 * s.D - 1 - rank) * s.c - s.c;  // chunk 2D-1-r
+  p.status = status;
+  p.timeout_ns = kDefaultTimeoutNs;
+}
+
+// N-split projection of xn [L, h] by nseg weight families (each D shards
+// [h/D, h]) into nseg outputs [*, h]; remap[i] sends rows to global rows.
+int launch_proj(const Sizes& s, int rank, const __nv_bfloat16* xn, const void* const* fam[3], void* out[3],
+                const int remap[3], int nseg, int epi, int F_cols, int* status, cudaStream_t st) {
+  static thread_local GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  const int shard_n = F_cols / s.D;
+  int rc = make_map(&p.map_a, xn, s.L, s.h, s.h, kGemmBM);
+  if (rc) return rc;
+  const int bn = pick_bn(shard_n);
+  for (int seg = 0; seg < nseg; ++seg)
+    for (int k = 0; k < s.D; ++k) {
+      rc = make_map(&p.map_b[seg * s.D + k], fam[seg][k], shard_n, s.h, s.h, bn);
+      if (rc) return rc;
+    }
+  p.M = static_cast<int>(s.L);
+  p.N = nseg * F_cols;
+  p.K = s.h;
+  p.ksplit = 0;
+  p.shard_n = shard_n;
+  p.shard_k = s.h;
+  p.seg_n = F_cols;
+  p.epi = epi;
+  for (int i = 0; i < nseg; ++i) {
+    p.out[i] = out[i];
+    p.remap[i] = remap[i];
+  }
+  p.ldo = F_cols;
+  gemm_common(p, s, rank, status);
+  return launch_gemm(p, bn, st);
+}
+
+// K-split: out = resid + sum_k A[:, k-block] W_k^T, W_k [h, Kdim/D].
+int launch_ksplit(const Sizes& s, int rank, const __nv_bfloat16* a, int Kdim, const void* const* fam, const void* resid,
+                  int resid_f32, void* out, int out_f32, int* status, cudaStream_t st) {
+  static thread_local GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  const int shard_k = Kdim / s.D;
+  const int bn = pick_bn(s.h);
+  int rc = make_map(&p.map_a, a, s.L, Kdim, Kdim, kGemmBM);
+  if (rc) return rc;
+  for (int k = 0; k < s.D; ++k) {
+    rc = make_map(&p.map_b[k], fam[k], s.h, shard_k, shard_k, bn);
+    if (rc) return rc;
+  }
+  p.M = static_cast<int>(s.L);
+  p.N = s.h;
+  p.K = Kdim;
+  p.ksplit = 1;
+  p.shard_n = s.h;
+  p.shard_k = shard_k;
+  p.seg_n = s.h;
+  p.epi = kEpiResidual;
+  p.out[0] = out;
+  p.ldo = s.h;
+  p.resid = resid;
+  p.resid_f32 = resid_f32;
+  p.out_f32 = out_f32;
+  gemm_common(p, s, rank, status);
+  return launch_gemm(p, bn, st);
+}
+
+int launch_attention(const Sizes& s, int rank, const tsp_dims* dims, const __nv_bfloat16* q, const void* k_full,
+                     const void* v_full, __nv_bfloat16* out, int* counter, int* status, cudaStream_t st) {
+  if (s.L == 0) return TSP_OK;
+  static thread_local AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  int rc = make_map(&p.map_q, q, s.L, s.h, s.h, kAttnBM);
+  if (rc) return rc;
+  rc = make_map(&p.map_k, k_full, s.T, s.h, s.h, kAttnBN);
+  if (rc) return rc;
+  rc = make_map(&p.map_v, v_full, s.T, s.h, s.h, kAttnBN);
+  if (rc) return rc;
+  p.out = out;
+  p.ldo = s.h;
+  p.c = static_cast<int>(s.c);
+  p.rank = rank;
+  p.D = s.D;
+  p.H = s.H;
+  p.nqt = static_cast<int>((s.c + kAttnBM - 1) / kAttnBM);
+  p.n_items = 2 * p.nqt * s.H;
+  p.scale_log2 = dims->softmax_scale * 1.4426950408889634f;
+  p.counter = counter;
+  p.status = status;
+  p.timeout_ns = kDefaultTimeoutNs;
+  TSP_CUDA(cudaMemsetAsync(counter, 0, sizeof(int), st));
+  const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
+  if (s.d == 128) {
+    static std::once_flag once;
+    static cudaError_t e = cudaSuccess;
+    std::call_once(once, [] {
+      e = cudaFuncSetAttribute(attn_fwd_tcgen05<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               AttnShape<128>::kSmemBytes);
+    });
+    TSP_CUDA(e);
+    attn_fwd_tcgen05<128><<<grid, kAttnThreads, AttnShape<128>::kSmemBytes, st>>>(p);
+  } else {
+    static std::once_flag once;
+    static cudaError_t e = cudaSuccess;
+    std::call_once(once, [] {
+      e = cudaFuncSetAttribute(attn_fwd_tcgen05<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               AttnShape<64>::kSmemBytes);
+    });
+    TSP_CUDA(e);
+    attn_fwd_tcgen05<64><<<grid, kAttnThreads, AttnShape<64>::kSmemBytes, st>>>(p);
+  }
+  TSP_CUDA(cudaGetLastError());
+  return TSP_OK;
+}
+
+struct Ctx {
+  Sizes s;
+  WsLayout lay;
+  uint8_t* ws;
+  int* status;
+  int* counters;
+  __nv_bfloat16 *xn, *q, *a, *hbuf;
+  float* y1;
+};
+
+int make_ctx(Ctx& c, const tsp_dims* dims, const tsp_weights* w, int rank, void* ws, size_t ws_bytes) {
+  int D = w ? w->D : 0;
+  int rc = check_dims(dims, D);
+  if (rc) return rc;
+  rc = check_weights(w, D);
+  if (rc) return rc;
+  if (rank < 0 || rank >= D) return TSP_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return TSP_ERR_INVALID_ARG;
+  c.s = sizes_of(dims, D);
+  c.lay = ws_layout(c.s);
+  if (ws_bytes < c.lay.total) return TSP_ERR_WORKSPACE;
+  c.ws = static_cast<uint8_t*>(ws);
+  c.status = reinterpret_cast<int*>(c.ws + c.lay.status);
+  c.counters = reinterpret_cast<int*>(c.ws + c.lay.counters);
+  c.xn = reinterpret_cast<__nv_bfloat16*>(c.ws + c.lay.xn);
+  c.q = reinterpret_cast<__nv_bfloat16*>(c.ws + c.lay.q);
+  c.a = reinterpret_cast<__nv_bfloat16*>(c.ws + c.lay.a);
+  c.y1 = reinterpret_cast<float*>(c.ws + c.lay.y1);
+  c.hbuf = reinterpret_cast<__nv_bfloat16*>(c.ws + c.lay.hbuf);
+  return TSP_OK;
+}
+
+int record(cudaEvent_t* ev, int i, cudaStream_t st) {
+  if (ev) TSP_CUDA(cudaEventRecord(ev[i], st));
+  return TSP_OK;
+}
+
+// Everything after the projections: attention, O, LN2, W1, W2.
+int layer_tail(Ctx& c, const tsp_dims* dims, const tsp_weights* w, int rank, const void* x_local, const void* k_full,
+               const void* v_full, void* y_local, int y_dtype, cudaStream_t st, cudaEvent_t* ev) {
+  const Sizes& s = c.s;
+  int rc = launch_attention(s, rank, dims, c.q, k_full, v_full, c.a, c.counters, c.status, st);
+  if (rc) return rc;
+  if ((rc = record(ev, 3, st))) return rc;
+  rc = launch_ksplit(s, rank, c.a, s.h, reinterpret_cast<const void* const*>(w->wo), x_local, 0, c.y1, 1, c.status, st);
+  if (rc) return rc;
+  if ((rc = record(ev, 4, st))) return rc;
+  rc = launch_layernorm<float>(c.y1, c.xn, s.L, s.h, dims->ln_eps, st);
+  if (rc) return rc;
+  if ((rc = record(ev, 5, st))) return rc;
+  const void* const* w1fam[3] = {reinterpret_cast<const void* const*>(w->w1), nullptr, nullptr};
+  void* hout[3] = {c.hbuf, nullptr, nullptr};
+  const int noremap[3] = {0, 0, 0};
+  rc = launch_proj(s, rank, c.xn, w1fam, hout, noremap, 1, kEpiGeluBf16, s.F, c.status, st);
+  if (rc) return rc;
+  if ((rc = record(ev, 6, st))) return rc;
+  rc = launch_ksplit(s, rank, c.hbuf, s.F, reinterpret_cast<const void* const*>(w->w2), c.y1, 1, y_local,
+                     y_dtype == TSP_OUT_F32, c.status, st);
+  if (rc) return rc;
+  return record(ev, 7, st);
+}
+
+}  // namespace
+
+// ============================================================================
+// C ABI
+// ============================================================================
+extern "C" {
+
+const char* tsp_status_string(int status) {
+  switch (status) {
+    case TSP_OK: return "ok";
+    case TSP_ERR_INVALID_ARG: return "invalid argument";
+    case TSP_ERR_UNSUPPORTED: return "unsupported shape";
+    case TSP_ERR_CUDA: return "CUDA error";
+    case TSP_ERR_TIMEOUT: return "device wait timed out";
+    case TSP_ERR_WORKSPACE: return "workspace too small";
+    default: return "unknown status";
+  }
+}
+
+const char* tsp_last_cuda_error(void) { return g_cuda_err; }
+
+int tsp_check_dims(const tsp_dims* dims, int D) { return check_dims(dims, D); }
+
+int tsp_zigzag_index(int64_t T, int D, int rank, int32_t* d_idx, cudaStream_t stream) {
+  if (D < 1 || D > TSP_MAX_D || rank < 0 || rank >= D || T < 0 || T % (2 * D) != 0) return TSP_ERR_INVALID_ARG;
+  if (T >= (int64_t(1) << 31)) return TSP_ERR_UNSUPPORTED;
+  const int64_t c = T / (2 * D);
+  if (c == 0) return TSP_OK;
+  if (!d_idx) return TSP_ERR_INVALID_ARG;
+  const int threads = 256;
+  const unsigned blocks = static_cast<unsigned>((2 * c + threads - 1) / threads);
+  zigzag_index_kernel<<<blocks, threads, 0, stream>>>(d_idx, c, D, rank);
+  TSP_CUDA(cudaGetLastError());
+  return TSP_OK;
+}
+
+size_t tsp_shard_buffer_bytes(const tsp_dims* dims, int D) {
+  if (check_dims(dims, D) != TSP_OK) return 0;
+  const size_t h = dims->h, F = dims->ffn;
+  // per shard: 4 attention matrices of h*h/D, 2 FFN matrices of h*F/D
+  return static_cast<size_t>(D) * (4 * align_up(h * (h / D) * 2) + 2 * align_up(h * (F / D) * 2));
+}
+
+int tsp_pack_shards(const tsp_dims* dims, int D, const void* const w_full[6], void* d_buf, size_t buf_bytes,
+                    tsp_weights* out, cudaStream_t stream) {
+  int rc = check_dims(dims, D);
+  if (rc) return rc;
+  if (!w_full || !d_buf || !out) return TSP_ERR_INVALID_ARG;
+  for (int i = 0; i < 6; ++i)
+    if (!w_full[i]) return TSP_ERR_INVALID_ARG;
+  if (buf_bytes < tsp_shard_buffer_bytes(dims, D)) return TSP_ERR_WORKSPACE;
+  const int h = dims->h, F = dims->ffn, hs = h / D, Fs = F / D;
+  std::memset(out, 0, sizeof(*out));
+  out->D = D;
+  uint8_t* p = static_cast<uint8_t*>(d_buf);
+  const dim3 blk(32, 8);
+  auto pack = [&](const void* src, int64_t ld, int64_t row0, int64_t col0, int n_out, int n_in, const void** dst) -> int {
+    *dst = p;
+    const dim3 grid((n_in + 31) / 32, (n_out + 31) / 32);
+    pack_transpose_kernel<<<grid, blk, 0, stream>>>(static_cast<const __nv_bfloat16*>(src), ld, row0, col0,
+                                                    reinterpret_cast<__nv_bfloat16*>(p), n_out, n_in);
+    TSP_CUDA(cudaGetLastError());
+    p += align_up(static_cast<size_t>(n_out) * n_in * 2);
+    return TSP_OK;
+  };
+  for (int k = 0; k < D; ++k) {
+    // column shards (head group / FFN block k of the output features): [n/D, in]
+    if ((rc = pack(w_full[0], h, 0, int64_t(k) * hs, hs, h, &out->wq[k]))) return rc;
+    if ((rc = pack(w_full[1], h, 0, int64_t(k) * hs, hs, h, &out->wk[k]))) return rc;
+    if ((rc = pack(w_full[2], h, 0, int64_t(k) * hs, hs, h, &out->wv[k]))) return rc;
+    // row shards (the same head group / FFN block on the input side): [h, in/D]
+    if ((rc = pack(w_full[3], h, int64_t(k) * hs, 0, h, hs, &out->wo[k]))) return rc;
+    if ((rc = pack(w_full[4], F, 0, int64_t(k) * Fs, Fs, h, &out->w1[k]))) return rc;
+    if ((rc = pack(w_full[5], h, int64_t(k) * Fs, 0, h, Fs, &out->w2[k]))) return rc;
+  }
+  return TSP_OK;
+}
+
+size_t tsp_workspace_bytes(const tsp_dims* dims, int D) {
+  if (check_dims(dims, D) != TSP_OK) return 0;
+  return ws_layout(sizes_of(dims, D)).total;
+}
+
+int tsp_workspace_offsets(const tsp_dims* dims, int D, size_t off[8]) {
+  if (!off) return TSP_ERR_INVALID_ARG;
+  int rc = check_dims(dims, D);
+  if (rc) return rc;
+  const WsLayout w = ws_layout(sizes_of(dims, D));
+  off[0] = w.status; off[1] = w.xn; off[2] = w.q; off[3] = w.a;
+  off[4] = w.y1; off[5] = w.hbuf; off[6] = w.counters; off[7] = w.total;
+  return TSP_OK;
+}
+
+int tsp_reset_device_status(void* ws, cudaStream_t stream) {
+  if (!ws) return TSP_ERR_INVALID_ARG;
+  TSP_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), stream));
+  return TSP_OK;
+}
+
+int tsp_get_device_status(const void* ws, cudaStream_t stream) {
+  if (!ws) return TSP_ERR_INVALID_ARG;
+  int h = 0;
+  TSP_CUDA(cudaMemcpyAsync(&h, ws, sizeof(int), cudaMemcpyDeviceToHost, stream));
+  TSP_CUDA(cudaStreamSynchronize(stream));
+  return h == 0 ? TSP_OK : (h == TSP_ERR_TIMEOUT ? TSP_ERR_TIMEOUT : TSP_ERR_CUDA);
+}
+
+int tsp_kv_project(const tsp_dims* dims, const tsp_weights* w, int rank, const void* x_local, void* k_full,
+                   void* v_full, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  Ctx c;
+  int rc = make_ctx(c, dims, w, rank, ws, ws_bytes);
+  if (rc) return rc;
+  if (c.s.L == 0) return TSP_OK;
+  if (!x_local || !k_full || !v_full || !aligned16(x_local) || !aligned16(k_full) || !aligned16(v_full))
+    return TSP_ERR_INVALID_ARG;
+  rc = launch_layernorm<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x_local), c.xn, c.s.L, c.s.h, dims->ln_eps,
+                                       stream);
+  if (rc) return rc;
+  const void* const* fam[3] = {reinterpret_cast<const void* const*>(w->wk),
+                               reinterpret_cast<const void* const*>(w->wv), nullptr};
+  void* out[3] = {k_full, v_full, nullptr};
+  const int remap[3] = {1, 1, 0};
+  return launch_proj(c.s, rank, c.xn, fam, out, remap, 2, kEpiStoreBf16, c.s.h, c.status, stream);
+}
+
+int tsp_layer_forward(const tsp_dims* dims, const tsp_weights* w, int rank, const void* x_local, const void* k_full,
+                      const void* v_full, void* y_local, int y_dtype, void* ws, size_t ws_bytes, cudaStream_t stream,
+                      cudaEvent_t* step_events) {
+  Ctx c;
+  int rc = make_ctx(c, dims, w, rank, ws, ws_bytes);
+  if (rc) return rc;
+  if (y_dtype != TSP_OUT_BF16 && y_dtype != TSP_OUT_F32) return TSP_ERR_INVALID_ARG;
+  if (c.s.L == 0) return TSP_OK;
+  if (!x_local || !k_full || !v_full || !y_local || !aligned16(x_local) || !aligned16(k_full) ||
+      !aligned16(v_full) || !aligned16(y_local))
+    return TSP_ERR_INVALID_ARG;
+  if ((rc = record(step_events, 0, stream))) return rc;
+  rc = launch_layernorm<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x_local), c.xn, c.s.L, c.s.h, dims->ln_eps,
+                                       stream);
+  if (rc) return rc;
+  if ((rc = record(step_events, 1, stream))) return rc;
+  const void* const* fam[3] = {reinterpret_cast<const void* const*>(w->wq), nullptr, nullptr};
+  void* out[3] = {c.q, nullptr, nullptr};
+  const int remap[3] = {0, 0, 0};
+  rc = launch_proj(c.s, rank, c.xn, fam, out, remap, 1, kEpiStoreBf16, c.s.h, c.status, stream);
+  if (rc) return rc;
+  if ((rc = record(step_events, 2, stream))) return rc;
+  return layer_tail(c, dims, w, rank, x_local, k_full, v_full, y_local, y_dtype, stream, step_events);
+}
+
+int tsp_rank_step(const tsp_dims* dims, const tsp_weights* w, int rank, const void* x_local, void* k_full,
+                  void* v_full, void* y_local, int y_dtype, void* ws, size_t ws_bytes, cudaStream_t stream,
+                  cudaEvent_t* step_events) {
+  Ctx c;
+  int rc = make_ctx(c, dims, w, rank, ws, ws_bytes);
+  if (rc) return rc;
+  if (y_dtype != TSP_OUT_BF16 && y_dtype != TSP_OUT_F32) return TSP_ERR_INVALID_ARG;
+  if (c.s.L == 0) return TSP_OK;
+  if (!x_local || !k_full || !v_full || !y_local || !aligned16(x_local) || !aligned16(k_full) ||
+      !aligned16(v_full) || !aligned16(y_local))
+    return TSP_ERR_INVALID_ARG;
+  if ((rc = record(step_events, 0, stream))) return rc;
+  rc = launch_layernorm<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x_local), c.xn, c.s.L, c.s.h, dims->ln_eps,
+                                       stream);
+  if (rc) return rc;
+  if ((rc = record(step_events, 1, stream))) return rc;
+  const void* const* fam[3] = {reinterpret_cast<const void* const*>(w->wq),
+                               reinterpret_cast<const void* const*>(w->wk),
+                               reinterpret_cast<const void* const*>(w->wv)};
+  void* out[3] = {c.q, k_full, v_full};
+  const int remap[3] = {0, 1, 1};
+  rc = launch_proj(c.s, rank, c.xn, fam, out, remap, 3, kEpiStoreBf16, c.s.h, c.status, stream);
+  if (rc) return rc;
+  if ((rc = record(step_events, 2, stream))) return rc;
+  return layer_tail(c, dims, w, rank, x_local, k_full, v_full, y_local, y_dtype, stream, step_events);
+}
+
+int tsp_rank_step_host(const tsp_dims* dims, const tsp_weights* w, int rank, const void* h_x_local,
+                       void* d_x_staging, void* k_full, void* v_full, void* d_y_staging, void* h_y_local, int y_dtype,
+                       void* ws, size_t ws_bytes, cudaStream_t stream) {
+  Ctx c;
+  int rc = make_ctx(c, dims, w, rank, ws, ws_bytes);
+  if (rc) return rc;
+  if (c.s.L == 0) return TSP_OK;
+  if (!h_x_local || !d_x_staging || !d_y_staging || !h_y_local) return TSP_ERR_INVALID_ARG;
+  const size_t xb = static_cast<size_t>(c.s.L) * c.s.h * 2;
+  const size_t yb = static_cast<size_t>(c.s.L) * c.s.h * (y_dtype == TSP_OUT_F32 ? 4 : 2);
+  TSP_CUDA(cudaMemcpyAsync(d_x_staging, h_x_local, xb, cudaMemcpyHostToDevice, stream));
+  rc = tsp_rank_step(dims, w, rank, d_x_staging, k_full, v_full, d_y_staging, y_dtype, ws, ws_bytes, stream, nullptr);
+  if (rc) return rc;
+  TSP_CUDA(cudaMemcpyAsync(h_y_local, d_y_staging, yb, cudaMemcpyDeviceToHost, stream));
+  return TSP_OK;
+}
+
+int tsp_selftest_wait_timeout(void* ws, uint64_t timeout_ns, cudaStream_t stream) {
+  if (!ws || timeout_ns == 0 || timeout_ns > 2000000000ull) return TSP_ERR_INVALID_ARG;
+  wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(static_cast<int*>(ws), timeout_ns);
+  TSP_CUDA(cudaGetLastError());
+  return TSP_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,210 @@
+/*
+ * tsp.h - C ABI of the TSP (Tensor + Sequence Parallelism) per-rank layer
+ * forward for NVIDIA B200 (sm_100a).
+ *
+ * The method (zubnet.ai news item "Zyphra TSP folds TP+SP onto one GPU
+ * axis", paragraphs 1-2): tensor parallelism (weights split) and sequence
+ * parallelism (tokens split) are folded onto ONE mesh axis of size D.  Each
+ * rank holds 1/D of the weights and 1/D of the tokens.  For attention the
+ * weight shards are broadcast one after another and every rank applies each
+ * shard to its own tokens; K/V are all-gathered under a zigzag sequence
+ * partition.  For the MLP a ring passes the weight shards point to point, so
+ * the MLP output is a sum of shard contributions computed locally and no
+ * all-reduce is needed.
+ *
+ * This library computes what ONE rank computes for one dense decoder layer.
+ * On one GPU the broadcast, ring and all-gather become loops over shard
+ * pointers that already sit in device memory; ranks can be run one after
+ * another.  Layer form: pre-LayerNorm (gamma=1, beta=0, biased variance,
+ * eps inside the square root), multi-head causal attention with as many K/V
+ * heads as Q heads and no positional encoding, GELU (tanh form), no biases:
+ *
+ *     Y1 = X + Attn(LN1(X)) Wo,       Y = Y1 + GELU(LN2(Y1) W1) W2.
+ *
+ * Conventions shared by every call
+ *   - All matrices are row-major.  "K-major [n, k]" means n rows of k
+ *     contiguous elements (the layout of a Linear layer's weight).
+ *   - Tokens: the T-token sequence is cut into 2D chunks of c = T/(2D)
+ *     tokens; rank r holds chunk r then chunk 2D-1-r.  "Rank-local order"
+ *     is that order: local row i < c is global position r*c + i, local row
+ *     i >= c is global position (2D-1-r)*c + (i-c).  L = 2c local tokens.
+ *   - Shard k of the attention weights is head group k (heads
+ *     k*H/D .. (k+1)*H/D-1, i.e. hidden columns k*h/D .. (k+1)*h/D-1); shard
+ *     k of the FFN is FFN columns k*F/D .. (k+1)*F/D-1.
+ *   - K/V full-sequence tensors are [T, h] bf16 in natural (global) order,
+ *     head j in columns j*d .. (j+1)*d-1.
+ *   - Every device buffer is allocated and freed by the caller.  Functions
+ *     that take a stream only enqueue work on it (asynchronous) unless
+ *     stated otherwise; the library allocates no device memory and keeps no
+ *     state between calls.
+ *   - Host-detectable errors are returned synchronously and nothing is
+ *     enqueued.  There is no fallback path: an unsupported shape is an
+ *     error.  Device-side timeouts (a bounded wait inside a kernel that ran
+ *     out) are recorded in the workspace status word and reported by
+ *     tsp_get_device_status.
+ */
+#ifndef TSP_H_
+#define TSP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TSP_MAX_D 16
+#define TSP_N_STEP_EVENTS 8
+
+typedef enum {
+  TSP_OK = 0,
+  TSP_ERR_INVALID_ARG = 1, /* null pointer, rank out of range, T % 2D != 0, H % D, F % D, ... */
+  TSP_ERR_UNSUPPORTED = 2, /* a shape the kernels do not implement (see tsp_check_dims) */
+  TSP_ERR_CUDA = 3,        /* a CUDA runtime call failed; see tsp_last_cuda_error */
+  TSP_ERR_TIMEOUT = 4,     /* a bounded wait inside a kernel ran out */
+  TSP_ERR_WORKSPACE = 5    /* workspace or buffer smaller than required */
+} tsp_status;
+
+/* Layer and sequence sizes. */
+typedef struct {
+  int64_t T;           /* sequence length (global tokens); T % (2D) == 0 */
+  int32_t h;           /* hidden size; h == n_heads * head_dim */
+  int32_t n_heads;     /* H: attention heads (Q and K/V) */
+  int32_t head_dim;    /* d: 64 or 128 */
+  int32_t ffn;         /* F: FFN width */
+  float ln_eps;        /* LayerNorm epsilon (1e-5 for the 7B layer) */
+  float softmax_scale; /* applied to q.k; 1/sqrt(d) for the 7B layer */
+} tsp_dims;
+
+/* Per-shard device pointers (bf16), each shard one contiguous K-major
+ * buffer:  wq/wk/wv[k] [h/D, h],  wo[k] [h, h/D],  w1[k] [F/D, h],
+ * w2[k] [h, F/D].  Only entries 0..D-1 are read.  Pointers must be 16-byte
+ * aligned. */
+typedef struct {
+  int32_t D;
+  const void* wq[TSP_MAX_D];
+  const void* wk[TSP_MAX_D];
+  const void* wv[TSP_MAX_D];
+  const void* wo[TSP_MAX_D];
+  const void* w1[TSP_MAX_D];
+  const void* w2[TSP_MAX_D];
+} tsp_weights;
+
+/* Output dtypes of tsp_layer_forward. */
+#define TSP_OUT_BF16 0
+#define TSP_OUT_F32 1
+
+/* Short English text for a status code (static storage). */
+const char* tsp_status_string(int status);
+
+/* Text of the last CUDA error seen by this thread (static per-thread storage). */
+const char* tsp_last_cuda_error(void);
+
+/* Checks sizes against what the kernels implement; returns TSP_OK,
+ * TSP_ERR_INVALID_ARG or TSP_ERR_UNSUPPORTED.  Supported: head_dim 64 or
+ * 128, h % 64 == 0, h/D % 64 == 0, F/D % 64 == 0, H % D == 0, F % D == 0,
+ * 1 <= D <= TSP_MAX_D, T % (2D) == 0, T < 2^31.  Pure host function. */
+int tsp_check_dims(const tsp_dims* dims, int D);
+
+/* Zigzag index map [zubnet.ai TSP item, paragraph 2: "zigzag partition"]:
+ * d_idx[i] = global position of rank `rank`'s local token i, for
+ * i in [0, T/D).  d_idx: device int32 [T/D].  Bit-exact integer result. */
+int tsp_zigzag_index(int64_t T, int D, int rank, int32_t* d_idx, cudaStream_t stream);
+
+/* Bytes of one packed shard buffer for all six weights at this D. */
+size_t tsp_shard_buffer_bytes(const tsp_dims* dims, int D);
+
+/* Splits full weights into per-rank shards [zubnet.ai TSP item, paragraph 1:
+ * "each GPU holds 1/D of the weights"].  w_full[6] = {Wq, Wk, Wv, Wo, W1, W2}
+ * are device bf16 in the math orientation y = x W ([in, out]: Wq/Wk/Wv/Wo
+ * [h, h], W1 [h, F], W2 [F, h]).  Writes the K-major shards into d_buf
+ * (tsp_shard_buffer_bytes bytes, caller-owned) and fills *out with
+ * pointers into d_buf. */
+int tsp_pack_shards(const tsp_dims* dims, int D, const void* const w_full[6],
+                    void* d_buf, size_t buf_bytes, tsp_weights* out, cudaStream_t stream);
+
+/* Workspace bytes that tsp_kv_project / tsp_layer_forward / tsp_rank_step
+ * need for one rank at this D (activations of L = T/D tokens plus a status
+ * word).  The workspace is caller-owned device memory, 256-byte aligned. */
+size_t tsp_workspace_bytes(const tsp_dims* dims, int D);
+
+/* Byte offsets inside the workspace of the per-rank intermediates, for
+ * inspection after a call (all rank-local order, row-major):
+ *   off[0] status word (int32),  off[1] LN output xn bf16 [L, h] (LN2's
+ *   output after tsp_layer_forward),  off[2] Q bf16 [L, h],  off[3]
+ *   attention output bf16 [L, h],  off[4] Y1 = X + attention projection,
+ *   fp32 [L, h],  off[5] H = GELU(LN2(Y1) W1) bf16 [L, F],  off[6]
+ *   scheduler counters,  off[7] total bytes.  Returns TSP_OK or
+ *   TSP_ERR_INVALID_ARG. */
+int tsp_workspace_offsets(const tsp_dims* dims, int D, size_t off[8]);
+
+/* Clears the workspace status word (enqueued on `stream`). */
+int tsp_reset_device_status(void* ws, cudaStream_t stream);
+
+/* Synchronises `stream`, then reads the workspace status word: TSP_OK or
+ * TSP_ERR_TIMEOUT (sticky until tsp_reset_device_status). */
+int tsp_get_device_status(const void* ws, cudaStream_t stream);
+
+/* K/V projection of one rank's tokens [zubnet.ai TSP item, paragraph 2:
+ * every rank applies each weight shard to its own tokens; K/V are then
+ * all-gathered with the zigzag partition]:
+ *     K[pos(i)] = LN1(x_local[i]) Wk,   V[pos(i)] = LN1(x_local[i]) Wv
+ * for all D shards (head groups), written at the tokens' GLOBAL rows of
+ * k_full / v_full ([T, h] bf16) - the place the all-gather puts them.
+ * x_local: bf16 [T/D, h] rank-local order.  With D=1, rank 0 this projects
+ * a whole natural-order sequence.  ws: tsp_workspace_bytes(dims, D). */
+int tsp_kv_project(const tsp_dims* dims, const tsp_weights* w, int rank,
+                   const void* x_local, void* k_full, void* v_full,
+                   void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* The rank's layer forward given the all-gathered K/V [zubnet.ai TSP item,
+ * paragraphs 1-2, 4]:
+ *   Xn = LN1(x_local);  for each shard k: Q_k = Xn Wq_k^T,
+ *   A_k = causal softmax(scale Q_k K_k^T) V_k  (query at global position p
+ *   sees keys 0..p),  Y1 = x_local + sum_k A_k Wo_k^T;
+ *   Y = Y1 + sum_k GELU(LN2(Y1) W1_k^T) W2_k^T  (the shard sum is local:
+ *   no all-reduce).
+ * x_local bf16 [T/D, h] rank-local order; k_full, v_full bf16 [T, h]
+ * natural order (read only); y_local [T/D, h] rank-local order, bf16
+ * (y_dtype TSP_OUT_BF16) or fp32 (TSP_OUT_F32); the bf16 result is the
+ * fp32 result rounded to nearest even.  step_events: NULL, or
+ * TSP_N_STEP_EVENTS caller-created events recorded on `stream` after the
+ * launches of LN1, Q, attention, O, LN2, W1, W2 (event 0 before LN1). */
+int tsp_layer_forward(const tsp_dims* dims, const tsp_weights* w, int rank,
+                      const void* x_local, const void* k_full, const void* v_full,
+                      void* y_local, int y_dtype, void* ws, size_t ws_bytes,
+                      cudaStream_t stream, cudaEvent_t* step_events);
+
+/* One whole TSP rank step: tsp_kv_project of the rank's own tokens followed
+ * by tsp_layer_forward, with LN1 computed once and the Q, K and V
+ * projections done in one launch.  k_full / v_full are read-write: the
+ * rank's own rows are written, the other ranks' rows must already be there.
+ * step_events as in tsp_layer_forward (the Q launch also projects K/V). */
+int tsp_rank_step(const tsp_dims* dims, const tsp_weights* w, int rank,
+                  const void* x_local, void* k_full, void* v_full,
+                  void* y_local, int y_dtype, void* ws, size_t ws_bytes,
+                  cudaStream_t stream, cudaEvent_t* step_events);
+
+/* tsp_rank_step with the token buffers in HOST memory: copies h_x_local
+ * ([T/D, h] bf16) to `d_x_staging` (device, T/D*h*2 bytes, caller-owned),
+ * runs the step, copies the result back to h_y_local, all enqueued on
+ * `stream`.  Pinned host memory makes the copies asynchronous. */
+int tsp_rank_step_host(const tsp_dims* dims, const tsp_weights* w, int rank,
+                       const void* h_x_local, void* d_x_staging,
+                       void* k_full, void* v_full, void* d_y_staging,
+                       void* h_y_local, int y_dtype, void* ws, size_t ws_bytes,
+                       cudaStream_t stream);
+
+/* Fault-detection self test: launches one block that waits on a barrier
+ * nothing will ever complete, with a limit of `timeout_ns` nanoseconds
+ * (at most 2e9).  The wait gives up, the kernel records TSP_ERR_TIMEOUT in
+ * the workspace status word and returns normally, so the context stays
+ * usable.  ws: at least 256 bytes. */
+int tsp_selftest_wait_timeout(void* ws, uint64_t timeout_ns, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TSP_H_ */

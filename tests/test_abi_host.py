@@ -1,0 +1,138 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports every
+function include/tsp.h declares, and rejects bad arguments before touching
+the device.  No compute call is made here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from folded_tensor_sequence_rank_b200 import build as tsp_build
+from folded_tensor_sequence_rank_b200 import tsp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tsp.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    tsp_build.build()
+    return tsp.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(tsp_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("tsp_zigzag_index", "tsp_kv_project", "tsp_layer_forward", "tsp_rank_step",
+                     "tsp_pack_shards", "tsp_workspace_bytes", "tsp_get_device_status"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_struct_layouts_match_header():
+    # tsp_dims: int64 + 4 x int32 + 2 x float; tsp_weights: int32 D + 6 x 16 pointers
+    assert ctypes.sizeof(tsp.Dims) == 32
+    assert ctypes.sizeof(tsp.Weights) == 8 + 6 * 16 * 8
+
+
+def test_status_strings(L):
+    for code in range(6):
+        assert L.tsp_status_string(code).decode() == tsp.STATUS[code]
+
+
+def dims(T=512, h=256, H=4, F=1024):
+    return tsp.make_dims(T, h, H, F)
+
+
+@pytest.mark.parametrize("kw,D,expect", [
+    (dict(), 2, tsp.TSP_OK),
+    (dict(T=0), 2, tsp.TSP_OK),
+    (dict(T=800), 2, tsp.TSP_OK),             # ragged chunk (c = 200)
+    (dict(T=131072, h=4096, H=32, F=16384), 8, tsp.TSP_OK),
+    (dict(T=32768, h=4096, H=32, F=16384), 16, tsp.TSP_OK),
+    (dict(T=510), 2, tsp.TSP_ERR_INVALID_ARG),   # T % 2D
+    (dict(), 3, tsp.TSP_ERR_INVALID_ARG),        # H % D
+    (dict(), 0, tsp.TSP_ERR_INVALID_ARG),
+    (dict(), 32, tsp.TSP_ERR_UNSUPPORTED),       # D > TSP_MAX_D
+    (dict(h=384, H=4), 2, tsp.TSP_ERR_UNSUPPORTED),   # head_dim 96
+    (dict(T=768, h=192, H=3, F=768), 3, tsp.TSP_OK),       # D = 3: h/D = 64, F/D = 256
+    (dict(T=768, h=192, H=3, F=768), 2, tsp.TSP_ERR_INVALID_ARG),  # H % D
+    (dict(h=256, H=4, F=1024), 4, tsp.TSP_OK),   # h/D = 64
+    (dict(h=256, H=4, F=96), 2, tsp.TSP_ERR_UNSUPPORTED),  # F/D = 48
+])
+def test_check_dims(L, kw, D, expect):
+    d = dims(**kw)
+    assert tsp.check_dims(d, D) == expect
+
+
+def test_workspace_sizes_and_offsets(L):
+    d = dims(T=131072, h=4096, H=32, F=16384)
+    off = tsp.workspace_offsets(d, 8)
+    assert off[7] == tsp.workspace_bytes(d, 8)
+    L_tok = 131072 // 8
+    assert off[5] + L_tok * 16384 * 2 <= off[7]
+    assert all(o % 1024 == 0 for o in off)
+    # shard buffer: all six weights once
+    assert tsp.shard_buffer_bytes(d, 8) == 2 * (4 * 4096 * 4096 + 2 * 4096 * 16384)
+
+
+def test_bad_arguments_fail_before_any_device_work(L):
+    d = dims()
+    w = tsp.Weights()
+    w.D = 2
+    # null weight pointers
+    rc = L.tsp_layer_forward(ctypes.byref(d), ctypes.byref(w), 0, None, None, None, None, 0, None, 0, None, None)
+    assert rc == tsp.TSP_ERR_INVALID_ARG
+    for name in tsp.WEIGHT_NAMES:
+        arr = getattr(w, name)
+        for k in range(2):
+            arr[k] = 0x10000 * (k + 1)
+    # rank out of range
+    rc = L.tsp_layer_forward(ctypes.byref(d), ctypes.byref(w), 2, 16, 16, 16, 16, 0, 256, 1 << 30, None, None)
+    assert rc == tsp.TSP_ERR_INVALID_ARG
+    # workspace too small
+    rc = L.tsp_layer_forward(ctypes.byref(d), ctypes.byref(w), 0, 16, 16, 16, 16, 0, 256, 1024, None, None)
+    assert rc == tsp.TSP_ERR_WORKSPACE
+    # misaligned workspace
+    rc = L.tsp_kv_project(ctypes.byref(d), ctypes.byref(w), 0, 16, 16, 16, 257, 1 << 30, None)
+    assert rc == tsp.TSP_ERR_INVALID_ARG
+    # bad output dtype
+    rc = L.tsp_rank_step(ctypes.byref(d), ctypes.byref(w), 0, 16, 16, 16, 16, 7, 256, 1 << 30, None, None)
+    assert rc == tsp.TSP_ERR_INVALID_ARG
+    # zigzag argument checks
+    assert L.tsp_zigzag_index(510, 2, 0, None, None) == tsp.TSP_ERR_INVALID_ARG
+    assert L.tsp_zigzag_index(512, 2, 2, None, None) == tsp.TSP_ERR_INVALID_ARG
+    assert L.tsp_zigzag_index(0, 2, 0, None, None) == tsp.TSP_OK
+    # self-test limits
+    assert L.tsp_selftest_wait_timeout(None, 1000, None) == tsp.TSP_ERR_INVALID_ARG
+    assert L.tsp_selftest_wait_timeout(256, 3 * 10 ** 9, None) == tsp.TSP_ERR_INVALID_ARG
+
+
+def test_empty_sequence_is_a_no_op(L):
+    d = dims(T=0)
+    w = tsp.Weights()
+    w.D = 2
+    for name in tsp.WEIGHT_NAMES:
+        arr = getattr(w, name)
+        for k in range(2):
+            arr[k] = 0x10000 * (k + 1)
+    ws = tsp.workspace_bytes(d, 2)
+    assert ws > 0
+    rc = L.tsp_layer_forward(ctypes.byref(d), ctypes.byref(w), 1, None, None, None, None, 0, 1024, ws, None, None)
+    assert rc == tsp.TSP_OK
+
+
+def test_binding_refuses_cpu_tensors(L):
+    import torch
+    d = dims()
+    with pytest.raises(ValueError):
+        tsp.pack_shards(d, 2, {n: torch.zeros(1, dtype=torch.bfloat16) for n in tsp.WEIGHT_NAMES})

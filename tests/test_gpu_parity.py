@@ -1,0 +1,308 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Gates (the layer's stated tolerance for bf16 layer outputs): max-abs <= 2e-2
+and relative-L2 <= 5e-3 on the layer output, computed in fp32 by the kernels
+(y_dtype fp32); the bf16 output equals the fp32 output rounded to nearest
+even bit for bit.  The zigzag index map and the weight shard packing are
+integer / byte work and must match exactly.  Intermediates get looser
+diagnostic gates that catch errors the residual stream would hide.
+
+Sizes: the tiny layer (h=256, 4 heads of 64, FFN 1024, T=512, D=2) and
+variants (D=1, D=4, ragged chunks) are compared in full; the 7B layer at
+T=8192 (D=8) in full for a rank; at T=131072 (D=8) and T=32768 (D=1..16) on
+sampled rows the oracle computes one by one, in the launch configuration the
+benchmark uses.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from folded_tensor_sequence_rank_b200 import build as tsp_build
+from folded_tensor_sequence_rank_b200 import inputs
+from folded_tensor_sequence_rank_b200 import tsp
+from oracle import tsp_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS, REL_L2 = 2e-2, 5e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    tsp_build.build()
+    tsp.lib()
+    torch.cuda.init()
+
+
+def f64(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def rel_l2(a, b):
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+
+
+def assert_layer_close(y_gpu, y_ref, what, x=None):
+    err = float(np.max(np.abs(y_gpu - y_ref)))
+    rl = rel_l2(y_gpu, y_ref)
+    assert np.isfinite(y_gpu).all(), what
+    assert err <= MAX_ABS and rl <= REL_L2, f"{what}: max-abs {err:.3e}, rel-L2 {rl:.3e}"
+    if x is not None:  # the layer's own contribution, without the residual
+        rd = rel_l2(y_gpu - x, y_ref - x)
+        assert rd <= 2e-2, f"{what}: rel-L2 of (Y - X) {rd:.3e}"
+
+
+def to_cuda(d):
+    return {k: v.cuda() for k, v in d.items()}
+
+
+def weights_f64(raw):
+    return {n: f64(raw[n]) for n in inputs.WEIGHT_NAMES}
+
+
+# --------------------------------------------------------------------------
+def test_zigzag_bit_exact():
+    for T, D in [(512, 2), (8192, 8), (131072, 8), (32768, 16), (100, 2), (8, 1), (768, 3)]:
+        for r in sorted({0, D // 2, D - 1}):
+            got = tsp.zigzag_index(T, D, r).cpu().numpy()
+            assert np.array_equal(got.astype(np.int64), O.zigzag_index(T, D, r)), (T, D, r)
+
+
+def test_pack_shards_exact():
+    T, h, H, F, D = 512, 256, 4, 1024, 4
+    raw = to_cuda(inputs.layer_inputs(T, h, F, 3))
+    dims = tsp.make_dims(T, h, H, F)
+    sw = tsp.pack_shards(dims, D, raw)
+    torch.cuda.synchronize()
+    hs, Fs = h // D, F // D
+    for k in range(D):
+        cols, fcols = slice(k * hs, (k + 1) * hs), slice(k * Fs, (k + 1) * Fs)
+        expect = {"wq": raw["wq"][:, cols].t(), "wk": raw["wk"][:, cols].t(), "wv": raw["wv"][:, cols].t(),
+                  "wo": raw["wo"][cols, :].t(), "w1": raw["w1"][:, fcols].t(), "w2": raw["w2"][fcols, :].t()}
+        for n, e in expect.items():
+            got = sw.shard(n, k, tuple(e.shape))
+            assert torch.equal(got.view(torch.int16), e.contiguous().view(torch.int16)), (n, k)
+
+
+# --------------------------------------------------------------------------
+def run_full_sequence(T, h, H, F, D, seed, y_dtype=torch.float32):
+    """All D ranks on one GPU: every rank projects its K/V, then every rank runs
+    its layer forward.  Returns the outputs scattered to natural order."""
+    raw = inputs.layer_inputs(T, h, F, seed)
+    dev = to_cuda(raw)
+    dims = tsp.make_dims(T, h, H, F)
+    sw = tsp.pack_shards(dims, D, dev)
+    ws = tsp.alloc_workspace(dims, D)
+    K = torch.zeros(T, h, dtype=torch.bfloat16, device="cuda")
+    V = torch.zeros_like(K)
+    idx = [tsp.zigzag_index(T, D, r).long() for r in range(D)]
+    x_loc = [dev["x"].index_select(0, i).contiguous() for i in idx]
+    for r in range(D):
+        tsp.kv_project(dims, sw, r, x_loc[r], K, V, ws)
+    Y = torch.zeros(T, h, dtype=y_dtype, device="cuda")
+    inter = []
+    for r in range(D):
+        y = torch.empty(T // D, h, dtype=y_dtype, device="cuda")
+        tsp.layer_forward(dims, sw, r, x_loc[r], K, V, y, ws)
+        Y[idx[r]] = y
+        inter.append({n: tsp.workspace_view(ws, dims, D, n).clone() for n in ("q", "a", "y1", "h", "xn")})
+    assert tsp.get_device_status(ws) == tsp.TSP_OK
+    torch.cuda.synchronize()
+    return raw, K, V, Y, idx, inter
+
+
+@pytest.mark.parametrize("T,h,H,F,D,seed", [
+    (512, 256, 4, 1024, 2, 0),     # the tiny TSP layer
+    (512, 256, 4, 1024, 1, 5),     # D = 1: plain layer
+    (1024, 256, 4, 1024, 4, 6),    # h/D = 64, F/D = 256
+    (800, 256, 4, 1024, 2, 7),     # ragged chunks: c = 200
+    (288, 256, 2, 512, 2, 8),      # head_dim 128, c = 72 (< one tile)
+    (2048, 512, 4, 2048, 2, 9),    # head_dim 128, several tiles per chunk
+])
+def test_full_sequence_all_ranks(T, h, H, F, D, seed):
+    raw, K, V, Y, idx, inter = run_full_sequence(T, h, H, F, D, seed)
+    x = f64(raw["x"])
+    ref = O.layer_forward(x, weights_f64(raw), H)
+    # K/V: bf16 results; allow a rounding flip of one bf16 unit
+    for name, got in (("k", K), ("v", V)):
+        g, e = f64(got), ref[name]
+        assert np.all(np.abs(g - e) <= 2.0 ** -7 * np.abs(e) + 1e-6), name
+    for r in range(D):
+        rows = idx[r].cpu().numpy()
+        for n, gate in (("q", 1e-2), ("a", 1e-2), ("y1", 1e-3), ("h", 2e-2)):
+            rl = rel_l2(f64(inter[r][n]), ref[n if n != "xn" else "xn2"][rows])
+            assert rl <= gate, (r, n, rl)
+    assert_layer_close(f64(Y), ref["y"], f"T={T} D={D}", x)
+
+
+def test_bf16_output_is_rounded_fp32_output():
+    T, h, H, F, D = 1024, 256, 4, 1024, 2
+    raw = to_cuda(inputs.layer_inputs(T, h, F, 11))
+    dims = tsp.make_dims(T, h, H, F)
+    sw = tsp.pack_shards(dims, D, raw)
+    ws = tsp.alloc_workspace(dims, D)
+    K = torch.zeros(T, h, dtype=torch.bfloat16, device="cuda")
+    V = torch.zeros_like(K)
+    for r in range(D):
+        xl = raw["x"].index_select(0, tsp.zigzag_index(T, D, r).long()).contiguous()
+        tsp.kv_project(dims, sw, r, xl, K, V, ws)
+    xl = raw["x"].index_select(0, tsp.zigzag_index(T, D, 1).long()).contiguous()
+    y32 = torch.empty(T // D, h, dtype=torch.float32, device="cuda")
+    y16 = torch.empty(T // D, h, dtype=torch.bfloat16, device="cuda")
+    tsp.layer_forward(dims, sw, 1, xl, K, V, y32, ws)
+    tsp.layer_forward(dims, sw, 1, xl, K, V, y16, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y32.to(torch.bfloat16).view(torch.int16), y16.view(torch.int16))
+
+
+def test_rank_step_equals_projection_then_layer():
+    T, h, H, F, D = 2048, 512, 4, 2048, 4
+    raw = to_cuda(inputs.layer_inputs(T, h, F, 12))
+    dims = tsp.make_dims(T, h, H, F)
+    sw = tsp.pack_shards(dims, D, raw)
+    ws = tsp.alloc_workspace(dims, D)
+    K = torch.zeros(T, h, dtype=torch.bfloat16, device="cuda")
+    V = torch.zeros_like(K)
+    xs = [raw["x"].index_select(0, tsp.zigzag_index(T, D, r).long()).contiguous() for r in range(D)]
+    for r in range(D):
+        tsp.kv_project(dims, sw, r, xs[r], K, V, ws)
+    K2, V2 = K.clone(), V.clone()
+    r = 2
+    ya = torch.empty(T // D, h, dtype=torch.float32, device="cuda")
+    tsp.layer_forward(dims, sw, r, xs[r], K, V, ya, ws)
+    # wipe the rank's own rows: rank_step must write them again
+    for i in tsp.zigzag_index(T, D, r).long().cpu().tolist()[:: max(1, T // D // 8)]:
+        K2[i].zero_()
+        V2[i].zero_()
+    yb = torch.empty_like(ya)
+    tsp.rank_step(dims, sw, r, xs[r], K2, V2, yb, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(K, K2) and torch.equal(V, V2)
+    assert torch.equal(ya, yb)
+
+
+def test_rank_step_host_buffers():
+    T, h, H, F, D = 1024, 256, 4, 1024, 2
+    raw = to_cuda(inputs.layer_inputs(T, h, F, 13))
+    dims = tsp.make_dims(T, h, H, F)
+    sw = tsp.pack_shards(dims, D, raw)
+    ws = tsp.alloc_workspace(dims, D)
+    K = torch.zeros(T, h, dtype=torch.bfloat16, device="cuda")
+    V = torch.zeros_like(K)
+    xs = [raw["x"].index_select(0, tsp.zigzag_index(T, D, r).long()).contiguous() for r in range(D)]
+    for r in range(D):
+        tsp.kv_project(dims, sw, r, xs[r], K, V, ws)
+    yd = torch.empty(T // D, h, dtype=torch.float32, device="cuda")
+    tsp.rank_step(dims, sw, 0, xs[0], K, V, yd, ws)
+    hx = xs[0].cpu().pin_memory()
+    hy = torch.empty(T // D, h, dtype=torch.float32).pin_memory()
+    xst = torch.empty_like(xs[0])
+    yst = torch.empty_like(yd)
+    tsp.rank_step_host(dims, sw, 0, hx, xst, K, V, yst, hy, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(hy, yd.cpu())
+
+
+# --------------------------------------------------------------------------
+# the 7B layer
+# --------------------------------------------------------------------------
+H7, h7, F7 = 32, 4096, 16384
+
+
+def test_7b_layer_T8192_rank_in_full():
+    T, D = 8192, 8
+    raw = inputs.layer_inputs(T, h7, F7, 1)
+    dev = to_cuda(raw)
+    dims = tsp.make_dims(T, h7, H7, F7)
+    sw = tsp.pack_shards(dims, D, dev)
+    ws = tsp.alloc_workspace(dims, D)
+    K = torch.zeros(T, h7, dtype=torch.bfloat16, device="cuda")
+    V = torch.zeros_like(K)
+    xs = [dev["x"].index_select(0, tsp.zigzag_index(T, D, r).long()).contiguous() for r in range(D)]
+    for r in range(D):
+        tsp.kv_project(dims, sw, r, xs[r], K, V, ws)
+    ys = {}
+    for r in (0, 5):
+        y = torch.empty(T // D, h7, dtype=torch.float32, device="cuda")
+        tsp.layer_forward(dims, sw, r, xs[r], K, V, y, ws)
+        ys[r] = y.cpu()
+    assert tsp.get_device_status(ws) == tsp.TSP_OK
+    x = f64(raw["x"])
+    w = weights_f64(raw)
+    Kr, Vr = O.kv_project(x, w)
+    assert np.all(np.abs(f64(K) - Kr) <= 2.0 ** -7 * np.abs(Kr) + 1e-6)
+    for r, y in ys.items():
+        idx = O.zigzag_index(T, D, r)
+        ref = O.rank_rows_forward(x[idx], idx, Kr, Vr, w, H7)
+        assert_layer_close(f64(y), ref["y"], f"7B T=8192 rank {r}", x[idx])
+
+
+def sampled_rank_check(T, D, rank, seed, n_sample=62):
+    """Full-size launch (as benchmarked) of one rank, checked on sampled rows."""
+    L = T // D
+    c = L // 2
+    raw = inputs.rank_inputs(L, T, h7, F7, seed)
+    dev = to_cuda(raw)
+    dims = tsp.make_dims(T, h7, H7, F7)
+    sw = tsp.pack_shards(dims, D, dev)
+    ws = tsp.alloc_workspace(dims, D)
+    y = torch.empty(L, h7, dtype=torch.float32, device="cuda")
+    tsp.layer_forward(dims, sw, rank, dev["x_local"], dev["k_full"], dev["v_full"], y, ws)
+    # the rank's own K/V projection, into scratch copies
+    Kp = torch.zeros(T, h7, dtype=torch.bfloat16, device="cuda")
+    Vp = torch.zeros_like(Kp)
+    tsp.kv_project(dims, sw, rank, dev["x_local"], Kp, Vp, ws)
+    assert tsp.get_device_status(ws) == tsp.TSP_OK
+    rows = inputs.sample_rows(L, n_sample, seed, must=(0, c - 1, c, L - 1))
+    pos = O.zigzag_index(T, D, rank)
+    x = f64(raw["x_local"])
+    w = weights_f64(raw)
+    Kf = raw["k_full"].float().numpy()
+    Vf = raw["v_full"].float().numpy()
+    ref = O.rank_rows_forward(x[rows], pos[rows], Kf, Vf, w, H7)
+    y_s = f64(y[rows])
+    assert_layer_close(y_s, ref["y"], f"7B T={T} D={D} rank {rank}", x[rows])
+    kr, vr = O.kv_project(x[rows], w)
+    gk, gv = f64(Kp[torch.as_tensor(pos[rows])]), f64(Vp[torch.as_tensor(pos[rows])])
+    assert np.all(np.abs(gk - kr) <= 2.0 ** -7 * np.abs(kr) + 1e-6)
+    assert np.all(np.abs(gv - vr) <= 2.0 ** -7 * np.abs(vr) + 1e-6)
+
+
+def test_7b_layer_128k_rank0_sampled():
+    sampled_rank_check(131072, 8, 0, 2)
+
+
+def test_7b_layer_128k_last_rank_sampled():
+    sampled_rank_check(131072, 8, 7, 3, n_sample=30)
+
+
+@pytest.mark.parametrize("D", [1, 2, 4, 8, 16])
+def test_7b_layer_T32768_shard_sweep_sampled(D):
+    sampled_rank_check(32768, D, 0, 4, n_sample=30)
+
+
+# --------------------------------------------------------------------------
+# failure detection without a GPU fault
+# --------------------------------------------------------------------------
+def test_bounded_wait_times_out_and_context_survives():
+    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    assert tsp.get_device_status(ws) == tsp.TSP_OK
+    tsp.selftest_wait_timeout(ws, 20_000_000)  # 20 ms
+    assert tsp.get_device_status(ws) == tsp.TSP_ERR_TIMEOUT
+    tsp.reset_device_status(ws)
+    assert tsp.get_device_status(ws) == tsp.TSP_OK
+    # the context still runs real work
+    got = tsp.zigzag_index(512, 2, 1).cpu().numpy()
+    assert np.array_equal(got.astype(np.int64), O.zigzag_index(512, 2, 1))
+
+
+def test_empty_sequence():
+    dims = tsp.make_dims(0, 256, 4, 1024)
+    raw = to_cuda(inputs.layer_inputs(4, 256, 1024, 0))
+    sw = tsp.pack_shards(tsp.make_dims(4, 256, 4, 1024), 2, raw)
+    ws = tsp.alloc_workspace(dims, 2)
+    e = torch.empty(0, 256, dtype=torch.bfloat16, device="cuda")
+    tsp.layer_forward(dims, sw, 0, e, e, e, torch.empty(0, 256, device="cuda"), ws)
+    torch.cuda.synchronize()
