@@ -231,16 +231,16 @@ def run_tsp(args, wl):
     # synthetic inputs, drawn on the device (parity is the tests' job)
     g = torch.Generator(device="cuda")
     g.manual_seed(wl["seed"] * 1000 + grank)
-    def rnd(*shape, std=1.0):
-        return (torch.randn(*shape, generator=g, device="cuda", dtype=torch.float32) * std).to(torch.bfloat16)
+    def rnd(*shape, std=1.0, dtype=torch.bfloat16):
+        return (torch.randn(*shape, generator=g, device="cuda", dtype=torch.float32) * std).to(dtype)
     w_full = {"wq": rnd(h, h, std=0.02), "wk": rnd(h, h, std=0.02), "wv": rnd(h, h, std=0.02),
               "wo": rnd(h, h, std=0.02), "w1": rnd(h, F, std=0.02), "w2": rnd(F, h, std=0.02)}
     sw = tsp.pack_shards(dims, D, w_full)
     del w_full
     kv_std = 0.02 * math.sqrt(h)
     x_local = rnd(L, h)
-    K = rnd(T, h, std=kv_std)
-    V = rnd(T, h, std=kv_std)
+    K = rnd(T, h, std=kv_std, dtype=torch.float16)
+    V = rnd(T, h, std=kv_std, dtype=torch.float16)
     y = torch.empty(L, h, dtype=torch.bfloat16, device="cuda")
     ws = tsp.alloc_workspace(dims, D)
     stream = torch.cuda.current_stream()
@@ -312,7 +312,7 @@ def run_tsp(args, wl):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "vs_baseline": None, "dtype": "fp16", "data": "synthetic",
             "config": {"workload": wl["desc"], "T": T, "D": D, "tsp_rank": trank, "local_tokens": L,
                        "parallelism": f"{world} GPU(s), each an independent TSP rank (rank = gpu mod {D})",
                        "l2": "inputs larger than L2 (K/V 2 x 1 GiB, weights 384 MiB); no flush"},

@@ -24,8 +24,9 @@
 //   warp 1     TMEM allocator + single-thread tcgen05.mma issuer
 //   warps 2-5  softmax / correction / epilogue, one thread per query row
 // Tensor memory (512 columns): S0 | S1 (128 fp32 columns each, double
-// buffered scores), O (d fp32 columns), P0 | P1 (64 columns each: 128 bf16
-// probabilities packed in pairs, the A operand of O += P V).
+// buffered scores), O (d fp32 columns), P0 | P1 (64 columns each: 128 fp16
+// probabilities packed in pairs, the A operand of O += P V).  Q, K, V and
+// the output are fp16; scores, the softmax statistics and O are fp32.
 // Online softmax in base 2 with a lazily updated row maximum: the running
 // output is rescaled only when the maximum grows by more than 2^8, which is
 // exact (the final division by the row sum cancels the common factor).
@@ -40,10 +41,10 @@ constexpr int kAttnBM = 128;
 constexpr int kAttnBN = 128;
 
 struct __align__(64) AttnParams {
-  CUtensorMap map_q;  // Q [L, h], box {64, 128}
-  CUtensorMap map_k;  // K [T, h], box {64, 128}
-  CUtensorMap map_v;  // V [T, h], box {64, 128}
-  __nv_bfloat16* out; // A [L, h]
+  CUtensorMap map_q;  // Q [L, h] fp16, box {64, 128}
+  CUtensorMap map_k;  // K [T, h] fp16, box {64, 128}
+  CUtensorMap map_v;  // V [T, h] fp16, box {64, 128}
+  __half* out;        // A [L, h] fp16
   int64_t ldo;        // h
   int c;              // chunk length
   int rank, D, H;
@@ -209,8 +210,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (elect_one()) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(kAttnBM, kAttnBN, 0, 0);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(kAttnBM, HD, 0, 1);
+      constexpr uint32_t idesc_s = idesc_f32acc(kAttnBM, kAttnBN, 0, 0, kFmtF16);
+      constexpr uint32_t idesc_o = idesc_f32acc(kAttnBM, HD, 0, 1, kFmtF16);
       int ks = 0, vs = 0;
       uint32_t kph = 0, vph = 0, qph = 0;
       uint32_t g = 0;      // global score-tile counter (S/P buffer = g & 1)
@@ -346,7 +347,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
               const float p0 = ex2_approx(fmaf(s[j * 64 + 2 * i], sl2, -m_used));
               const float p1 = ex2_approx(fmaf(s[j * 64 + 2 * i + 1], sl2, -m_used));
               l += p0 + p1;
-              r[i] = pack_bf16x2(p0, p1);
+              r[i] = pack_half2(p0, p1);
             }
             tmem_st32(tmem + lane_off + S::kColP + pb * 64 + j * 32, r);
           }
@@ -357,12 +358,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
         }
       }
       if (!ok) break;
-      // epilogue: O / l -> bf16 -> A[m0 + row, head]
+      // epilogue: O / l -> fp16 -> A[m0 + row, head]
       const uint32_t gl = g - 1;
       if (!warp_wait(&o_done[gl & 1], (gl >> 1) & 1, ctl)) break;
       tc_fence_after();
       const float inv = 1.0f / l;
-      __nv_bfloat16* dst = p.out + static_cast<int64_t>(w.m0 + row) * p.ldo + w.head * HD;
+      __half* dst = p.out + static_cast<int64_t>(w.m0 + row) * p.ldo + w.head * HD;
 #pragma unroll
       for (int j = 0; j < HD / 32; ++j) {
         uint32_t r[32];
@@ -372,10 +373,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
           uint4* d4 = reinterpret_cast<uint4*>(dst + j * 32);
 #pragma unroll
           for (int i = 0; i < 4; ++i)
-            d4[i] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * i]) * inv, __uint_as_float(r[8 * i + 1]) * inv),
-                               pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv, __uint_as_float(r[8 * i + 3]) * inv),
-                               pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv, __uint_as_float(r[8 * i + 5]) * inv),
-                               pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv, __uint_as_float(r[8 * i + 7]) * inv));
+            d4[i] = make_uint4(pack_half2(__uint_as_float(r[8 * i]) * inv, __uint_as_float(r[8 * i + 1]) * inv),
+                               pack_half2(__uint_as_float(r[8 * i + 2]) * inv, __uint_as_float(r[8 * i + 3]) * inv),
+                               pack_half2(__uint_as_float(r[8 * i + 4]) * inv, __uint_as_float(r[8 * i + 5]) * inv),
+                               pack_half2(__uint_as_float(r[8 * i + 6]) * inv, __uint_as_float(r[8 * i + 7]) * inv));
         }
         __syncwarp();
       }

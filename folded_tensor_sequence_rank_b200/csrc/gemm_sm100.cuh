@@ -1,7 +1,7 @@
 // gemm_sm100.cuh - persistent tcgen05 GEMM C = A * B^T for the TSP shard loops.
 //
-// A [M, K] bf16 K-major (one tensor map), B given as a list of per-shard
-// K-major tensor maps.  Two ways the shard list is walked, both without any
+// A [M, K] fp16 K-major (one tensor map), B given as a list of per-shard
+// fp16 K-major tensor maps; fp32 accumulation in tensor memory.  Two ways the shard list is walked, both without any
 // reduction kernel:
 //   N-split (Q/K/V and W1 shards: each shard owns a block of output columns):
 //     output column block n belongs to map n / shard_n.
@@ -14,7 +14,9 @@
 //   warp 0     TMA producer: A and B tiles into a STAGES-deep shared ring
 //   warp 1     TMEM allocator + single-thread tcgen05.mma issuer
 //   warps 2-5  epilogue: tcgen05.ld the 128 x BN fp32 accumulator (thread =
-//              row), apply store / GELU / residual, write to global memory.
+//              row), apply store / GELU / residual, write to global memory
+//              (fp16 operands for the next matmul, or the fp32 / bf16
+//              residual stream).
 // Two TMEM accumulators let the epilogue of tile i overlap the K loop of
 // tile i+1.
 #pragma once
@@ -39,7 +41,7 @@ struct __align__(64) GemmParams {
   int shard_k;    // K-split: reduction length per B map
   int seg_n;      // N-split: output columns per output segment
   int epi;        // GemmEpi
-  void* out[3];   // per segment (N-split) or out[0] (K-split)
+  void* out[3];   // per segment (N-split, fp16) or out[0] (K-split, fp32 / bf16)
   int remap[3];   // per segment: 1 = write local row m at its global zigzag row
   int64_t ldo;    // output row stride, elements
   const void* resid;  // kEpiResidual: residual [M, N] (row stride ldo)
@@ -71,10 +73,14 @@ __device__ __forceinline__ void gemm_tile_coords(int tile, int num_m, int num_n,
   nb = local / gm;
 }
 
+// GELU, tanh form, through the identity 0.5 (1 + tanh(u)) = 1 / (1 + e^(-2u)):
+//   GELU(x) = x / (1 + 2^(-2 u log2(e))),  u = sqrt(2/pi) (x + 0.044715 x^3).
+// ex2.approx has ~2^-22 relative error and the division is IEEE-rounded, so
+// the result is accurate to a few fp32 ulps before its bf16 rounding.
 __device__ __forceinline__ float gelu_tanh_f(float x) {
-  const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
-  const float u = k0 * fmaf(0.044715f * x, x * x, x);
-  return 0.5f * x * (1.0f + tanh_approx(u));
+  const float k = -2.0f * 0.7978845608028654f * 1.4426950408889634f;  // -2 sqrt(2/pi) log2(e)
+  const float u = fmaf(0.044715f * x, x * x, x);
+  return x / (1.0f + ex2_approx(k * u));
 }
 
 // Bounded wait that ignores the abort flag: used only to drain copies and
@@ -88,7 +94,7 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, uint6
 }
 
 template <int BN>
-__global__ void __launch_bounds__(kGemmThreads, 1) gemm_bf16_tcgen05(const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(kGemmThreads, 1) gemm_f16_tcgen05(const __grid_constant__ GemmParams p) {
   using S = GemmShape<BN>;
   constexpr int STAGES = S::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -171,7 +177,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_bf16_tcgen05(const __gri
     }
   } else if (warp == 1) {
     if (elect_one()) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kGemmBM, BN, 0, 0);
+      constexpr uint32_t idesc = idesc_f32acc(kGemmBM, BN, 0, 0, kFmtF16);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -271,13 +277,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_bf16_tcgen05(const __gri
           if (p.epi == kEpiGeluBf16) {
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-              packed[i] = pack_bf16x2(gelu_tanh_f(__uint_as_float(r[2 * i])), gelu_tanh_f(__uint_as_float(r[2 * i + 1])));
+              packed[i] = pack_half2(gelu_tanh_f(__uint_as_float(r[2 * i])), gelu_tanh_f(__uint_as_float(r[2 * i + 1])));
           } else {
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-              packed[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+              packed[i] = pack_half2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
           }
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out[seg]) + orow * p.ldo + col);
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__half*>(p.out[seg]) + orow * p.ldo + col);
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);

@@ -1,5 +1,5 @@
 // misc_kernels.cuh - the bandwidth-bound pieces of the TSP rank forward:
-// zigzag index map, pre-LayerNorm with bf16 output, weight shard packing, and
+// zigzag index map, pre-LayerNorm with fp16 output, weight shard packing, and
 // the bounded-wait self test.
 #pragma once
 #include "ptx.cuh"
@@ -40,9 +40,10 @@ __device__ __forceinline__ void load8<float>(const float* src, float (&v)[8]) {
 // LayerNorm of one row per warp, gamma=1, beta=0:
 //   y = (x - mean) / sqrt(var + eps), var biased, statistics in fp32 over the
 //   row held in registers (two passes: mean, then centred sum of squares).
-// Output bf16 (round to nearest even).  MAXC = 8-element chunks per lane.
+// Output fp16 (round to nearest even), the operand format of the matmul that
+// follows.  MAXC = 8-element chunks per lane.
 template <typename Tin, int MAXC>
-__global__ void __launch_bounds__(256) layernorm_rows_kernel(const Tin* __restrict__ x, __nv_bfloat16* __restrict__ y,
+__global__ void __launch_bounds__(256) layernorm_rows_kernel(const Tin* __restrict__ x, __half* __restrict__ y,
                                                              int64_t rows, int h, float eps) {
   const int warps = blockDim.x >> 5;
   const int64_t r = blockIdx.x * static_cast<int64_t>(warps) + (threadIdx.x >> 5);
@@ -82,38 +83,43 @@ __global__ void __launch_bounds__(256) layernorm_rows_kernel(const Tin* __restri
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
   const float rstd = rsqrtf(sq / h + eps);
-  __nv_bfloat16* yr = y + r * h;
+  __half* yr = y + r * h;
 #pragma unroll
   for (int c = 0; c < MAXC; ++c) {
     const int ch = lane + 32 * c;
     if (ch < nch) {
       uint4 o;
-      o.x = pack_bf16x2((v[c][0] - mean) * rstd, (v[c][1] - mean) * rstd);
-      o.y = pack_bf16x2((v[c][2] - mean) * rstd, (v[c][3] - mean) * rstd);
-      o.z = pack_bf16x2((v[c][4] - mean) * rstd, (v[c][5] - mean) * rstd);
-      o.w = pack_bf16x2((v[c][6] - mean) * rstd, (v[c][7] - mean) * rstd);
+      o.x = pack_half2((v[c][0] - mean) * rstd, (v[c][1] - mean) * rstd);
+      o.y = pack_half2((v[c][2] - mean) * rstd, (v[c][3] - mean) * rstd);
+      o.z = pack_half2((v[c][4] - mean) * rstd, (v[c][5] - mean) * rstd);
+      o.w = pack_half2((v[c][6] - mean) * rstd, (v[c][7] - mean) * rstd);
       *reinterpret_cast<uint4*>(yr + ch * 8) = o;
     }
   }
 }
 
 // Shard packing: out[o][i] = w[(row0 + i) * ld + col0 + o] for o < n_out,
-// i < n_in; i.e. a transposed sub-block of the math-orientation weight, giving
-// the K-major [n_out, n_in] layout the GEMM's B operand uses.  32x32 tiles
-// staged through shared memory so both sides are coalesced.
+// i < n_in; i.e. a transposed sub-block of the math-orientation bf16 weight,
+// converted to fp16 (round to nearest even, saturating) in the K-major
+// [n_out, n_in] layout the GEMM's B operand uses.  32x32 tiles staged through
+// shared memory so both sides are coalesced.
 __global__ void pack_transpose_kernel(const __nv_bfloat16* __restrict__ w, int64_t ld, int64_t row0, int64_t col0,
-                                      __nv_bfloat16* __restrict__ out, int n_out, int n_in) {
-  __shared__ __nv_bfloat16 tile[32][33];
+                                      __half* __restrict__ out, int n_out, int n_in) {
+  __shared__ float tile[32][33];
   const int i0 = blockIdx.x * 32, o0 = blockIdx.y * 32;
   const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
   for (int k = ty; k < 32; k += 8) {
     const int i = i0 + k, o = o0 + tx;
-    if (i < n_in && o < n_out) tile[k][tx] = w[(row0 + i) * ld + col0 + o];
+    if (i < n_in && o < n_out) tile[k][tx] = __bfloat162float(w[(row0 + i) * ld + col0 + o]);
   }
   __syncthreads();
   for (int k = ty; k < 32; k += 8) {
     const int o = o0 + k, i = i0 + tx;
-    if (i < n_in && o < n_out) out[static_cast<int64_t>(o) * n_in + i] = tile[tx][k];
+    if (i < n_in && o < n_out) {
+      uint16_t hbits;
+      asm("cvt.rn.satfinite.f16.f32 %0, %1;" : "=h"(hbits) : "f"(tile[tx][k]));
+      reinterpret_cast<uint16_t*>(out)[static_cast<int64_t>(o) * n_in + i] = hbits;
+    }
   }
 }
 

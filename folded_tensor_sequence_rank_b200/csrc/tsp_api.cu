@@ -56,7 +56,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D bf16 row-major [rows, cols] with row stride ld elements; box = 64
+// 2-D fp16 row-major [rows, cols] with row stride ld elements; box = 64
 // columns (128 bytes, 128B swizzle) x box_rows rows.
 int make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld, int box_rows) {
   auto fn = encode_fn();
@@ -68,7 +68,7 @@ int make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
   cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
@@ -154,7 +154,7 @@ int check_weights(const tsp_weights* w, int D) {
 
 // ---------------------------------------------------------------- launches
 template <typename Tin>
-int launch_layernorm(const Tin* x, __nv_bfloat16* y, int64_t rows, int h, float eps, cudaStream_t st) {
+int launch_layernorm(const Tin* x, __half* y, int64_t rows, int h, float eps, cudaStream_t st) {
   if (rows == 0) return TSP_OK;
   const int warps = 8;
   const dim3 grid(static_cast<unsigned>((rows + warps - 1) / warps));
@@ -175,12 +175,12 @@ int launch_gemm_bn(GemmParams& p, cudaStream_t st) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(gemm_bf16_tcgen05<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes);
+    attr_err = cudaFuncSetAttribute(gemm_f16_tcgen05<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes);
   });
   TSP_CUDA(attr_err);
   const int tiles = ((p.M + kGemmBM - 1) / kGemmBM) * (p.N / BN);
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  gemm_bf16_tcgen05<BN><<<grid, kGemmThreads, S::kSmemBytes, st>>>(p);
+  gemm_f16_tcgen05<BN><<<grid, kGemmThreads, S::kSmemBytes, st>>>(p);
   TSP_CUDA(cudaGetLastError());
   return TSP_OK;
 }
@@ -210,7 +210,7 @@ void gemm_common(GemmParams& p, const Sizes& s, int rank, int* status) {
 
 // N-split projection of xn [L, h] by nseg weight families (each D shards
 // [h/D, h]) into nseg outputs [*, h]; remap[i] sends rows to global rows.
-int launch_proj(const Sizes& s, int rank, const __nv_bfloat16* xn, const void* const* fam[3], void* out[3],
+int launch_proj(const Sizes& s, int rank, const __half* xn, const void* const* fam[3], void* out[3],
                 const int remap[3], int nseg, int epi, int F_cols, int* status, cudaStream_t st) {
   static thread_local GemmParams p;
   std::memset(&p, 0, sizeof(p));
@@ -241,7 +241,7 @@ int launch_proj(const Sizes& s, int rank, const __nv_bfloat16* xn, const void* c
 }
 
 // K-split: out = resid + sum_k A[:, k-block] W_k^T, W_k [h, Kdim/D].
-int launch_ksplit(const Sizes& s, int rank, const __nv_bfloat16* a, int Kdim, const void* const* fam, const void* resid,
+int launch_ksplit(const Sizes& s, int rank, const __half* a, int Kdim, const void* const* fam, const void* resid,
                   int resid_f32, void* out, int out_f32, int* status, cudaStream_t st) {
   static thread_local GemmParams p;
   std::memset(&p, 0, sizeof(p));
@@ -270,8 +270,8 @@ int launch_ksplit(const Sizes& s, int rank, const __nv_bfloat16* a, int Kdim, co
   return launch_gemm(p, bn, st);
 }
 
-int launch_attention(const Sizes& s, int rank, const tsp_dims* dims, const __nv_bfloat16* q, const void* k_full,
-                     const void* v_full, __nv_bfloat16* out, int* counter, int* status, cudaStream_t st) {
+int launch_attention(const Sizes& s, int rank, const tsp_dims* dims, const __half* q, const void* k_full,
+                     const void* v_full, __half* out, int* counter, int* status, cudaStream_t st) {
   if (s.L == 0) return TSP_OK;
   static thread_local AttnParams p;
   std::memset(&p, 0, sizeof(p));
@@ -324,7 +324,7 @@ struct Ctx {
   uint8_t* ws;
   int* status;
   int* counters;
-  __nv_bfloat16 *xn, *q, *a, *hbuf;
+  __half *xn, *q, *a, *hbuf;
   float* y1;
 };
 
@@ -342,11 +342,11 @@ int make_ctx(Ctx& c, const tsp_dims* dims, const tsp_weights* w, int rank, void*
   c.ws = static_cast<uint8_t*>(ws);
   c.status = reinterpret_cast<int*>(c.ws + c.lay.status);
   c.counters = reinterpret_cast<int*>(c.ws + c.lay.counters);
-  c.xn = reinterpret_cast<__nv_bfloat16*>(c.ws + c.lay.xn);
-  c.q = reinterpret_cast<__nv_bfloat16*>(c.ws + c.lay.q);
-  c.a = reinterpret_cast<__nv_bfloat16*>(c.ws + c.lay.a);
+  c.xn = reinterpret_cast<__half*>(c.ws + c.lay.xn);
+  c.q = reinterpret_cast<__half*>(c.ws + c.lay.q);
+  c.a = reinterpret_cast<__half*>(c.ws + c.lay.a);
   c.y1 = reinterpret_cast<float*>(c.ws + c.lay.y1);
-  c.hbuf = reinterpret_cast<__nv_bfloat16*>(c.ws + c.lay.hbuf);
+  c.hbuf = reinterpret_cast<__half*>(c.ws + c.lay.hbuf);
   return TSP_OK;
 }
 
@@ -440,7 +440,7 @@ int tsp_pack_shards(const tsp_dims* dims, int D, const void* const w_full[6], vo
     *dst = p;
     const dim3 grid((n_in + 31) / 32, (n_out + 31) / 32);
     pack_transpose_kernel<<<grid, blk, 0, stream>>>(static_cast<const __nv_bfloat16*>(src), ld, row0, col0,
-                                                    reinterpret_cast<__nv_bfloat16*>(p), n_out, n_in);
+                                                    reinterpret_cast<__half*>(p), n_out, n_in);
     TSP_CUDA(cudaGetLastError());
     p += align_up(static_cast<size_t>(n_out) * n_in * 2);
     return TSP_OK;

@@ -13,7 +13,8 @@ each tensor rounded once to bf16 round-to-nearest-even):
   ``y = x @ W`` ([in, out]).
 * ``rank_inputs``: the rank's own tokens x_local [L, h] ~ N(0, 1), the six
   weights as above, then a stand-in for the all-gathered key/value tensors
-  K, V [T, h] ~ N(0, kv_std^2).  ``kv_std`` defaults to 0.02*sqrt(h), the
+  K, V [T, h] ~ N(0, kv_std^2), rounded to fp16 (the format the layer keeps
+  K and V in) instead of bf16.  ``kv_std`` defaults to 0.02*sqrt(h), the
   standard deviation of LayerNorm(x) @ W for such weights, so attention
   logits have the spread the real projection gives.
 """
@@ -27,11 +28,11 @@ WEIGHT_STD = 0.02
 WEIGHT_NAMES = ("wq", "wk", "wv", "wo", "w1", "w2")
 
 
-def _draw(gen: torch.Generator, shape, std: float) -> torch.Tensor:
+def _draw(gen: torch.Generator, shape, std: float, dtype=torch.bfloat16) -> torch.Tensor:
     t = torch.randn(*shape, generator=gen, dtype=torch.float32)
     if std != 1.0:
         t.mul_(std)
-    return t.to(torch.bfloat16)
+    return t.to(dtype)
 
 
 def _weights(gen: torch.Generator, h: int, F: int) -> dict:
@@ -51,15 +52,15 @@ def layer_inputs(T: int, h: int, F: int, seed: int) -> dict:
 
 def rank_inputs(L: int, T: int, h: int, F: int, seed: int,
                 kv_std: float | None = None) -> dict:
-    """One rank's tokens, the weights and stand-in full-sequence K/V (bf16, CPU)."""
+    """One rank's tokens and the weights (bf16), stand-in full-sequence K/V (fp16); CPU."""
     if kv_std is None:
         kv_std = WEIGHT_STD * math.sqrt(h)
     gen = torch.Generator(device="cpu")
     gen.manual_seed(seed)
     out = {"x_local": _draw(gen, (L, h), 1.0)}
     out.update(_weights(gen, h, F))
-    out["k_full"] = _draw(gen, (T, h), kv_std)
-    out["v_full"] = _draw(gen, (T, h), kv_std)
+    out["k_full"] = _draw(gen, (T, h), kv_std, torch.float16)
+    out["v_full"] = _draw(gen, (T, h), kv_std, torch.float16)
     return out
 
 

@@ -150,11 +150,11 @@ class ShardedWeights:
         ptr = getattr(self.struct, name)[k]
         n = int(torch.tensor(shape).prod())
         off = ptr - base
-        return self.buf[off: off + 2 * n].view(torch.bfloat16).view(*shape)
+        return self.buf[off: off + 2 * n].view(torch.float16).view(*shape)
 
 
 def pack_shards(dims: Dims, D: int, w_full: dict, stream=None) -> ShardedWeights:
-    """Splits full math-orientation weights ([in, out], bf16, CUDA) into D shards."""
+    """Splits full math-orientation bf16 weights ([in, out], CUDA) into D fp16 shards."""
     h, F = dims.h, dims.ffn
     shapes = {"wq": (h, h), "wk": (h, h), "wv": (h, h), "wo": (h, h), "w1": (h, F), "w2": (F, h)}
     ptrs = (ctypes.c_void_p * 6)(*[_ptr(w_full[n], n, torch.bfloat16, shapes[n]) for n in WEIGHT_NAMES])
@@ -190,9 +190,9 @@ def workspace_view(ws: torch.Tensor, dims: Dims, D: int, name: str) -> torch.Ten
     """Views of the per-rank intermediates left in the workspace."""
     off = workspace_offsets(dims, D)
     L, h, F = dims.T // D, dims.h, dims.ffn
-    table = {"xn": (1, torch.bfloat16, (L, h)), "q": (2, torch.bfloat16, (L, h)),
-             "a": (3, torch.bfloat16, (L, h)), "y1": (4, torch.float32, (L, h)),
-             "h": (5, torch.bfloat16, (L, F))}
+    table = {"xn": (1, torch.float16, (L, h)), "q": (2, torch.float16, (L, h)),
+             "a": (3, torch.float16, (L, h)), "y1": (4, torch.float32, (L, h)),
+             "h": (5, torch.float16, (L, F))}
     i, dt, shape = table[name]
     nb = int(torch.tensor(shape).prod()) * (4 if dt == torch.float32 else 2)
     return ws[off[i]: off[i] + nb].view(dt).view(*shape)
@@ -212,8 +212,8 @@ def get_device_status(ws: torch.Tensor, stream=None) -> int:
 def _rank_io(dims: Dims, w: ShardedWeights, x_local, k_full, v_full, y_local, ws):
     L, h, T = dims.T // w.D, dims.h, dims.T
     px = _ptr(x_local, "x_local", torch.bfloat16, (L, h))
-    pk = _ptr(k_full, "k_full", torch.bfloat16, (T, h))
-    pv = _ptr(v_full, "v_full", torch.bfloat16, (T, h))
+    pk = _ptr(k_full, "k_full", torch.float16, (T, h))
+    pv = _ptr(v_full, "v_full", torch.float16, (T, h))
     if y_local is not None and y_local.dtype not in (torch.bfloat16, torch.float32):
         raise ValueError("y_local must be bf16 or fp32")
     py = _ptr(y_local, "y_local", None, (L, h)) if y_local is not None else None
@@ -226,6 +226,9 @@ def _events(events):
         return None
     if len(events) != N_STEP_EVENTS:
         raise ValueError(f"need {N_STEP_EVENTS} events")
+    for e in events:
+        if not e.cuda_event:  # torch creates the CUDA event on its first record
+            e.record()
     return (ctypes.c_void_p * N_STEP_EVENTS)(*[e.cuda_event for e in events])
 
 
@@ -261,8 +264,8 @@ def rank_step_host(dims: Dims, w: ShardedWeights, rank: int, h_x_local, x_stagin
     phy = _ptr(h_y_local, "h_y_local", y_staging.dtype, (L, h), cuda=False)
     pxs = _ptr(x_staging, "x_staging", torch.bfloat16, (L, h))
     pys = _ptr(y_staging, "y_staging", None, (L, h))
-    pk = _ptr(k_full, "k_full", torch.bfloat16, (dims.T, h))
-    pv = _ptr(v_full, "v_full", torch.bfloat16, (dims.T, h))
+    pk = _ptr(k_full, "k_full", torch.float16, (dims.T, h))
+    pv = _ptr(v_full, "v_full", torch.float16, (dims.T, h))
     yd = OUT_F32 if y_staging.dtype == torch.float32 else OUT_BF16
     _check(lib().tsp_rank_step_host(ctypes.byref(dims), ctypes.byref(w.struct), rank, phx, pxs, pk, pv, pys, phy,
                                     yd, _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream)),

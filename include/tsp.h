@@ -31,8 +31,15 @@
  *   - Shard k of the attention weights is head group k (heads
  *     k*H/D .. (k+1)*H/D-1, i.e. hidden columns k*h/D .. (k+1)*h/D-1); shard
  *     k of the FFN is FFN columns k*F/D .. (k+1)*F/D-1.
- *   - K/V full-sequence tensors are [T, h] bf16 in natural (global) order,
+ *   - K/V full-sequence tensors are [T, h] fp16 in natural (global) order,
  *     head j in columns j*d .. (j+1)*d-1.
+ *   - Number formats: the model's tensors (X, the weights, Y) are bf16; the
+ *     operands of every matmul inside the layer (LayerNorm outputs, Q, K, V,
+ *     softmax probabilities, attention output, GELU output, weight shards)
+ *     are held in fp16 - the same 16 bits and tensor-core rate, three more
+ *     significand bits - with fp32 accumulation; the residual stream
+ *     X + attention is fp32.  Conversions round to nearest even and
+ *     saturate at +-65504.
  *   - Every device buffer is allocated and freed by the caller.  Functions
  *     that take a stream only enqueue work on it (asynchronous) unless
  *     stated otherwise; the library allocates no device memory and keeps no
@@ -77,10 +84,10 @@ typedef struct {
   float softmax_scale; /* applied to q.k; 1/sqrt(d) for the 7B layer */
 } tsp_dims;
 
-/* Per-shard device pointers (bf16), each shard one contiguous K-major
+/* Per-shard device pointers (fp16), each shard one contiguous K-major
  * buffer:  wq/wk/wv[k] [h/D, h],  wo[k] [h, h/D],  w1[k] [F/D, h],
  * w2[k] [h, F/D].  Only entries 0..D-1 are read.  Pointers must be 16-byte
- * aligned. */
+ * aligned.  tsp_pack_shards builds them from the bf16 model weights. */
 typedef struct {
   int32_t D;
   const void* wq[TSP_MAX_D];
@@ -118,7 +125,7 @@ size_t tsp_shard_buffer_bytes(const tsp_dims* dims, int D);
 /* Splits full weights into per-rank shards [zubnet.ai TSP item, paragraph 1:
  * "each GPU holds 1/D of the weights"].  w_full[6] = {Wq, Wk, Wv, Wo, W1, W2}
  * are device bf16 in the math orientation y = x W ([in, out]: Wq/Wk/Wv/Wo
- * [h, h], W1 [h, F], W2 [F, h]).  Writes the K-major shards into d_buf
+ * [h, h], W1 [h, F], W2 [F, h]).  Writes the K-major fp16 shards into d_buf
  * (tsp_shard_buffer_bytes bytes, caller-owned) and fills *out with
  * pointers into d_buf. */
 int tsp_pack_shards(const tsp_dims* dims, int D, const void* const w_full[6],
@@ -131,10 +138,10 @@ size_t tsp_workspace_bytes(const tsp_dims* dims, int D);
 
 /* Byte offsets inside the workspace of the per-rank intermediates, for
  * inspection after a call (all rank-local order, row-major):
- *   off[0] status word (int32),  off[1] LN output xn bf16 [L, h] (LN2's
- *   output after tsp_layer_forward),  off[2] Q bf16 [L, h],  off[3]
- *   attention output bf16 [L, h],  off[4] Y1 = X + attention projection,
- *   fp32 [L, h],  off[5] H = GELU(LN2(Y1) W1) bf16 [L, F],  off[6]
+ *   off[0] status word (int32),  off[1] LN output xn fp16 [L, h] (LN2's
+ *   output after tsp_layer_forward),  off[2] Q fp16 [L, h],  off[3]
+ *   attention output fp16 [L, h],  off[4] Y1 = X + attention projection,
+ *   fp32 [L, h],  off[5] H = GELU(LN2(Y1) W1) fp16 [L, F],  off[6]
  *   scheduler counters,  off[7] total bytes.  Returns TSP_OK or
  *   TSP_ERR_INVALID_ARG. */
 int tsp_workspace_offsets(const tsp_dims* dims, int D, size_t off[8]);
@@ -151,7 +158,7 @@ int tsp_get_device_status(const void* ws, cudaStream_t stream);
  * all-gathered with the zigzag partition]:
  *     K[pos(i)] = LN1(x_local[i]) Wk,   V[pos(i)] = LN1(x_local[i]) Wv
  * for all D shards (head groups), written at the tokens' GLOBAL rows of
- * k_full / v_full ([T, h] bf16) - the place the all-gather puts them.
+ * k_full / v_full ([T, h] fp16) - the place the all-gather puts them.
  * x_local: bf16 [T/D, h] rank-local order.  With D=1, rank 0 this projects
  * a whole natural-order sequence.  ws: tsp_workspace_bytes(dims, D). */
 int tsp_kv_project(const tsp_dims* dims, const tsp_weights* w, int rank,
@@ -165,7 +172,7 @@ int tsp_kv_project(const tsp_dims* dims, const tsp_weights* w, int rank,
  *   sees keys 0..p),  Y1 = x_local + sum_k A_k Wo_k^T;
  *   Y = Y1 + sum_k GELU(LN2(Y1) W1_k^T) W2_k^T  (the shard sum is local:
  *   no all-reduce).
- * x_local bf16 [T/D, h] rank-local order; k_full, v_full bf16 [T, h]
+ * x_local bf16 [T/D, h] rank-local order; k_full, v_full fp16 [T, h]
  * natural order (read only); y_local [T/D, h] rank-local order, bf16
  * (y_dtype TSP_OUT_BF16) or fp32 (TSP_OUT_F32); the bf16 result is the
  * fp32 result rounded to nearest even.  step_events: NULL, or

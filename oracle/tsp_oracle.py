@@ -33,12 +33,18 @@ the all-gathered K/V, ``rank_rows_forward``).  ``rank_forward_sharded`` and
 pin them to the plain definition (the sum over shards equals the unsharded
 contraction).
 
-Precision: every product and sum is fp64.  A bf16 layer stores the
-activations that feed its matmuls in bf16, so the oracle rounds exactly
-those to bf16 (round to nearest even): LN1 output, Q, K, V, the attention
-output, LN2 output and the GELU output H.  The residual stream (X + attn,
-and the layer output) stays fp64.  ``bf16_points=False`` gives the pure
-fp64 layer for diagnostics.
+Precision: every product and sum is fp64.  The layer holds the operands
+of its matmuls in a 16-bit float, so the oracle rounds exactly those values
+(round to nearest even) at the points where the layer stores them: the
+weights, the LN1 output, Q, K, V, the attention output, the LN2 output and
+the GELU output H.  The residual stream (X + attention, and the layer
+output) stays unrounded.  The pages give the model's dtype as bf16; inputs X
+and weights arrive in bf16.  The storage format of the matmul operands is
+``storage``: "fp16" (11 significant bits, the default, what the CUDA path
+uses), "bf16" (8 bits) or None (no rounding: the pure fp64 layer).  fp16
+holds every value this pre-LayerNorm layer produces exactly as bf16 would
+(same 16 bits) but with three more significand bits; bf16 weights convert
+to fp16 exactly down to |w| = 2^-14 and within 2^-25 below that.
 
 Zigzag partition: the sequence is cut into 2D equal chunks of c = T/(2D)
 tokens, and rank r holds chunks r and 2D-1-r, in that order.
@@ -54,7 +60,7 @@ LN_EPS = 1e-5
 
 
 # ----------------------------------------------------------------------------
-# bf16 storage rounding
+# 16-bit storage rounding
 # ----------------------------------------------------------------------------
 def round_bf16(x) -> np.ndarray:
     """Round each value to the nearest bf16 number (ties to even), kept as fp64.
@@ -69,8 +75,21 @@ def round_bf16(x) -> np.ndarray:
     return np.ldexp(np.rint(m * 256.0) / 256.0, e)
 
 
-def _maybe_round(x, on: bool):
-    return round_bf16(x) if on else x
+def round_fp16(x) -> np.ndarray:
+    """Round each value to the nearest IEEE binary16 number (ties to even),
+    subnormals included, kept as fp64.  numpy's float64 -> float16 cast rounds
+    once, directly from the fp64 value."""
+    return np.asarray(x, dtype=np.float64).astype(np.float16).astype(np.float64)
+
+
+def _rounder(storage):
+    if storage is None:
+        return lambda a: np.asarray(a, dtype=np.float64)
+    if storage == "fp16":
+        return round_fp16
+    if storage == "bf16":
+        return round_bf16
+    raise ValueError(f"unknown storage format {storage!r}")
 
 
 # ----------------------------------------------------------------------------
@@ -150,52 +169,52 @@ def causal_attention(q, k, v, q_pos, n_heads: int, scale: float,
 # ----------------------------------------------------------------------------
 # the plain (unsharded) layer
 # ----------------------------------------------------------------------------
-def _f64(w: dict) -> dict:
-    return {n: np.asarray(a, dtype=np.float64) for n, a in w.items()}
+def _weights(w: dict, rnd) -> dict:
+    """The weights as the layer holds them for its matmuls."""
+    return {n: rnd(np.asarray(a, dtype=np.float64)) for n, a in w.items()}
 
 
-def kv_project(x_rows, w: dict, eps: float = LN_EPS, bf16_points: bool = True):
+def kv_project(x_rows, w: dict, eps: float = LN_EPS, storage="fp16"):
     """K and V rows of tokens `x_rows`: LN1(x) @ Wk and LN1(x) @ Wv."""
-    w = _f64(w)
-    xn = _maybe_round(layer_norm(x_rows, eps), bf16_points)
-    k = _maybe_round(xn @ w["wk"], bf16_points)
-    v = _maybe_round(xn @ w["wv"], bf16_points)
-    return k, v
+    rnd = _rounder(storage)
+    w = _weights(w, rnd)
+    xn = rnd(layer_norm(x_rows, eps))
+    return rnd(xn @ w["wk"]), rnd(xn @ w["wv"])
 
 
 def rank_rows_forward(x_rows, q_pos, k_full, v_full, w: dict, n_heads: int,
                       eps: float = LN_EPS, scale: float | None = None,
-                      bf16_points: bool = True) -> dict:
+                      storage="fp16") -> dict:
     """Layer output for tokens `x_rows` at global positions `q_pos`.
 
     `k_full`, `v_full` [T, h] are the keys and values of the whole sequence
     (what every rank holds after the all-gather).  Every step is row-local
     except attention, so any subset of a rank's rows can be computed alone.
-    Returns the output and the bf16-stored intermediates.
+    Returns the output and the stored intermediates.
     """
-    w = _f64(w)
+    rnd = _rounder(storage)
+    w = _weights(w, rnd)
     x = np.asarray(x_rows, dtype=np.float64)
     h = x.shape[1]
     if scale is None:
         scale = 1.0 / np.sqrt(h // n_heads)
-    r = bf16_points
-    xn1 = _maybe_round(layer_norm(x, eps), r)
-    q = _maybe_round(xn1 @ w["wq"], r)
-    a = _maybe_round(causal_attention(q, k_full, v_full, q_pos, n_heads, scale), r)
+    xn1 = rnd(layer_norm(x, eps))
+    q = rnd(xn1 @ w["wq"])
+    a = rnd(causal_attention(q, k_full, v_full, q_pos, n_heads, scale))
     y1 = x + a @ w["wo"]
-    xn2 = _maybe_round(layer_norm(y1, eps), r)
-    hh = _maybe_round(gelu_tanh(xn2 @ w["w1"]), r)
+    xn2 = rnd(layer_norm(y1, eps))
+    hh = rnd(gelu_tanh(xn2 @ w["w1"]))
     y = y1 + hh @ w["w2"]
     return {"xn1": xn1, "q": q, "a": a, "y1": y1, "xn2": xn2, "h": hh, "y": y}
 
 
 def layer_forward(x, w: dict, n_heads: int, eps: float = LN_EPS,
-                  scale: float | None = None, bf16_points: bool = True) -> dict:
+                  scale: float | None = None, storage="fp16") -> dict:
     """The whole unsharded layer over a full sequence x [T, h] (natural order)."""
     x = np.asarray(x, dtype=np.float64)
-    k, v = kv_project(x, w, eps, bf16_points)
+    k, v = kv_project(x, w, eps, storage)
     out = rank_rows_forward(x, np.arange(x.shape[0]), k, v, w, n_heads, eps,
-                            scale, bf16_points)
+                            scale, storage)
     out["k"], out["v"] = k, v
     return out
 
@@ -204,14 +223,15 @@ def layer_forward(x, w: dict, n_heads: int, eps: float = LN_EPS,
 # the pages' shard-by-shard schedule  [TSP ¶1, ¶2]
 # ----------------------------------------------------------------------------
 def kv_all_gather_sharded(x_full, D: int, w: dict, eps: float = LN_EPS,
-                          bf16_points: bool = True):
+                          storage="fp16"):
     """Full-sequence K/V as TSP builds it.
 
     Every rank r projects its own zigzag tokens with every attention shard
     k (head group k = columns k*h/D .. (k+1)*h/D of Wk, Wv); the all-gather
     places each rank's rows back at their global positions.
     """
-    w = _f64(w)
+    rnd = _rounder(storage)
+    w = _weights(w, rnd)
     x_full = np.asarray(x_full, dtype=np.float64)
     T, h = x_full.shape
     hs = h // D
@@ -219,18 +239,18 @@ def kv_all_gather_sharded(x_full, D: int, w: dict, eps: float = LN_EPS,
     V = np.zeros((T, h))
     for rank in range(D):
         idx = zigzag_index(T, D, rank)
-        xn = _maybe_round(layer_norm(x_full[idx], eps), bf16_points)
+        xn = rnd(layer_norm(x_full[idx], eps))
         for s in range(D):
             cols = slice(s * hs, (s + 1) * hs)
-            K[idx, cols] = _maybe_round(xn @ w["wk"][:, cols], bf16_points)
-            V[idx, cols] = _maybe_round(xn @ w["wv"][:, cols], bf16_points)
+            K[idx, cols] = rnd(xn @ w["wk"][:, cols])
+            V[idx, cols] = rnd(xn @ w["wv"][:, cols])
     return K, V
 
 
 def rank_forward_sharded(rank: int, D: int, x_local, k_full, v_full, w: dict,
                          n_heads: int, eps: float = LN_EPS,
                          scale: float | None = None,
-                         bf16_points: bool = True) -> np.ndarray:
+                         storage="fp16") -> np.ndarray:
     """Rank `rank`'s output computed the way TSP schedules it.
 
     Attention: shard k (heads k*H/D .. (k+1)*H/D of Wq and Wo) is applied to
@@ -239,7 +259,8 @@ def rank_forward_sharded(rank: int, D: int, x_local, k_full, v_full, w: dict,
     of W1, rows of W2) and adds GELU(x W1_k) W2_k; the sum over shards is
     local, so no all-reduce is needed.
     """
-    w = _f64(w)
+    rnd = _rounder(storage)
+    w = _weights(w, rnd)
     x = np.asarray(x_local, dtype=np.float64)
     L, h = x.shape
     T = np.asarray(k_full).shape[0]
@@ -247,23 +268,21 @@ def rank_forward_sharded(rank: int, D: int, x_local, k_full, v_full, w: dict,
     hs, Fs, Hs = h // D, F // D, n_heads // D
     if scale is None:
         scale = 1.0 / np.sqrt(h // n_heads)
-    r = bf16_points
     pos = zigzag_index(T, D, rank)
-    xn1 = _maybe_round(layer_norm(x, eps), r)
+    xn1 = rnd(layer_norm(x, eps))
     y1 = x.copy()
     for s in range(D):
         cols = slice(s * hs, (s + 1) * hs)
-        q_s = _maybe_round(xn1 @ w["wq"][:, cols], r)
-        a_s = _maybe_round(causal_attention(q_s, np.asarray(k_full)[:, cols],
-                                            np.asarray(v_full)[:, cols], pos,
-                                            Hs, scale), r)
+        q_s = rnd(xn1 @ w["wq"][:, cols])
+        a_s = rnd(causal_attention(q_s, np.asarray(k_full)[:, cols],
+                                   np.asarray(v_full)[:, cols], pos, Hs, scale))
         y1 = y1 + a_s @ w["wo"][cols, :]
-    xn2 = _maybe_round(layer_norm(y1, eps), r)
+    xn2 = rnd(layer_norm(y1, eps))
     y = y1.copy()
     for step in range(D):
         s = (rank + step) % D
         cols = slice(s * Fs, (s + 1) * Fs)
-        h_s = _maybe_round(gelu_tanh(xn2 @ w["w1"][:, cols]), r)
+        h_s = rnd(gelu_tanh(xn2 @ w["w1"][:, cols]))
         y = y + h_s @ w["w2"][cols, :]
     return y
 

@@ -3,7 +3,8 @@
 Gates (the layer's stated tolerance for bf16 layer outputs): max-abs <= 2e-2
 and relative-L2 <= 5e-3 on the layer output, computed in fp32 by the kernels
 (y_dtype fp32); the bf16 output equals the fp32 output rounded to nearest
-even bit for bit.  The zigzag index map and the weight shard packing are
+even bit for bit.  The oracle rounds the matmul operands to fp16 where the
+kernels store them (its default storage format).  The zigzag index map and the weight shard packing are
 integer / byte work and must match exactly.  Intermediates get looser
 diagnostic gates that catch errors the residual stream would hide.
 
@@ -47,11 +48,27 @@ def rel_l2(a, b):
 def assert_layer_close(y_gpu, y_ref, what, x=None):
     err = float(np.max(np.abs(y_gpu - y_ref)))
     rl = rel_l2(y_gpu, y_ref)
+    print(f"{what}: max-abs {err:.3e} rel-L2 {rl:.3e}")
     assert np.isfinite(y_gpu).all(), what
     assert err <= MAX_ABS and rl <= REL_L2, f"{what}: max-abs {err:.3e}, rel-L2 {rl:.3e}"
     if x is not None:  # the layer's own contribution, without the residual
         rd = rel_l2(y_gpu - x, y_ref - x)
         assert rd <= 2e-2, f"{what}: rel-L2 of (Y - X) {rd:.3e}"
+
+
+def assert_operand_close(g, e, what):
+    """A stored fp16 operand (K, V): equal up to rounding flips.  An LN output
+    that rounds the other way moves a K entry by up to ulp(xn) * |w| (about
+    2e-4 here), so a rare entry lands two fp16 units away; the bound allows
+    four units of the entry plus a floor of 2^-10 of the tensor's rms, and at
+    most 1e-4 of the entries may differ by more than one unit."""
+    scale = float(np.sqrt(np.mean(e * e)))
+    diff = np.abs(g - e)
+    ulp = np.maximum(2.0 ** (np.floor(np.log2(np.maximum(np.abs(e), 2.0 ** -14))) - 10), 2.0 ** -24)
+    assert np.all(diff <= 4 * ulp + 2.0 ** -10 * scale), f"{what}: max {diff.max():.3e} (rms {scale:.3e})"
+    frac = float(np.mean(diff > ulp * 1.0000001))
+    assert frac <= 1e-4, f"{what}: {frac:.2e} of entries more than one unit off"
+    assert rel_l2(g, e) <= 1e-3, f"{what}: rel-L2 {rel_l2(g, e):.3e}"
 
 
 def to_cuda(d):
@@ -83,7 +100,7 @@ def test_pack_shards_exact():
                   "wo": raw["wo"][cols, :].t(), "w1": raw["w1"][:, fcols].t(), "w2": raw["w2"][fcols, :].t()}
         for n, e in expect.items():
             got = sw.shard(n, k, tuple(e.shape))
-            assert torch.equal(got.view(torch.int16), e.contiguous().view(torch.int16)), (n, k)
+            assert torch.equal(got.view(torch.int16), e.to(torch.float16).contiguous().view(torch.int16)), (n, k)
 
 
 # --------------------------------------------------------------------------
@@ -95,7 +112,7 @@ def run_full_sequence(T, h, H, F, D, seed, y_dtype=torch.float32):
     dims = tsp.make_dims(T, h, H, F)
     sw = tsp.pack_shards(dims, D, dev)
     ws = tsp.alloc_workspace(dims, D)
-    K = torch.zeros(T, h, dtype=torch.bfloat16, device="cuda")
+    K = torch.zeros(T, h, dtype=torch.float16, device="cuda")
     V = torch.zeros_like(K)
     idx = [tsp.zigzag_index(T, D, r).long() for r in range(D)]
     x_loc = [dev["x"].index_select(0, i).contiguous() for i in idx]
@@ -125,16 +142,14 @@ def test_full_sequence_all_ranks(T, h, H, F, D, seed):
     raw, K, V, Y, idx, inter = run_full_sequence(T, h, H, F, D, seed)
     x = f64(raw["x"])
     ref = O.layer_forward(x, weights_f64(raw), H)
-    # K/V: bf16 results; allow a rounding flip of one bf16 unit
+    assert_layer_close(f64(Y), ref["y"], f"T={T} D={D}", x)
     for name, got in (("k", K), ("v", V)):
-        g, e = f64(got), ref[name]
-        assert np.all(np.abs(g - e) <= 2.0 ** -7 * np.abs(e) + 1e-6), name
+        assert_operand_close(f64(got), ref[name], name)
     for r in range(D):
         rows = idx[r].cpu().numpy()
-        for n, gate in (("q", 1e-2), ("a", 1e-2), ("y1", 1e-3), ("h", 2e-2)):
-            rl = rel_l2(f64(inter[r][n]), ref[n if n != "xn" else "xn2"][rows])
+        for n, gate in (("q", 1e-3), ("a", 2e-3), ("y1", 1e-4), ("h", 2e-3)):
+            rl = rel_l2(f64(inter[r][n]), ref[n][rows])
             assert rl <= gate, (r, n, rl)
-    assert_layer_close(f64(Y), ref["y"], f"T={T} D={D}", x)
 
 
 def test_bf16_output_is_rounded_fp32_output():
@@ -143,7 +158,7 @@ def test_bf16_output_is_rounded_fp32_output():
     dims = tsp.make_dims(T, h, H, F)
     sw = tsp.pack_shards(dims, D, raw)
     ws = tsp.alloc_workspace(dims, D)
-    K = torch.zeros(T, h, dtype=torch.bfloat16, device="cuda")
+    K = torch.zeros(T, h, dtype=torch.float16, device="cuda")
     V = torch.zeros_like(K)
     for r in range(D):
         xl = raw["x"].index_select(0, tsp.zigzag_index(T, D, r).long()).contiguous()
@@ -163,7 +178,7 @@ def test_rank_step_equals_projection_then_layer():
     dims = tsp.make_dims(T, h, H, F)
     sw = tsp.pack_shards(dims, D, raw)
     ws = tsp.alloc_workspace(dims, D)
-    K = torch.zeros(T, h, dtype=torch.bfloat16, device="cuda")
+    K = torch.zeros(T, h, dtype=torch.float16, device="cuda")
     V = torch.zeros_like(K)
     xs = [raw["x"].index_select(0, tsp.zigzag_index(T, D, r).long()).contiguous() for r in range(D)]
     for r in range(D):
@@ -189,7 +204,7 @@ def test_rank_step_host_buffers():
     dims = tsp.make_dims(T, h, H, F)
     sw = tsp.pack_shards(dims, D, raw)
     ws = tsp.alloc_workspace(dims, D)
-    K = torch.zeros(T, h, dtype=torch.bfloat16, device="cuda")
+    K = torch.zeros(T, h, dtype=torch.float16, device="cuda")
     V = torch.zeros_like(K)
     xs = [raw["x"].index_select(0, tsp.zigzag_index(T, D, r).long()).contiguous() for r in range(D)]
     for r in range(D):
@@ -218,7 +233,7 @@ def test_7b_layer_T8192_rank_in_full():
     dims = tsp.make_dims(T, h7, H7, F7)
     sw = tsp.pack_shards(dims, D, dev)
     ws = tsp.alloc_workspace(dims, D)
-    K = torch.zeros(T, h7, dtype=torch.bfloat16, device="cuda")
+    K = torch.zeros(T, h7, dtype=torch.float16, device="cuda")
     V = torch.zeros_like(K)
     xs = [dev["x"].index_select(0, tsp.zigzag_index(T, D, r).long()).contiguous() for r in range(D)]
     for r in range(D):
@@ -232,11 +247,12 @@ def test_7b_layer_T8192_rank_in_full():
     x = f64(raw["x"])
     w = weights_f64(raw)
     Kr, Vr = O.kv_project(x, w)
-    assert np.all(np.abs(f64(K) - Kr) <= 2.0 ** -7 * np.abs(Kr) + 1e-6)
     for r, y in ys.items():
         idx = O.zigzag_index(T, D, r)
         ref = O.rank_rows_forward(x[idx], idx, Kr, Vr, w, H7)
         assert_layer_close(f64(y), ref["y"], f"7B T=8192 rank {r}", x[idx])
+    assert_operand_close(f64(K), Kr, "k")
+    assert_operand_close(f64(V), Vr, "v")
 
 
 def sampled_rank_check(T, D, rank, seed, n_sample=62):
@@ -251,7 +267,7 @@ def sampled_rank_check(T, D, rank, seed, n_sample=62):
     y = torch.empty(L, h7, dtype=torch.float32, device="cuda")
     tsp.layer_forward(dims, sw, rank, dev["x_local"], dev["k_full"], dev["v_full"], y, ws)
     # the rank's own K/V projection, into scratch copies
-    Kp = torch.zeros(T, h7, dtype=torch.bfloat16, device="cuda")
+    Kp = torch.zeros(T, h7, dtype=torch.float16, device="cuda")
     Vp = torch.zeros_like(Kp)
     tsp.kv_project(dims, sw, rank, dev["x_local"], Kp, Vp, ws)
     assert tsp.get_device_status(ws) == tsp.TSP_OK
@@ -266,8 +282,8 @@ def sampled_rank_check(T, D, rank, seed, n_sample=62):
     assert_layer_close(y_s, ref["y"], f"7B T={T} D={D} rank {rank}", x[rows])
     kr, vr = O.kv_project(x[rows], w)
     gk, gv = f64(Kp[torch.as_tensor(pos[rows])]), f64(Vp[torch.as_tensor(pos[rows])])
-    assert np.all(np.abs(gk - kr) <= 2.0 ** -7 * np.abs(kr) + 1e-6)
-    assert np.all(np.abs(gv - vr) <= 2.0 ** -7 * np.abs(vr) + 1e-6)
+    assert_operand_close(gk, kr, "k rows")
+    assert_operand_close(gv, vr, "v rows")
 
 
 def test_7b_layer_128k_rank0_sampled():
@@ -304,5 +320,6 @@ def test_empty_sequence():
     sw = tsp.pack_shards(tsp.make_dims(4, 256, 4, 1024), 2, raw)
     ws = tsp.alloc_workspace(dims, 2)
     e = torch.empty(0, 256, dtype=torch.bfloat16, device="cuda")
-    tsp.layer_forward(dims, sw, 0, e, e, e, torch.empty(0, 256, device="cuda"), ws)
+    e16 = torch.empty(0, 256, dtype=torch.float16, device="cuda")
+    tsp.layer_forward(dims, sw, 0, e, e16, e16, torch.empty(0, 256, device="cuda"), ws)
     torch.cuda.synchronize()

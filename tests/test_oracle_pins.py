@@ -38,11 +38,27 @@ def bf16_rne_bits(t: torch.Tensor) -> torch.Tensor:
     return bits.view(torch.float64)
 
 
-def torch_layer(x, w, n_heads, eps=1e-5, bf16=True):
+def fp16_rne_bits(t: torch.Tensor) -> torch.Tensor:
+    """fp64 -> nearest IEEE half (ties to even): for |x| >= 2^-14 drop the low
+    42 of 52 fraction bits with round-half-even on the bit pattern; below that
+    the half grid is uniform with step 2^-24, rounded with torch.round (which
+    rounds halves to even)."""
+    t = t.contiguous()
+    bits = t.view(torch.int64)
+    lsb = (bits >> 42) & 1
+    normal = ((bits + ((1 << 41) - 1) + lsb) & ~((1 << 42) - 1)).view(torch.float64)
+    sub = torch.round(t * 2.0 ** 24) / 2.0 ** 24
+    return torch.where(t.abs() >= 2.0 ** -14, normal, sub)
+
+
+ROUNDERS = {None: (lambda t: t), "fp16": fp16_rne_bits, "bf16": bf16_rne_bits}
+
+
+def torch_layer(x, w, n_heads, eps=1e-5, storage="fp16"):
     """The layer composed from torch library routines, in fp64."""
-    rd = bf16_rne_bits if bf16 else (lambda t: t)
+    rd = ROUNDERS[storage]
     X = torch.as_tensor(np.asarray(x, dtype=np.float64))
-    W = {n: torch.as_tensor(np.asarray(a, dtype=np.float64)) for n, a in w.items()}
+    W = {n: rd(torch.as_tensor(np.asarray(a, dtype=np.float64))) for n, a in w.items()}
     T, h = X.shape
     d = h // n_heads
     xn = rd(Fn.layer_norm(X, (h,), eps=eps))
@@ -89,6 +105,28 @@ def test_round_bf16_matches_torch_cast_on_fp32_values():
     ref = vals.to(torch.bfloat16).to(torch.float64).numpy()
     got = O.round_bf16(vals.to(torch.float64).numpy())
     assert np.array_equal(got, ref)
+
+
+def test_round_fp16_matches_torch_cast_on_fp32_values():
+    g = torch.Generator().manual_seed(17)
+    vals = torch.cat([torch.randn(20000, generator=g) * s for s in (1e-6, 1e-4, 1.0, 300.0)])
+    bits = torch.randint(0, 1 << 20, (4000,), generator=g, dtype=torch.int64)
+    # fp32 values exactly halfway between halves, and next to halfway
+    base = ((bits << 13) & 0x0FFFE000) | 0x38000000
+    ties = torch.cat([base | 0x1000, base | 0x0FFF, base | 0x1001]).to(torch.int32).view(torch.float32)
+    vals = torch.cat([vals, ties, -ties])
+    ref = vals.to(torch.float16).to(torch.float64).numpy()
+    got = O.round_fp16(vals.to(torch.float64).numpy())
+    assert np.array_equal(got, ref)
+
+
+def test_round_fp16_direct_from_fp64():
+    assert O.round_fp16(np.array([1 + 2 ** -11 + 2 ** -40]))[0] == 1 + 2 ** -10  # just above a tie
+    assert O.round_fp16(np.array([1 + 2 ** -11]))[0] == 1.0                      # tie -> even
+    assert O.round_fp16(np.array([2 ** -25]))[0] == 0.0                          # subnormal tie -> even
+    assert O.round_fp16(np.array([3 * 2 ** -25]))[0] == 2 ** -23
+    x = np.random.default_rng(4).standard_normal(50000) * np.repeat([1e-6, 1e-3, 1.0, 50.0], 12500)
+    assert np.array_equal(O.round_fp16(x), fp16_rne_bits(torch.as_tensor(x)).numpy())
 
 
 def test_round_bf16_direct_from_fp64():
@@ -244,17 +282,18 @@ def test_attention_matches_sdpa_and_zigzag_rows():
 # whole layer against the independent torch composition
 # --------------------------------------------------------------------------
 @pytest.mark.parametrize("cfg,seed", [(TINY, 1), (SMALL, 0)])
-@pytest.mark.parametrize("bf16", [False, True])
-def test_layer_matches_torch_composition(cfg, seed, bf16):
+@pytest.mark.parametrize("storage", [None, "fp16", "bf16"])
+def test_layer_matches_torch_composition(cfg, seed, storage):
     x, w = tiny_inputs(cfg, seed)
-    got = O.layer_forward(x, w, cfg["H"], bf16_points=bf16)
-    ref = torch_layer(x, w, cfg["H"], bf16=bf16)
+    got = O.layer_forward(x, w, cfg["H"], storage=storage)
+    ref = torch_layer(x, w, cfg["H"], storage=storage)
     for key in ("k", "v", "a", "y1", "h", "y"):
         assert np.allclose(got[key], ref[key], rtol=1e-10, atol=1e-10), key
-    # the bf16 points really round: stored activations are bf16 numbers
-    if bf16:
+    # the storage points really round: stored operands are 16-bit numbers
+    if storage is not None:
+        rnd = O.round_fp16 if storage == "fp16" else O.round_bf16
         for key in ("xn1", "q", "a", "xn2", "h", "k", "v"):
-            assert np.array_equal(got[key], O.round_bf16(got[key])), key
+            assert np.array_equal(got[key], rnd(got[key])), key
 
 
 # --------------------------------------------------------------------------
@@ -278,8 +317,8 @@ def test_sharded_schedule_equals_unsharded_layer(D):
 def test_d1_reduces_to_plain_layer():
     cfg = TINY
     x, w = tiny_inputs(cfg, 31)
-    full = O.layer_forward(x, w, cfg["H"], bf16_points=False)
-    y = O.rank_forward_sharded(0, 1, x, full["k"], full["v"], w, cfg["H"], bf16_points=False)
+    full = O.layer_forward(x, w, cfg["H"], storage=None)
+    y = O.rank_forward_sharded(0, 1, x, full["k"], full["v"], w, cfg["H"], storage=None)
     assert np.allclose(y, full["y"], rtol=1e-12, atol=1e-12)
 
 
@@ -289,8 +328,8 @@ def test_d1_reduces_to_plain_layer():
 def _layer_error(monkeypatch_fn=None):
     cfg = TINY
     x, w = tiny_inputs(cfg, 41)
-    got = O.layer_forward(x, w, cfg["H"], bf16_points=False)
-    ref = torch_layer(x, w, cfg["H"], bf16=False)
+    got = O.layer_forward(x, w, cfg["H"], storage=None)
+    ref = torch_layer(x, w, cfg["H"], storage=None)
     return float(np.max(np.abs(got["y"] - ref["y"])))
 
 
