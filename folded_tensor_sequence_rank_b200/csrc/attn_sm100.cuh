@@ -19,10 +19,17 @@
 // head-major order makes the ~148 concurrent items stream the same head's
 // K/V so each tile is read from HBM about once and served from L2.
 //
-// Roles (192 threads, one CTA per SM, persistent):
+// Roles (320 threads, one CTA per SM, persistent):
 //   warp 0     work queue + TMA producer (Q tile, K ring, V ring)
 //   warp 1     TMEM allocator + single-thread tcgen05.mma issuer
-//   warps 2-5  softmax / correction / epilogue, one thread per query row
+//   warps 2-9  softmax / correction / epilogue.  Warp w reads TMEM lanes
+//              32*(w%4).. (its 32 query rows) and owns half (w-2)/4 of the
+//              128 key columns of each score tile and of the d output
+//              columns: two warps per row quarter, so each SM sub-partition
+//              interleaves two softmax warps.  Both compute the full row
+//              maximum (the lazy rescale must agree); each exponentiates and
+//              stores only its 64 columns; the two partial row sums are
+//              added once per work item through shared memory.
 // Tensor memory (512 columns): S0 | S1 (128 fp32 columns each, double
 // buffered scores), O (d fp32 columns), P0 | P1 (64 columns each: 128 fp16
 // probabilities packed in pairs, the A operand of O += P V).  Q, K, V and
@@ -36,7 +43,8 @@
 
 namespace tsp {
 
-constexpr int kAttnThreads = 192;
+constexpr int kAttnSoftmaxWarps = 8;
+constexpr int kAttnThreads = 64 + 32 * kAttnSoftmaxWarps;
 constexpr int kAttnBM = 128;
 constexpr int kAttnBN = 128;
 
@@ -61,7 +69,7 @@ struct AttnShape {
   static constexpr int kQBytes = kAttnBM * HD * 2;
   static constexpr int kKVBytes = kAttnBN * HD * 2;
   static constexpr int kStages = (HD == 128) ? 3 : 4;
-  static constexpr int kBarBytes = 512;
+  static constexpr int kBarBytes = 512 + 1024;  // barriers + row-sum exchange
   static constexpr int kSmemBytes = kQBytes + 2 * kStages * kKVBytes + kBarBytes + 1024;
   static constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
 };
@@ -119,9 +127,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
   uint64_t* it_full = o_free + 1;       // [2]
   uint64_t* it_empty = it_full + 2;     // [2]
   uint64_t* drain = it_empty + 2;
-  int* it_slot = reinterpret_cast<int*>(drain + 1);  // [2]
+  uint64_t* sum_bar = drain + 1;        // [4], one per row quarter: both halves' row sums written
+  int* it_slot = reinterpret_cast<int*>(sum_bar + 4);  // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(it_slot + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* red_sum = reinterpret_cast<float*>(bars) + 128;  // [2 halves][128 rows], after 512 B of barriers
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -137,14 +147,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], 4);
-      mbar_init(&p_full[b], 4);
+      mbar_init(&s_free[b], kAttnSoftmaxWarps);
+      mbar_init(&p_full[b], kAttnSoftmaxWarps);
       mbar_init(&o_done[b], 1);
       mbar_init(&it_full[b], 1);
-      mbar_init(&it_empty[b], 5);
+      mbar_init(&it_empty[b], 1 + kAttnSoftmaxWarps);
     }
-    mbar_init(o_free, 4);
+    mbar_init(o_free, kAttnSoftmaxWarps);
     mbar_init(drain, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(&sum_bar[q], 2);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -217,6 +228,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
       uint32_t g = 0;      // global score-tile counter (S/P buffer = g & 1)
       int items = 0;
       bool ok = true;
+      // S_gg = Q K^T into S buffer gg & 1; last = the item's final score tile
+      auto issue_s = [&](uint32_t gg, bool last) -> bool {
+        const int sb = gg & 1;
+        if (!mbar_wait(&s_free[sb], ((gg >> 1) & 1) ^ 1, ctl)) return false;
+        if (!mbar_wait(&k_full[ks], kph, ctl)) return false;
+        tc_fence_after();
+        const uint32_t q0 = smem_u32(sQ);
+        const uint32_t k0 = smem_u32(sK + ks * S::kKVBytes);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(tmem + S::kColS + sb * 128, smem_desc_sw128(q0 + off, 16, 1024),
+                 smem_desc_sw128(k0 + off, 16, 1024), idesc_s, kk != 0);
+        }
+        mma_commit(&k_empty[ks]);
+        mma_commit(&s_full[sb]);
+        if (last) mma_commit(q_empty);
+        if (++ks == STAGES) { ks = 0; kph ^= 1; }
+        return true;
+      };
       // O += P_gg V; first = first PV of the item (overwrites O)
       auto issue_pv = [&](uint32_t gg, bool first) -> bool {
         const int pb = gg & 1;
@@ -235,6 +266,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
         if (++vs == STAGES) { vs = 0; vph ^= 1; }
         return true;
       };
+      // Issue order per item: S_0, S_1, then for each tile j: S_{j+2}, PV_j.
+      // Scores run two tiles ahead of the softmax, so the tensor core computes
+      // S_{j+2} while the softmax works on tile j and PV_j follows as soon as
+      // P_j is written.
       for (int n = 0; ok; ++n) {
         const int slot = n & 1;
         if (!mbar_wait(&it_full[slot], (n >> 1) & 1, ctl)) break;
@@ -244,28 +279,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
         const AttnItem w = attn_decode(p, it);
         if (!mbar_wait(q_full, qph, ctl)) break;
         qph ^= 1;
-        tc_fence_after();
-        const uint32_t q0 = smem_u32(sQ);
-        for (int kt = 0; kt < w.nkv; ++kt, ++g) {
-          const int sb = g & 1;
-          if (!mbar_wait(&s_free[sb], ((g >> 1) & 1) ^ 1, ctl)) { ok = false; break; }
-          if (!mbar_wait(&k_full[ks], kph, ctl)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t k0 = smem_u32(sK + ks * S::kKVBytes);
-#pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_ss(tmem + S::kColS + sb * 128, smem_desc_sw128(q0 + off, 16, 1024),
-                   smem_desc_sw128(k0 + off, 16, 1024), idesc_s, kk != 0);
-          }
-          mma_commit(&k_empty[ks]);
-          mma_commit(&s_full[sb]);
-          if (++ks == STAGES) { ks = 0; kph ^= 1; }
-          if (kt == w.nkv - 1) mma_commit(q_empty);
-          if (kt > 0 && !issue_pv(g - 1, kt == 1)) { ok = false; break; }
+        const int pre = w.nkv < 2 ? w.nkv : 2;
+        for (int t = 0; ok && t < pre; ++t) ok = issue_s(g + t, t == w.nkv - 1);
+        for (int kt = 0; ok && kt < w.nkv; ++kt) {
+          if (kt + 2 < w.nkv) ok = issue_s(g + kt + 2, kt + 2 == w.nkv - 1);
+          if (ok) ok = issue_pv(g + kt, kt == 0);
         }
         if (!ok) break;
-        if (!issue_pv(g - 1, w.nkv == 1)) break;
+        g += w.nkv;
         ++items;
       }
       mma_commit(drain);
@@ -273,11 +294,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
     }
   } else {
     // ---------------------------------------------------------------- softmax
+    constexpr int HALF_D = HD / 2;
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const float sl2 = p.scale_log2;
     uint32_t g = 0;
+    uint32_t done_items = 0;
     for (int n = 0;; ++n) {
       const int slot = n & 1;
       if (!warp_wait(&it_full[slot], (n >> 1) & 1, ctl)) break;
@@ -289,35 +313,51 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
       const int qpos = w.p0 + row;
       const bool row_valid = row < w.nvalid;
       float m_used = -INFINITY;
-      float l = 0.f;
+      float l = 0.f;  // this warp's half of the row sum
       bool ok = true;
       for (int kt = 0; kt < w.nkv; ++kt, ++g) {
         const int sb = g & 1;
         if (!warp_wait(&s_full[sb], (g >> 1) & 1, ctl)) { ok = false; break; }
         tc_fence_after();
-        float s[kAttnBN];
+        // own[]: this warp's 64 key columns; oth[]: the partner warp's 64
+        uint32_t own[64], oth[64];
         {
-          uint32_t r[32];
-#pragma unroll
-          for (int j = 0; j < kAttnBN / 32; ++j) {
-            tmem_ld32(tmem + lane_off + S::kColS + sb * 128 + j * 32, r);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) s[j * 32 + i] = __uint_as_float(r[i]);
-          }
+          const uint32_t sbase = tmem + lane_off + S::kColS + sb * 128;
+          tmem_ld32p(sbase + half * 64, &own[0]);
+          tmem_ld32p(sbase + half * 64 + 32, &own[32]);
+          tmem_ld32p(sbase + (1 - half) * 64, &oth[0]);
+          tmem_ld32p(sbase + (1 - half) * 64 + 32, &oth[32]);
+          tmem_ld_wait();
+          reg_fence32(&own[0]);
+          reg_fence32(&own[32]);
+          reg_fence32(&oth[0]);
+          reg_fence32(&oth[32]);
         }
+        float* so = reinterpret_cast<float*>(own);
+        float* st = reinterpret_cast<float*>(oth);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[sb]);
         const int kbase = kt * kAttnBN;
         if (kbase + kAttnBN - 1 > w.p0) {
+          const int ko = kbase + half * 64, kx = kbase + (1 - half) * 64;
 #pragma unroll
-          for (int i = 0; i < kAttnBN; ++i)
-            if (kbase + i > qpos) s[i] = -INFINITY;
+          for (int i = 0; i < 64; ++i) {
+            if (ko + i > qpos) so[i] = -INFINITY;
+            if (kx + i > qpos) st[i] = -INFINITY;
+          }
         }
-        float mx = s[0];
+        float mx;
+        {  // full row maximum (both warps of the row quarter get the same value)
+          float m8[8];
 #pragma unroll
-        for (int i = 1; i < kAttnBN; ++i) mx = fmaxf(mx, s[i]);
+          for (int k = 0; k < 8; ++k) m8[k] = fmaxf(so[k], st[k]);
+#pragma unroll
+          for (int i = 8; i < 64; i += 8)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) m8[k] = fmax3(m8[k], so[i + k], st[i + k]);
+          mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+        }
         const float m_new = fmaxf(m_used, mx * sl2);
         const bool need = m_new > m_used + 8.0f;
         if (kt > 0 && __any_sync(0xffffffffu, need)) {
@@ -326,31 +366,46 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
           tc_fence_after();
           const float f = need ? ex2_approx(m_used - m_new) : 1.0f;
 #pragma unroll
-          for (int j = 0; j < HD / 32; ++j) {
+          for (int j = 0; j < HALF_D / 32; ++j) {
             uint32_t r[32];
-            tmem_ld32(tmem + lane_off + S::kColO + j * 32, r);
+            const uint32_t a = tmem + lane_off + S::kColO + half * HALF_D + j * 32;
+            tmem_ld32(a, r);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
-            tmem_st32(tmem + lane_off + S::kColO + j * 32, r);
+            tmem_st32(a, r);
           }
           if (need) l *= f;
         }
         if (need) m_used = m_new;
+        // P buffer g & 1 was last read by PV_{g-2}, which the tensor core may
+        // still be running (scores are issued ahead of it)
+        if (g >= 2 && !warp_wait(&o_done[g & 1], ((g - 2) >> 1) & 1, ctl)) { ok = false; break; }
         {
+          // this warp's 64 probabilities 2^(s*scale*log2e - m) as 32 pairs in
+          // f32x2 arithmetic; one pair in four on the FMA pipes (polynomial),
+          // the rest on MUFU; the partial row sum in two packed accumulators
           const int pb = g & 1;
+          const float neg_m = -m_used;
+          const float2 sl2v = make_float2(sl2, sl2), negm = make_float2(neg_m, neg_m);
+          float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
           uint32_t r[32];
 #pragma unroll
-          for (int j = 0; j < kAttnBN / 64; ++j) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float p0 = ex2_approx(fmaf(s[j * 64 + 2 * i], sl2, -m_used));
-              const float p1 = ex2_approx(fmaf(s[j * 64 + 2 * i + 1], sl2, -m_used));
-              l += p0 + p1;
-              r[i] = pack_half2(p0, p1);
+          for (int i = 0; i < 32; ++i) {
+            const float2 x = ffma2(make_float2(so[2 * i], so[2 * i + 1]), sl2v, negm);
+            float2 pr;
+            if ((i & 3) == 3) {
+              pr = exp2_poly2(x);
+            } else {
+              pr.x = ex2_approx(x.x);
+              pr.y = ex2_approx(x.y);
             }
-            tmem_st32(tmem + lane_off + S::kColP + pb * 64 + j * 32, r);
+            if (i & 1) lb = fadd2(lb, pr); else la = fadd2(la, pr);
+            r[i] = pack_half2(pr.x, pr.y);
           }
+          tmem_st32(tmem + lane_off + S::kColP + pb * 64 + half * 32, r);
+          const float2 lab = fadd2(la, lb);
+          l += lab.x + lab.y;
           tmem_st_wait();
           tc_fence_before();
           __syncwarp();
@@ -358,16 +413,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
         }
       }
       if (!ok) break;
-      // epilogue: O / l -> fp16 -> A[m0 + row, head]
+      // epilogue: row sum from both halves, then O / l -> fp16 -> A[m0 + row, head]
       const uint32_t gl = g - 1;
       if (!warp_wait(&o_done[gl & 1], (gl >> 1) & 1, ctl)) break;
       tc_fence_after();
-      const float inv = 1.0f / l;
-      __half* dst = p.out + static_cast<int64_t>(w.m0 + row) * p.ldo + w.head * HD;
+      red_sum[half * 128 + row] = l;
+      __threadfence_block();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sum_bar[quarter]);
+      if (!warp_wait(&sum_bar[quarter], done_items & 1, ctl)) break;
+      ++done_items;
+      const float inv = 1.0f / (red_sum[row] + red_sum[128 + row]);
+      __half* dst = p.out + static_cast<int64_t>(w.m0 + row) * p.ldo + w.head * HD + half * HALF_D;
 #pragma unroll
-      for (int j = 0; j < HD / 32; ++j) {
+      for (int j = 0; j < HALF_D / 32; ++j) {
         uint32_t r[32];
-        tmem_ld32(tmem + lane_off + S::kColO + j * 32, r);
+        tmem_ld32(tmem + lane_off + S::kColO + half * HALF_D + j * 32, r);
         tmem_ld_wait();
         if (row_valid) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + j * 32);

@@ -61,13 +61,14 @@ def assert_operand_close(g, e, what):
     that rounds the other way moves a K entry by up to ulp(xn) * |w| (about
     2e-4 here), so a rare entry lands two fp16 units away; the bound allows
     four units of the entry plus a floor of 2^-10 of the tensor's rms, and at
-    most 1e-4 of the entries may differ by more than one unit."""
+    most 1e-4 of the entries may differ by more than one unit plus 2^-12 of
+    the rms (near zero a unit is tiny, while these errors are absolute)."""
     scale = float(np.sqrt(np.mean(e * e)))
     diff = np.abs(g - e)
     ulp = np.maximum(2.0 ** (np.floor(np.log2(np.maximum(np.abs(e), 2.0 ** -14))) - 10), 2.0 ** -24)
     assert np.all(diff <= 4 * ulp + 2.0 ** -10 * scale), f"{what}: max {diff.max():.3e} (rms {scale:.3e})"
-    frac = float(np.mean(diff > ulp * 1.0000001))
-    assert frac <= 1e-4, f"{what}: {frac:.2e} of entries more than one unit off"
+    frac = float(np.mean(diff > ulp * 1.0000001 + 2.0 ** -12 * scale))
+    assert frac <= 1e-4, f"{what}: {frac:.2e} of entries more than one unit (plus floor) off"
     assert rel_l2(g, e) <= 1e-3, f"{what}: rel-L2 {rel_l2(g, e):.3e}"
 
 
