@@ -12,39 +12,44 @@
 // end are never loaded (chunk skipping).  Only tiles that reach past the
 // tile's first position apply the causal mask.
 //
-// Work item = (query tile, head).  Items are handed out through an atomic
-// counter in the order: heavy chunk (2D-1-r) first, head-major, descending
-// position; then the light chunk.  Heavy items come first so that the
-// greedy queue finishes balanced (longest-processing-time order), and
-// head-major order makes the ~148 concurrent items stream the same head's
-// K/V so each tile is read from HBM about once and served from L2.
+// Work item = (pair of adjacent query tiles of one chunk, head).  Both tiles
+// of a pair stream the same K/V tiles, so each K/V tile brought into shared
+// memory feeds two 128-row score tiles.  Items are handed out through an
+// atomic counter in the order: heavy chunk (2D-1-r) first, head-major,
+// descending position; then the light chunk.  Heavy items first makes the
+// greedy queue finish balanced (longest-processing-time order); head-major
+// order makes the ~148 concurrent items stream the same head's K/V, so each
+// K/V tile is read from HBM about once and then served from L2.
 //
 // Roles (320 threads, one CTA per SM, persistent):
-//   warp 0     work queue + TMA producer (Q tile, K ring, V ring)
+//   warp 0     work queue + TMA producer (Q_A, Q_B, K ring, V ring)
 //   warp 1     TMEM allocator + single-thread tcgen05.mma issuer
-//   warps 2-9  softmax / correction / epilogue.  Warp w reads TMEM lanes
-//              32*(w%4).. (its 32 query rows) and owns half (w-2)/4 of the
-//              128 key columns of each score tile and of the d output
-//              columns: two warps per row quarter, so each SM sub-partition
-//              interleaves two softmax warps.  Both compute the full row
-//              maximum (the lazy rescale must agree); each exponentiates and
-//              stores only its 64 columns; the two partial row sums are
-//              added once per work item through shared memory.
-// Tensor memory (512 columns): S0 | S1 (128 fp32 columns each, double
-// buffered scores), O (d fp32 columns), P0 | P1 (64 columns each: 128 fp16
-// probabilities packed in pairs, the A operand of O += P V).  Q, K, V and
-// the output are fp16; scores, the softmax statistics and O are fp32.
+//   warps 2-5  softmax, correction and epilogue of query tile A (thread = row)
+//   warps 6-9  the same for query tile B
+// Each SM sub-partition runs one warp of each tile.  The tensor core is fed
+// in the order S_A0 S_B0 | PV_A0 S_A1 PV_B0 S_B1 | PV_A1 S_A2 PV_B1 S_B2 ...,
+// so while one tile's softmax runs, the tensor core works on the other
+// tile's PV and next S, and the two softmax warps of a sub-partition work
+// out of phase.
+// Tensor memory (512 columns): [S_A / P_A | O_A | S_B / P_B | O_B], 128
+// columns each.  The softmax writes the fp16 probabilities P (64 columns, in
+// pairs) over the first half of its own score tile once the scores are in
+// registers; the next score tile of that query tile is issued after the
+// PV that reads P, and tcgen05.mma executes in issue order.  A finished
+// S_X(j) therefore also means PV_X(j-1) has finished, so the softmax may
+// rescale O_X with no further wait.
 // Online softmax in base 2 with a lazily updated row maximum: the running
 // output is rescaled only when the maximum grows by more than 2^8, which is
 // exact (the final division by the row sum cancels the common factor).
+// Q, K, V, P and the output are fp16; scores, softmax statistics and O are
+// fp32.
 #pragma once
 #include "gemm_sm100.cuh"
 #include "ptx.cuh"
 
 namespace tsp {
 
-constexpr int kAttnSoftmaxWarps = 8;
-constexpr int kAttnThreads = 64 + 32 * kAttnSoftmaxWarps;
+constexpr int kAttnThreads = 320;
 constexpr int kAttnBM = 128;
 constexpr int kAttnBN = 128;
 
@@ -57,7 +62,8 @@ struct __align__(64) AttnParams {
   int c;              // chunk length
   int rank, D, H;
   int nqt;            // query tiles per chunk
-  int n_items;        // 2 * nqt * H
+  int npairs;         // query-tile pairs per chunk, ceil(nqt / 2)
+  int n_items;        // 2 * npairs * H
   float scale_log2;   // softmax scale * log2(e)
   int* counter;       // work queue head (zeroed before launch)
   int* status;
@@ -68,29 +74,40 @@ template <int HD>
 struct AttnShape {
   static constexpr int kQBytes = kAttnBM * HD * 2;
   static constexpr int kKVBytes = kAttnBN * HD * 2;
-  static constexpr int kStages = (HD == 128) ? 3 : 4;
-  static constexpr int kBarBytes = 512 + 1024;  // barriers + row-sum exchange
-  static constexpr int kSmemBytes = kQBytes + 2 * kStages * kKVBytes + kBarBytes + 1024;
-  static constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
+  static constexpr int kKStages = (HD == 128) ? 3 : 4;
+  static constexpr int kVStages = (HD == 128) ? 2 : 4;
+  static constexpr int kBarBytes = 512;
+  static constexpr int kSmemBytes = 2 * kQBytes + (kKStages + kVStages) * kKVBytes + kBarBytes + 1024;
 };
 
+struct AttnTile {
+  int m0, p0, nvalid, nkv;  // nkv == 0: the tile does not exist
+};
 struct AttnItem {
-  int head, m0, p0, nvalid, nkv;
+  int head;
+  AttnTile t[2];
 };
 
 __device__ __forceinline__ AttnItem attn_decode(const AttnParams& p, int it) {
-  const int per_chunk = p.nqt * p.H;
+  const int per_chunk = p.npairs * p.H;
   const int heavy = it < per_chunk;
   const int ii = heavy ? it : it - per_chunk;
   AttnItem w;
-  w.head = ii / p.nqt;
-  const int t = p.nqt - 1 - (ii % p.nqt);
-  const int chunk_local = heavy ? 1 : 0;
+  w.head = ii / p.npairs;
+  const int pr = p.npairs - 1 - (ii % p.npairs);
   const int gchunk = heavy ? (2 * p.D - 1 - p.rank) : p.rank;
-  w.m0 = chunk_local * p.c + t * kAttnBM;
-  w.p0 = gchunk * p.c + t * kAttnBM;
-  w.nvalid = min(kAttnBM, p.c - t * kAttnBM);
-  w.nkv = (w.p0 + w.nvalid - 1) / kAttnBN + 1;
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    const int t = 2 * pr + x;
+    if (t < p.nqt) {
+      w.t[x].m0 = heavy * p.c + t * kAttnBM;
+      w.t[x].p0 = gchunk * p.c + t * kAttnBM;
+      w.t[x].nvalid = min(kAttnBM, p.c - t * kAttnBM);
+      w.t[x].nkv = (w.t[x].p0 + w.t[x].nvalid - 1) / kAttnBN + 1;
+    } else {
+      w.t[x].m0 = w.t[x].p0 = w.t[x].nvalid = w.t[x].nkv = 0;
+    }
+  }
   return w;
 }
 
@@ -105,57 +122,55 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
 template <int HD>
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid_constant__ AttnParams p) {
   using S = AttnShape<HD>;
-  constexpr int STAGES = S::kStages;
+  constexpr int KST = S::kKStages;
+  constexpr int VST = S::kVStages;
   constexpr int NB = HD / 64;  // 64-column (128-byte) boxes per row
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + S::kQBytes;
-  uint8_t* sV = sK + STAGES * S::kKVBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + STAGES * S::kKVBytes);
-  uint64_t* q_full = bars + 0;
-  uint64_t* q_empty = bars + 1;
-  uint64_t* k_full = bars + 2;
-  uint64_t* k_empty = k_full + STAGES;
-  uint64_t* v_full = k_empty + STAGES;
-  uint64_t* v_empty = v_full + STAGES;
-  uint64_t* s_full = v_empty + STAGES;  // [2]
-  uint64_t* s_free = s_full + 2;        // [2]
-  uint64_t* p_full = s_free + 2;        // [2]
-  uint64_t* o_done = p_full + 2;        // [2], by PV index parity
-  uint64_t* o_free = o_done + 2;
-  uint64_t* it_full = o_free + 1;       // [2]
-  uint64_t* it_empty = it_full + 2;     // [2]
+  uint8_t* sQ = smem;                       // [2][kQBytes]
+  uint8_t* sK = sQ + 2 * S::kQBytes;        // [KST][kKVBytes]
+  uint8_t* sV = sK + KST * S::kKVBytes;     // [VST][kKVBytes]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + VST * S::kKVBytes);
+  uint64_t* q_full = bars;                  // [2]
+  uint64_t* q_empty = q_full + 2;           // [2]
+  uint64_t* k_full = q_empty + 2;           // [KST]
+  uint64_t* k_empty = k_full + KST;         // [KST]
+  uint64_t* v_full = k_empty + KST;         // [VST]
+  uint64_t* v_empty = v_full + VST;         // [VST]
+  uint64_t* s_full = v_empty + VST;         // [2] score tile of query tile x ready
+  uint64_t* p_full = s_full + 2;            // [2] probabilities of tile x written
+  uint64_t* o_full = p_full + 2;            // [2] last PV of tile x done
+  uint64_t* o_free = o_full + 2;            // [2] epilogue of tile x has read O
+  uint64_t* it_full = o_free + 2;           // [2]
+  uint64_t* it_empty = it_full + 2;         // [2]
   uint64_t* drain = it_empty + 2;
-  uint64_t* sum_bar = drain + 1;        // [4], one per row quarter: both halves' row sums written
-  int* it_slot = reinterpret_cast<int*>(sum_bar + 4);  // [2]
+  int* it_slot = reinterpret_cast<int*>(drain + 1);  // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(it_slot + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* red_sum = reinterpret_cast<float*>(bars) + 128;  // [2 halves][128 rows], after 512 B of barriers
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
-    for (int s = 0; s < STAGES; ++s) {
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&q_full[x], 1);
+      mbar_init(&q_empty[x], 1);
+      mbar_init(&s_full[x], 1);
+      mbar_init(&p_full[x], 4);
+      mbar_init(&o_full[x], 1);
+      mbar_init(&o_free[x], 4);
+      mbar_init(&it_full[x], 1);
+      mbar_init(&it_empty[x], 9);
+    }
+    for (int s = 0; s < KST; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < VST; ++s) {
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], kAttnSoftmaxWarps);
-      mbar_init(&p_full[b], kAttnSoftmaxWarps);
-      mbar_init(&o_done[b], 1);
-      mbar_init(&it_full[b], 1);
-      mbar_init(&it_empty[b], 1 + kAttnSoftmaxWarps);
-    }
-    mbar_init(o_free, kAttnSoftmaxWarps);
     mbar_init(drain, 1);
-    for (int q = 0; q < 4; ++q) mbar_init(&sum_bar[q], 2);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -173,7 +188,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
       tma_prefetch_desc(&p.map_k);
       tma_prefetch_desc(&p.map_v);
       int ks = 0, vs = 0;
-      uint32_t kph = 0, vph = 0, qph = 0;
+      uint32_t kph = 0, vph = 0, qph[2] = {0, 0};
       uint32_t kused = 0, kpar = 0, vused = 0, vpar = 0, qused = 0, qpar = 0;
       bool ok = true;
       for (int n = 0; ok; ++n) {
@@ -186,14 +201,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
         if (it < 0) break;
         const AttnItem w = attn_decode(p, it);
         const int col0 = w.head * HD;
-        if (!mbar_wait(q_empty, qph ^ 1, ctl)) break;
-        mbar_arrive_expect_tx(q_full, S::kQBytes);
+        for (int x = 0; ok && x < 2; ++x) {
+          if (w.t[x].nkv == 0) continue;
+          if (!mbar_wait(&q_empty[x], qph[x] ^ 1, ctl)) { ok = false; break; }
+          mbar_arrive_expect_tx(&q_full[x], S::kQBytes);
 #pragma unroll
-        for (int b = 0; b < NB; ++b) tma_load_2d(sQ + b * 16384, &p.map_q, q_full, col0 + 64 * b, w.m0);
-        qused = 1;
-        qpar = qph;
-        qph ^= 1;
-        for (int kt = 0; kt < w.nkv; ++kt) {
+          for (int b = 0; b < NB; ++b)
+            tma_load_2d(sQ + x * S::kQBytes + b * 16384, &p.map_q, &q_full[x], col0 + 64 * b, w.t[x].m0);
+          qused |= 1u << x;
+          qpar = (qpar & ~(1u << x)) | (qph[x] << x);
+          qph[x] ^= 1;
+        }
+        const int nkv = max(w.t[0].nkv, w.t[1].nkv);
+        for (int kt = 0; ok && kt < nkv; ++kt) {
           if (!mbar_wait(&k_empty[ks], kph ^ 1, ctl)) { ok = false; break; }
           mbar_arrive_expect_tx(&k_full[ks], S::kKVBytes);
 #pragma unroll
@@ -201,7 +221,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
             tma_load_2d(sK + ks * S::kKVBytes + b * 16384, &p.map_k, &k_full[ks], col0 + 64 * b, kt * kAttnBN);
           kused |= 1u << ks;
           kpar = (kpar & ~(1u << ks)) | (kph << ks);
-          if (++ks == STAGES) { ks = 0; kph ^= 1; }
+          if (++ks == KST) { ks = 0; kph ^= 1; }
           if (!mbar_wait(&v_empty[vs], vph ^ 1, ctl)) { ok = false; break; }
           mbar_arrive_expect_tx(&v_full[vs], S::kKVBytes);
 #pragma unroll
@@ -209,14 +229,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
             tma_load_2d(sV + vs * S::kKVBytes + b * 16384, &p.map_v, &v_full[vs], col0 + 64 * b, kt * kAttnBN);
           vused |= 1u << vs;
           vpar = (vpar & ~(1u << vs)) | (vph << vs);
-          if (++vs == STAGES) { vs = 0; vph ^= 1; }
+          if (++vs == VST) { vs = 0; vph ^= 1; }
         }
       }
-      if (qused) mbar_drain(q_full, qpar, p.timeout_ns);
-      for (int s = 0; s < STAGES; ++s) {
+      for (int x = 0; x < 2; ++x)
+        if (qused & (1u << x)) mbar_drain(&q_full[x], (qpar >> x) & 1, p.timeout_ns);
+      for (int s = 0; s < KST; ++s)
         if (kused & (1u << s)) mbar_drain(&k_full[s], (kpar >> s) & 1, p.timeout_ns);
+      for (int s = 0; s < VST; ++s)
         if (vused & (1u << s)) mbar_drain(&v_full[s], (vpar >> s) & 1, p.timeout_ns);
-      }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -224,52 +245,47 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
       constexpr uint32_t idesc_s = idesc_f32acc(kAttnBM, kAttnBN, 0, 0, kFmtF16);
       constexpr uint32_t idesc_o = idesc_f32acc(kAttnBM, HD, 0, 1, kFmtF16);
       int ks = 0, vs = 0;
-      uint32_t kph = 0, vph = 0, qph = 0;
-      uint32_t g = 0;      // global score-tile counter (S/P buffer = g & 1)
-      int items = 0;
+      uint32_t kph = 0, vph = 0, qph[2] = {0, 0};
+      uint32_t pcnt[2] = {0, 0};  // probability tiles consumed, per query-tile slot
+      uint32_t icnt[2] = {0, 0};  // items finished, per query-tile slot
       bool ok = true;
-      // S_gg = Q K^T into S buffer gg & 1; last = the item's final score tile
-      auto issue_s = [&](uint32_t gg, bool last) -> bool {
-        const int sb = gg & 1;
-        if (!mbar_wait(&s_free[sb], ((gg >> 1) & 1) ^ 1, ctl)) return false;
-        if (!mbar_wait(&k_full[ks], kph, ctl)) return false;
-        tc_fence_after();
-        const uint32_t q0 = smem_u32(sQ);
+      // S_x = Q_x K^T for the K tile in slot ks
+      auto issue_s = [&](int x, bool last_s) {
+        const uint32_t q0 = smem_u32(sQ + x * S::kQBytes);
         const uint32_t k0 = smem_u32(sK + ks * S::kKVBytes);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tmem + S::kColS + sb * 128, smem_desc_sw128(q0 + off, 16, 1024),
-                 smem_desc_sw128(k0 + off, 16, 1024), idesc_s, kk != 0);
+          mma_ss(tmem + x * 256, smem_desc_sw128(q0 + off, 16, 1024), smem_desc_sw128(k0 + off, 16, 1024), idesc_s,
+                 kk != 0);
         }
-        mma_commit(&k_empty[ks]);
-        mma_commit(&s_full[sb]);
-        if (last) mma_commit(q_empty);
-        if (++ks == STAGES) { ks = 0; kph ^= 1; }
-        return true;
+        mma_commit(&s_full[x]);
+        if (last_s) mma_commit(&q_empty[x]);
       };
-      // O += P_gg V; first = first PV of the item (overwrites O)
-      auto issue_pv = [&](uint32_t gg, bool first) -> bool {
-        const int pb = gg & 1;
-        if (first && !mbar_wait(o_free, (items & 1) ^ 1, ctl)) return false;
-        if (!mbar_wait(&p_full[pb], (gg >> 1) & 1, ctl)) return false;
-        if (!mbar_wait(&v_full[vs], vph, ctl)) return false;
+      // O_x += P_x V for the V tile in slot vs
+      auto issue_pv = [&](int x, bool first, bool last) -> bool {
+        if (first && !mbar_wait(&o_free[x], (icnt[x] & 1) ^ 1, ctl)) return false;
+        if (!mbar_wait(&p_full[x], pcnt[x] & 1, ctl)) return false;
+        ++pcnt[x];
         tc_fence_after();
         const uint32_t v0 = smem_u32(sV + vs * S::kKVBytes);
 #pragma unroll
         for (int kk = 0; kk < kAttnBN / 16; ++kk) {
           const uint64_t bd = smem_desc_sw128(v0 + kk * 2048, 16384, 1024);
-          mma_ts(tmem + S::kColO, tmem + S::kColP + pb * 64 + kk * 8, bd, idesc_o, !(first && kk == 0));
+          mma_ts(tmem + x * 256 + 128, tmem + x * 256 + kk * 8, bd, idesc_o, !(first && kk == 0));
         }
-        mma_commit(&v_empty[vs]);
-        mma_commit(&o_done[gg & 1]);
-        if (++vs == STAGES) { vs = 0; vph ^= 1; }
+        if (last) mma_commit(&o_full[x]);
         return true;
       };
-      // Issue order per item: S_0, S_1, then for each tile j: S_{j+2}, PV_j.
-      // Scores run two tiles ahead of the softmax, so the tensor core computes
-      // S_{j+2} while the softmax works on tile j and PV_j follows as soon as
-      // P_j is written.
+      auto wait_k = [&]() -> bool {
+        if (!mbar_wait(&k_full[ks], kph, ctl)) return false;
+        tc_fence_after();
+        return true;
+      };
+      auto release_k = [&]() {
+        mma_commit(&k_empty[ks]);
+        if (++ks == KST) { ks = 0; kph ^= 1; }
+      };
       for (int n = 0; ok; ++n) {
         const int slot = n & 1;
         if (!mbar_wait(&it_full[slot], (n >> 1) & 1, ctl)) break;
@@ -277,31 +293,62 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
         mbar_arrive(&it_empty[slot]);
         if (it < 0) break;
         const AttnItem w = attn_decode(p, it);
-        if (!mbar_wait(q_full, qph, ctl)) break;
-        qph ^= 1;
-        const int pre = w.nkv < 2 ? w.nkv : 2;
-        for (int t = 0; ok && t < pre; ++t) ok = issue_s(g + t, t == w.nkv - 1);
-        for (int kt = 0; ok && kt < w.nkv; ++kt) {
-          if (kt + 2 < w.nkv) ok = issue_s(g + kt + 2, kt + 2 == w.nkv - 1);
-          if (ok) ok = issue_pv(g + kt, kt == 0);
+        const int na = w.t[0].nkv, nb = w.t[1].nkv;
+        const int nkv = max(na, nb);
+        for (int x = 0; ok && x < 2; ++x) {
+          if (w.t[x].nkv == 0) continue;
+          ok = mbar_wait(&q_full[x], qph[x], ctl);
+          qph[x] ^= 1;
         }
         if (!ok) break;
-        g += w.nkv;
-        ++items;
+        tc_fence_after();
+        // scores of K tile 0 for both query tiles
+        if (!wait_k()) break;
+        if (na > 0) issue_s(0, na == 1);
+        if (nb > 0) issue_s(1, nb == 1);
+        release_k();
+        for (int kt = 0; ok && kt < nkv; ++kt) {
+          if (!mbar_wait(&v_full[vs], vph, ctl)) { ok = false; break; }
+          bool k_waited = false;
+          if (kt < na) {
+            if (!issue_pv(0, kt == 0, kt == na - 1)) { ok = false; break; }
+            if (kt + 1 < na) {
+              if (!wait_k()) { ok = false; break; }
+              k_waited = true;
+              issue_s(0, kt + 1 == na - 1);
+            }
+          }
+          if (kt < nb) {
+            if (!issue_pv(1, kt == 0, kt == nb - 1)) { ok = false; break; }
+            if (kt + 1 < nb) {
+              if (!k_waited) {
+                if (!wait_k()) { ok = false; break; }
+                k_waited = true;
+              }
+              issue_s(1, kt + 1 == nb - 1);
+            }
+          }
+          if (k_waited) release_k();
+          mma_commit(&v_empty[vs]);
+          if (++vs == VST) { vs = 0; vph ^= 1; }
+        }
+        if (!ok) break;
+        for (int x = 0; x < 2; ++x)
+          if (w.t[x].nkv > 0) ++icnt[x];
       }
       mma_commit(drain);
       mbar_drain(drain, 0, p.timeout_ns);
     }
   } else {
     // ---------------------------------------------------------------- softmax
-    constexpr int HALF_D = HD / 2;
-    const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int x = (warp - 2) >> 2;     // query tile of this warp group
+    const int quarter = warp & 3;      // TMEM lane quarter = rows 32*quarter ..
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t t_s = tmem + lane_off + x * 256;        // S / P of this tile
+    const uint32_t t_o = tmem + lane_off + x * 256 + 128;  // O of this tile
     const float sl2 = p.scale_log2;
-    uint32_t g = 0;
-    uint32_t done_items = 0;
+    uint32_t scnt = 0, icnt = 0;
     for (int n = 0;; ++n) {
       const int slot = n & 1;
       if (!warp_wait(&it_full[slot], (n >> 1) & 1, ctl)) break;
@@ -310,125 +357,116 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
       if (lane == 0) mbar_arrive(&it_empty[slot]);
       if (it < 0) break;
       const AttnItem w = attn_decode(p, it);
-      const int qpos = w.p0 + row;
-      const bool row_valid = row < w.nvalid;
+      const AttnTile T = w.t[x];
+      if (T.nkv == 0) continue;
+      const int qpos = T.p0 + row;
+      const bool row_valid = row < T.nvalid;
       float m_used = -INFINITY;
-      float l = 0.f;  // this warp's half of the row sum
+      float l = 0.f;
       bool ok = true;
-      for (int kt = 0; kt < w.nkv; ++kt, ++g) {
-        const int sb = g & 1;
-        if (!warp_wait(&s_full[sb], (g >> 1) & 1, ctl)) { ok = false; break; }
+      for (int kt = 0; kt < T.nkv; ++kt) {
+        if (!warp_wait(&s_full[x], scnt & 1, ctl)) { ok = false; break; }
+        ++scnt;
         tc_fence_after();
-        // own[]: this warp's 64 key columns; oth[]: the partner warp's 64
-        uint32_t own[64], oth[64];
-        {
-          const uint32_t sbase = tmem + lane_off + S::kColS + sb * 128;
-          tmem_ld32p(sbase + half * 64, &own[0]);
-          tmem_ld32p(sbase + half * 64 + 32, &own[32]);
-          tmem_ld32p(sbase + (1 - half) * 64, &oth[0]);
-          tmem_ld32p(sbase + (1 - half) * 64 + 32, &oth[32]);
-          tmem_ld_wait();
-          reg_fence32(&own[0]);
-          reg_fence32(&own[32]);
-          reg_fence32(&oth[0]);
-          reg_fence32(&oth[32]);
-        }
-        float* so = reinterpret_cast<float*>(own);
-        float* st = reinterpret_cast<float*>(oth);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_free[sb]);
         const int kbase = kt * kAttnBN;
-        if (kbase + kAttnBN - 1 > w.p0) {
-          const int ko = kbase + half * 64, kx = kbase + (1 - half) * 64;
-#pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            if (ko + i > qpos) so[i] = -INFINITY;
-            if (kx + i > qpos) st[i] = -INFINITY;
-          }
-        }
+        const bool diag = kbase + kAttnBN - 1 > T.p0;  // some key may lie past this row
         float mx;
-        {  // full row maximum (both warps of the row quarter get the same value)
+        {  // pass 1: the row maximum over all 128 scores (8 chains of 3-input max)
+          uint32_t sr[kAttnBN];
+#pragma unroll
+          for (int j = 0; j < kAttnBN / 32; ++j) tmem_ld32p(t_s + j * 32, &sr[j * 32]);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < kAttnBN / 32; ++j) reg_fence32(&sr[j * 32]);
+          float* s = reinterpret_cast<float*>(sr);
+          if (diag) {
+#pragma unroll
+            for (int i = 0; i < kAttnBN; ++i)
+              if (kbase + i > qpos) s[i] = -INFINITY;
+          }
           float m8[8];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) m8[k] = fmaxf(so[k], st[k]);
+          for (int k = 0; k < 8; ++k) m8[k] = fmaxf(s[k], s[k + 8]);
 #pragma unroll
-          for (int i = 8; i < 64; i += 8)
+          for (int i = 16; i < kAttnBN; i += 16)
 #pragma unroll
-            for (int k = 0; k < 8; ++k) m8[k] = fmax3(m8[k], so[i + k], st[i + k]);
+            for (int k = 0; k < 8; ++k) m8[k] = fmax3(m8[k], s[i + k], s[i + k + 8]);
           mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
         }
         const float m_new = fmaxf(m_used, mx * sl2);
         const bool need = m_new > m_used + 8.0f;
         if (kt > 0 && __any_sync(0xffffffffu, need)) {
-          // the previous P V product must land before O is rescaled
-          if (!warp_wait(&o_done[(g - 1) & 1], ((g - 1) >> 1) & 1, ctl)) { ok = false; break; }
-          tc_fence_after();
+          // S_x(kt) finished, so PV_x(kt-1) has too: O may be rescaled now
           const float f = need ? ex2_approx(m_used - m_new) : 1.0f;
 #pragma unroll
-          for (int j = 0; j < HALF_D / 32; ++j) {
+          for (int j = 0; j < HD / 32; ++j) {
             uint32_t r[32];
-            const uint32_t a = tmem + lane_off + S::kColO + half * HALF_D + j * 32;
-            tmem_ld32(a, r);
+            tmem_ld32(t_o + j * 32, r);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
-            tmem_st32(a, r);
+            tmem_st32(t_o + j * 32, r);
           }
           if (need) l *= f;
         }
         if (need) m_used = m_new;
-        // P buffer g & 1 was last read by PV_{g-2}, which the tensor core may
-        // still be running (scores are issued ahead of it)
-        if (g >= 2 && !warp_wait(&o_done[g & 1], ((g - 2) >> 1) & 1, ctl)) { ok = false; break; }
         {
-          // this warp's 64 probabilities 2^(s*scale*log2e - m) as 32 pairs in
-          // f32x2 arithmetic; one pair in four on the FMA pipes (polynomial),
-          // the rest on MUFU; the partial row sum in two packed accumulators
-          const int pb = g & 1;
+          // pass 2: probabilities 2^(s*scale*log2e - m), 64 scores at a time,
+          // as pairs in f32x2 arithmetic; one pair in four on the FMA pipes
+          // (polynomial), the rest on MUFU.  Keys 64h.. 64h+63 become fp16
+          // pairs in columns 32h .. 32h+31, over scores already consumed.
           const float neg_m = -m_used;
           const float2 sl2v = make_float2(sl2, sl2), negm = make_float2(neg_m, neg_m);
           float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
-          uint32_t r[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float2 x = ffma2(make_float2(so[2 * i], so[2 * i + 1]), sl2v, negm);
-            float2 pr;
-            if ((i & 3) == 3) {
-              pr = exp2_poly2(x);
-            } else {
-              pr.x = ex2_approx(x.x);
-              pr.y = ex2_approx(x.y);
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t sr[64];
+            tmem_ld32p(t_s + hh * 64, &sr[0]);
+            tmem_ld32p(t_s + hh * 64 + 32, &sr[32]);
+            tmem_ld_wait();
+            reg_fence32(&sr[0]);
+            reg_fence32(&sr[32]);
+            float* s = reinterpret_cast<float*>(sr);
+            if (diag) {
+#pragma unroll
+              for (int i = 0; i < 64; ++i)
+                if (kbase + hh * 64 + i > qpos) s[i] = -INFINITY;
             }
-            if (i & 1) lb = fadd2(lb, pr); else la = fadd2(la, pr);
-            r[i] = pack_half2(pr.x, pr.y);
+            uint32_t r[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float2 xv = ffma2(make_float2(s[2 * i], s[2 * i + 1]), sl2v, negm);
+              float2 pr;
+              if ((i & 3) == 3) {
+                pr = exp2_poly2(xv);
+              } else {
+                pr.x = ex2_approx(xv.x);
+                pr.y = ex2_approx(xv.y);
+              }
+              if (i & 1) lb = fadd2(lb, pr); else la = fadd2(la, pr);
+              r[i] = pack_half2(pr.x, pr.y);
+            }
+            tmem_st32(t_s + hh * 32, r);
           }
-          tmem_st32(tmem + lane_off + S::kColP + pb * 64 + half * 32, r);
           const float2 lab = fadd2(la, lb);
           l += lab.x + lab.y;
           tmem_st_wait();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&p_full[pb]);
+          if (lane == 0) mbar_arrive(&p_full[x]);
         }
       }
       if (!ok) break;
-      // epilogue: row sum from both halves, then O / l -> fp16 -> A[m0 + row, head]
-      const uint32_t gl = g - 1;
-      if (!warp_wait(&o_done[gl & 1], (gl >> 1) & 1, ctl)) break;
+      // epilogue: O / l -> fp16 -> A[m0 + row, head]
+      if (!warp_wait(&o_full[x], icnt & 1, ctl)) break;
+      ++icnt;
       tc_fence_after();
-      red_sum[half * 128 + row] = l;
-      __threadfence_block();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sum_bar[quarter]);
-      if (!warp_wait(&sum_bar[quarter], done_items & 1, ctl)) break;
-      ++done_items;
-      const float inv = 1.0f / (red_sum[row] + red_sum[128 + row]);
-      __half* dst = p.out + static_cast<int64_t>(w.m0 + row) * p.ldo + w.head * HD + half * HALF_D;
+      const float inv = 1.0f / l;
+      __half* dst = p.out + static_cast<int64_t>(T.m0 + row) * p.ldo + w.head * HD;
 #pragma unroll
-      for (int j = 0; j < HALF_D / 32; ++j) {
+      for (int j = 0; j < HD / 32; ++j) {
         uint32_t r[32];
-        tmem_ld32(tmem + lane_off + S::kColO + half * HALF_D + j * 32, r);
+        tmem_ld32(t_o + j * 32, r);
         tmem_ld_wait();
         if (row_valid) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + j * 32);
@@ -443,7 +481,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(o_free);
+      if (lane == 0) mbar_arrive(&o_free[x]);
     }
   }
 

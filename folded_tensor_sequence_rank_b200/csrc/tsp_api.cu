@@ -288,7 +288,8 @@ int launch_attention(const Sizes& s, int rank, const tsp_dims* dims, const __hal
   p.D = s.D;
   p.H = s.H;
   p.nqt = static_cast<int>((s.c + kAttnBM - 1) / kAttnBM);
-  p.n_items = 2 * p.nqt * s.H;
+  p.npairs = (p.nqt + 1) / 2;
+  p.n_items = 2 * p.npairs * s.H;
   p.scale_log2 = dims->softmax_scale * 1.4426950408889634f;
   p.counter = counter;
   p.status = status;
