@@ -107,9 +107,8 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------------- dist
 def dist_setup(n_gpus):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from folded_tensor_sequence_rank_b200 import dist as tdist
+    world, rank, local = tdist.world_info()
     if world != n_gpus and world > 1:
         raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
     return world, rank, local
@@ -215,6 +214,7 @@ def run_tsp(args, wl):
     import torch
     import torch.distributed as dist
 
+    from folded_tensor_sequence_rank_b200 import dist as tdist
     from folded_tensor_sequence_rank_b200 import tsp
 
     world, grank, local = dist_setup(args.gpus)
@@ -223,7 +223,7 @@ def run_tsp(args, wl):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
     T, h, H, F, D = wl["T"], wl["h"], wl["H"], wl["F"], wl["D"]
-    trank = grank % D
+    trank = tdist.tsp_rank_for(grank, D)
     L = T // D
     dims = tsp.make_dims(T, h, H, F)
     tsp.lib()
@@ -295,12 +295,7 @@ def run_tsp(args, wl):
     e2e_ms = e0.elapsed_time(e1) / args.steps
     assert tsp.get_device_status(ws) == tsp.TSP_OK, "device wait timed out"
 
-    if world > 1:
-        t = torch.tensor([ms, e2e_ms, step_ms["attention"]], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_ms, attn_ms = t.tolist()
-    else:
-        attn_ms = step_ms["attention"]
+    ms, e2e_ms, attn_ms = tdist.max_over_ranks([ms, e2e_ms, step_ms["attention"]], device="cuda")
 
     if grank == 0:
         pk, src = peaks()

@@ -249,31 +249,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
       uint32_t pcnt[2] = {0, 0};  // probability tiles consumed, per query-tile slot
       uint32_t icnt[2] = {0, 0};  // items finished, per query-tile slot
       bool ok = true;
-      // S_x = Q_x K^T for the K tile in slot ks
+      // Shared-memory descriptors of every Q and K/V stage, built once; an MMA
+      // group then only adds immediate offsets (see mma_ss_x8 / mma_ts_x8).
+      const uint64_t qdesc0 = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t kdesc0 = smem_desc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t vdesc0 = smem_desc_sw128(smem_u32(sV), 16384, 1024);
+      auto qdesc = [&](int x) { return qdesc0 + static_cast<uint64_t>(x * (S::kQBytes >> 4)); };
+      auto kdesc = [&]() { return kdesc0 + static_cast<uint64_t>(ks * (S::kKVBytes >> 4)); };
+      auto vdesc = [&]() { return vdesc0 + static_cast<uint64_t>(vs * (S::kKVBytes >> 4)); };
+      // S_x = Q_x K^T for the K tile in slot ks (K = head_dim in 16-column steps:
+      // +32 bytes inside a 128-byte swizzle row, +16 KiB to the next 64 columns)
       auto issue_s = [&](int x, bool last_s) {
-        const uint32_t q0 = smem_u32(sQ + x * S::kQBytes);
-        const uint32_t k0 = smem_u32(sK + ks * S::kKVBytes);
+        if constexpr (HD == 128) {
+          mma_ss_x8<0, 2, 4, 6, 1024, 1026, 1028, 1030>(tmem + x * 256, qdesc(x), kdesc(), idesc_s, 0);
+        } else {
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tmem + x * 256, smem_desc_sw128(q0 + off, 16, 1024), smem_desc_sw128(k0 + off, 16, 1024), idesc_s,
-                 kk != 0);
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+            mma_ss(tmem + x * 256, qdesc(x) + off, kdesc() + off, idesc_s, kk != 0);
+          }
         }
         mma_commit(&s_full[x]);
         if (last_s) mma_commit(&q_empty[x]);
       };
-      // O_x += P_x V for the V tile in slot vs
+      // O_x += P_x V for the V tile in slot vs (K = 128 keys in 16-key steps:
+      // P advances 8 TMEM columns, V 2 KiB = 128 units)
       auto issue_pv = [&](int x, bool first, bool last) -> bool {
         if (first && !mbar_wait(&o_free[x], (icnt[x] & 1) ^ 1, ctl)) return false;
         if (!mbar_wait(&p_full[x], pcnt[x] & 1, ctl)) return false;
         ++pcnt[x];
         tc_fence_after();
-        const uint32_t v0 = smem_u32(sV + vs * S::kKVBytes);
-#pragma unroll
-        for (int kk = 0; kk < kAttnBN / 16; ++kk) {
-          const uint64_t bd = smem_desc_sw128(v0 + kk * 2048, 16384, 1024);
-          mma_ts(tmem + x * 256 + 128, tmem + x * 256 + kk * 8, bd, idesc_o, !(first && kk == 0));
-        }
+        mma_ts_x8<128>(tmem + x * 256 + 128, tmem + x * 256, vdesc(), idesc_o, first ? 0u : 1u);
         if (last) mma_commit(&o_full[x]);
         return true;
       };
@@ -370,72 +376,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
         tc_fence_after();
         const int kbase = kt * kAttnBN;
         const bool diag = kbase + kAttnBN - 1 > T.p0;  // some key may lie past this row
-        float mx;
-        {  // pass 1: the row maximum over all 128 scores (8 chains of 3-input max)
-          uint32_t sr[kAttnBN];
-#pragma unroll
-          for (int j = 0; j < kAttnBN / 32; ++j) tmem_ld32p(t_s + j * 32, &sr[j * 32]);
+        // Loads scores [64 hh, 64 hh + 64) and returns their maximum (masked
+        // keys -> -inf); with `exps`, also writes the probabilities
+        // 2^(s*scale*log2e - m) as fp16 pairs into P (one pair in four by the
+        // polynomial on the FMA pipes, the rest on MUFU) and adds them to la/lb.
+        auto half_tile = [&](int hh, bool exps, float neg_m, uint32_t (&P)[32], float2& la, float2& lb) -> float {
+          uint32_t sr[64];
+          tmem_ld32p(t_s + hh * 64, &sr[0]);
+          tmem_ld32p(t_s + hh * 64 + 32, &sr[32]);
           tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < kAttnBN / 32; ++j) reg_fence32(&sr[j * 32]);
-          float* s = reinterpret_cast<float*>(sr);
+          reg_fence32(&sr[0]);
+          reg_fence32(&sr[32]);
+          float* sv = reinterpret_cast<float*>(sr);
           if (diag) {
 #pragma unroll
-            for (int i = 0; i < kAttnBN; ++i)
-              if (kbase + i > qpos) s[i] = -INFINITY;
+            for (int i = 0; i < 64; ++i)
+              if (kbase + hh * 64 + i > qpos) sv[i] = -INFINITY;
           }
-          float m8[8];
+          float m4[4];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) m8[k] = fmaxf(s[k], s[k + 8]);
+          for (int k = 0; k < 4; ++k) m4[k] = fmaxf(sv[k], sv[k + 4]);
 #pragma unroll
-          for (int i = 16; i < kAttnBN; i += 16)
+          for (int i = 8; i < 64; i += 8)
 #pragma unroll
-            for (int k = 0; k < 8; ++k) m8[k] = fmax3(m8[k], s[i + k], s[i + k + 8]);
-          mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
-        }
-        const float m_new = fmaxf(m_used, mx * sl2);
-        const bool need = m_new > m_used + 8.0f;
-        if (kt > 0 && __any_sync(0xffffffffu, need)) {
-          // S_x(kt) finished, so PV_x(kt-1) has too: O may be rescaled now
-          const float f = need ? ex2_approx(m_used - m_new) : 1.0f;
-#pragma unroll
-          for (int j = 0; j < HD / 32; ++j) {
-            uint32_t r[32];
-            tmem_ld32(t_o + j * 32, r);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
-            tmem_st32(t_o + j * 32, r);
-          }
-          if (need) l *= f;
-        }
-        if (need) m_used = m_new;
-        {
-          // pass 2: probabilities 2^(s*scale*log2e - m), 64 scores at a time,
-          // as pairs in f32x2 arithmetic; one pair in four on the FMA pipes
-          // (polynomial), the rest on MUFU.  Keys 64h.. 64h+63 become fp16
-          // pairs in columns 32h .. 32h+31, over scores already consumed.
-          const float neg_m = -m_used;
-          const float2 sl2v = make_float2(sl2, sl2), negm = make_float2(neg_m, neg_m);
-          float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            uint32_t sr[64];
-            tmem_ld32p(t_s + hh * 64, &sr[0]);
-            tmem_ld32p(t_s + hh * 64 + 32, &sr[32]);
-            tmem_ld_wait();
-            reg_fence32(&sr[0]);
-            reg_fence32(&sr[32]);
-            float* s = reinterpret_cast<float*>(sr);
-            if (diag) {
-#pragma unroll
-              for (int i = 0; i < 64; ++i)
-                if (kbase + hh * 64 + i > qpos) s[i] = -INFINITY;
-            }
-            uint32_t r[32];
+            for (int k = 0; k < 4; ++k) m4[k] = fmax3(m4[k], sv[i + k], sv[i + k + 4]);
+          if (exps) {
+            const float2 sl2v = make_float2(sl2, sl2), negm = make_float2(neg_m, neg_m);
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-              const float2 xv = ffma2(make_float2(s[2 * i], s[2 * i + 1]), sl2v, negm);
+              const float2 xv = ffma2(make_float2(sv[2 * i], sv[2 * i + 1]), sl2v, negm);
               float2 pr;
               if ((i & 3) == 3) {
                 pr = exp2_poly2(xv);
@@ -444,17 +413,57 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
                 pr.y = ex2_approx(xv.y);
               }
               if (i & 1) lb = fadd2(lb, pr); else la = fadd2(la, pr);
-              r[i] = pack_half2(pr.x, pr.y);
+              P[i] = pack_half2(pr.x, pr.y);
             }
-            tmem_st32(t_s + hh * 32, r);
           }
-          const float2 lab = fadd2(la, lb);
-          l += lab.x + lab.y;
-          tmem_st_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&p_full[x]);
+          return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        };
+        uint32_t P0[32], P1[32];
+        float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
+        if (kt == 0) {
+          // first key tile of the item: row maximum first, then probabilities
+          const float mx = fmaxf(half_tile(0, false, 0.f, P0, la, lb), half_tile(1, false, 0.f, P1, la, lb));
+          m_used = mx * sl2;
+          half_tile(0, true, -m_used, P0, la, lb);
+          half_tile(1, true, -m_used, P1, la, lb);
+        } else {
+          // Speculate that the row maximum did not grow by more than 2^8 and
+          // compute P with the current one; P stays in registers (the scores
+          // stay intact in TMEM) until the check below.
+          const float mx = fmaxf(half_tile(0, true, -m_used, P0, la, lb), half_tile(1, true, -m_used, P1, la, lb));
+          const float m_new = fmaxf(m_used, mx * sl2);
+          const bool need = m_new > m_used + 8.0f;
+          if (__any_sync(0xffffffffu, need)) {
+            // rare: rescale O and l to the new maximum, then recompute P.
+            // S_x(kt) finished, so PV_x(kt-1) has too: O may be rescaled now.
+            const float f = need ? ex2_approx(m_used - m_new) : 1.0f;
+#pragma unroll
+            for (int j = 0; j < HD / 32; ++j) {
+              uint32_t r[32];
+              tmem_ld32(t_o + j * 32, r);
+              tmem_ld_wait();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
+              tmem_st32(t_o + j * 32, r);
+            }
+            l *= f;
+            if (need) m_used = m_new;
+            la = make_float2(0.f, 0.f);
+            lb = make_float2(0.f, 0.f);
+            half_tile(0, true, -m_used, P0, la, lb);
+            half_tile(1, true, -m_used, P1, la, lb);
+          }
         }
+        // keys 0..63 -> columns 0..31, keys 64..127 -> columns 32..63, over
+        // scores already consumed
+        tmem_st32(t_s, P0);
+        tmem_st32(t_s + 32, P1);
+        const float2 lab = fadd2(la, lb);
+        l += lab.x + lab.y;
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[x]);
       }
       if (!ok) break;
       // epilogue: O / l -> fp16 -> A[m0 + row, head]

@@ -15,7 +15,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/tsp.h"
+#include "tsp.h"
 #include "attn_sm100.cuh"
 #include "gemm_sm100.cuh"
 #include "misc_kernels.cuh"
