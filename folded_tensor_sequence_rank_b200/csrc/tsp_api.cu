@@ -20,6 +20,9 @@
 #include "gemm_sm100.cuh"
 #include "misc_kernels.cuh"
 
+// File-scope scratch of tsp_kv_project_noalloc (see noalloc_scratch below).
+static __device__ __align__(256) uint8_t g_noalloc_scratch[size_t(64) << 20];
+
 namespace {
 
 using namespace tsp;
@@ -381,6 +384,34 @@ int layer_tail(Ctx& c, const tsp_dims* dims, const tsp_weights* w, int rank, con
   return record(ev, 7, st);
 }
 
+// ---------------------------------------------------------------- allocation-free K/V projection
+// Scratch for tsp_kv_project_noalloc: a file-scope device array, so the call
+// needs no device allocation.  Layout: status word (256 B), 768 B spare, then
+// the LN1 output xn fp16 [L, h].  Every GPU that loads this library holds the
+// array until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
+constexpr size_t kNoAllocXnOffset = 1024;
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[256] = {};  // device address of the array, per device ordinal
+
+// In host code the array's name is only a host-side stand-in: the device
+// address comes from cudaGetSymbolAddress, looked up once per device with that
+// device current (the first call on a device does this lookup).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  TSP_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 256) return TSP_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    TSP_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return TSP_OK;
+}
+
 }  // namespace
 
 // ============================================================================
@@ -504,6 +535,40 @@ int tsp_kv_project(const tsp_dims* dims, const tsp_weights* w, int rank, const v
   void* out[3] = {k_full, v_full, nullptr};
   const int remap[3] = {1, 1, 0};
   return launch_proj(c.s, rank, c.xn, fam, out, remap, 2, kEpiStoreBf16, c.s.h, c.status, stream);
+}
+
+int tsp_kv_project_noalloc(const tsp_dims* dims, const tsp_weights* w, int rank, const void* x_local, void* k_full,
+                           void* v_full, cudaStream_t stream) {
+  const int D = w ? w->D : 0;
+  int rc = check_dims(dims, D);
+  if (rc) return rc;
+  if ((rc = check_weights(w, D))) return rc;
+  if (rank < 0 || rank >= D) return TSP_ERR_INVALID_ARG;
+  const Sizes sz = sizes_of(dims, D);
+  if (sz.L == 0) return TSP_OK;
+  if (!x_local || !k_full || !v_full || !aligned16(x_local) || !aligned16(k_full) || !aligned16(v_full))
+    return TSP_ERR_INVALID_ARG;
+  const size_t need = kNoAllocXnOffset + static_cast<size_t>(sz.L) * sz.h * 2;
+  if (need > kNoAllocScratchBytes) {
+    std::snprintf(g_cuda_err, sizeof(g_cuda_err),
+                  "tsp_kv_project_noalloc: T/D * h * 2 + 1024 = %zu bytes exceeds the %zu-byte static scratch", need,
+                  kNoAllocScratchBytes);
+    return TSP_ERR_WORKSPACE;
+  }
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch(&scratch))) return rc;
+  uint8_t* base = static_cast<uint8_t*>(scratch);
+  int* status = reinterpret_cast<int*>(base);
+  __half* xn = reinterpret_cast<__half*>(base + kNoAllocXnOffset);
+  // the array keeps the previous call's contents: the status word starts at zero
+  TSP_CUDA(cudaMemsetAsync(status, 0, sizeof(int), stream));
+  rc = launch_layernorm<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x_local), xn, sz.L, sz.h, dims->ln_eps, stream);
+  if (rc) return rc;
+  const void* const* fam[3] = {reinterpret_cast<const void* const*>(w->wk),
+                               reinterpret_cast<const void* const*>(w->wv), nullptr};
+  void* out[3] = {k_full, v_full, nullptr};
+  const int remap[3] = {1, 1, 0};
+  return launch_proj(sz, rank, xn, fam, out, remap, 2, kEpiStoreBf16, sz.h, status, stream);
 }
 
 int tsp_layer_forward(const tsp_dims* dims, const tsp_weights* w, int rank, const void* x_local, const void* k_full,

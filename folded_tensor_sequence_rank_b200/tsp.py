@@ -70,6 +70,7 @@ def lib() -> ctypes.CDLL:
         "tsp_reset_device_status": (i32, [vp, vp]),
         "tsp_get_device_status": (i32, [vp, vp]),
         "tsp_kv_project": (i32, [pd, pw, i32, vp, vp, vp, vp, sz, vp]),
+        "tsp_kv_project_noalloc": (i32, [pd, pw, i32, vp, vp, vp, vp]),
         "tsp_layer_forward": (i32, [pd, pw, i32, vp, vp, vp, vp, i32, vp, sz, vp, ctypes.POINTER(vp)]),
         "tsp_rank_step": (i32, [pd, pw, i32, vp, vp, vp, vp, i32, vp, sz, vp, ctypes.POINTER(vp)]),
         "tsp_rank_step_host": (i32, [pd, pw, i32, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]),
@@ -236,6 +237,15 @@ def kv_project(dims: Dims, w: ShardedWeights, rank: int, x_local, k_full, v_full
     px, pk, pv, _, pws = _rank_io(dims, w, x_local, k_full, v_full, None, ws)
     _check(lib().tsp_kv_project(ctypes.byref(dims), ctypes.byref(w.struct), rank, px, pk, pv, pws, ws.numel(),
                                 _stream(stream)), "tsp_kv_project")
+
+
+def kv_project_noalloc(dims: Dims, w: ShardedWeights, rank: int, x_local, k_full, v_full, stream=None):
+    """tsp_kv_project without a workspace (for callers that cannot allocate):
+    its scratch is a fixed 64 MiB device array inside the library."""
+    ws_dummy = torch.empty(0, dtype=torch.uint8, device=x_local.device)
+    px, pk, pv, _, _ = _rank_io(dims, w, x_local, k_full, v_full, None, ws_dummy)
+    _check(lib().tsp_kv_project_noalloc(ctypes.byref(dims), ctypes.byref(w.struct), rank, px, pk, pv,
+                                        _stream(stream)), "tsp_kv_project_noalloc")
 
 
 def layer_forward(dims: Dims, w: ShardedWeights, rank: int, x_local, k_full, v_full, y_local, ws,

@@ -165,6 +165,30 @@ int tsp_kv_project(const tsp_dims* dims, const tsp_weights* w, int rank,
                    const void* x_local, void* k_full, void* v_full,
                    void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* tsp_kv_project for callers that cannot allocate device memory.  The paper
+ * has no counterpart: this is a deployment variant of tsp_kv_project, not a
+ * step of the method.  Some callers are handed only their input and output
+ * buffers and own no device allocator (a plugin inside a host framework that
+ * manages all device memory), and some must not call cudaMalloc on their hot
+ * path because it can synchronise the device or fail at run time.  This
+ * entry point computes exactly what tsp_kv_project computes (same kernels,
+ * bit-identical K and V) and takes no workspace: its scratch - the LN1
+ * output of the rank's tokens and a status word - is a file-scope device
+ * array of 64 MiB inside this library, held by every GPU that loads the
+ * library until the process exits.  Limit: T/D * h * 2 + 1024 bytes must fit
+ * in 64 MiB (e.g. 8191 tokens at h = 4096); larger sizes return
+ * TSP_ERR_WORKSPACE with a message in tsp_last_cuda_error.  The first call on
+ * a device looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current; make that first call before any stream capture.  All
+ * calls share the one array, which keeps the last call's contents (the call
+ * clears its status word itself): calls that overlap on the GPU - from
+ * different streams or threads - race on it, so order them.  A device-side
+ * timeout inside this call is recorded only in the array's status word and is
+ * not reported.  No cudaMalloc, cudaFree or allocating library routine is
+ * used.  Arguments as in tsp_kv_project. */
+int tsp_kv_project_noalloc(const tsp_dims* dims, const tsp_weights* w, int rank,
+                           const void* x_local, void* k_full, void* v_full, cudaStream_t stream);
+
 /* The rank's layer forward given the all-gathered K/V [zubnet.ai TSP item,
  * paragraphs 1-2, 4]:
  *   Xn = LN1(x_local);  for each shard k: Q_k = Xn Wq_k^T,
