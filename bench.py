@@ -333,6 +333,136 @@ def run_tsp(args, wl):
         dist.destroy_process_group()
 
 
+STEP_NAMES = ("ln1", "qkv", "attention", "o", "ln2", "w1", "w2")
+
+
+def _synthetic(T, h, F, seed, device="cuda"):
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+
+    def rnd(*shape, std=1.0, dtype=torch.bfloat16):
+        return (torch.randn(*shape, generator=g, device=device, dtype=torch.float32) * std).to(dtype)
+    w = {"wq": rnd(h, h, std=0.02), "wk": rnd(h, h, std=0.02), "wv": rnd(h, h, std=0.02),
+         "wo": rnd(h, h, std=0.02), "w1": rnd(h, F, std=0.02), "w2": rnd(F, h, std=0.02)}
+    return rnd, w
+
+
+def run_sweep_ranks(args):
+    """All D = 8 ranks of the 128K layer back to back on one GPU (seed 3): the
+    K/V projection of every rank's tokens (what the all-gather assembles), then
+    every rank's layer forward.  Reports whole-layer tokens/s = T / (sum of all
+    projection and layer times) and the spread of the per-rank layer times,
+    (max - min) / mean, which the zigzag partition makes ~0."""
+    import torch
+    from folded_tensor_sequence_rank_b200 import tsp
+    T, h, H, F, D = 131072, 4096, 32, 16384, 8
+    L = T // D
+    torch.cuda.set_device(0)
+    dims = tsp.make_dims(T, h, H, F)
+    rnd, w_full = _synthetic(T, h, F, 3)
+    sw = tsp.pack_shards(dims, D, w_full)
+    del w_full
+    x = rnd(T, h)
+    xs = [x.index_select(0, tsp.zigzag_index(T, D, r).long()).contiguous() for r in range(D)]
+    del x
+    K = torch.empty(T, h, dtype=torch.float16, device="cuda")
+    V = torch.empty_like(K)
+    ys = [torch.empty(L, h, dtype=torch.bfloat16, device="cuda") for _ in range(D)]
+    ws = tsp.alloc_workspace(dims, D)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def one_layer(record):
+        kv_ev = [ev() for _ in range(D + 1)] if record else None
+        fw_ev = [ev() for _ in range(D + 1)] if record else None
+        s = torch.cuda.current_stream()
+        if record:
+            kv_ev[0].record(s)
+        for r in range(D):
+            tsp.kv_project(dims, sw, r, xs[r], K, V, ws)
+            if record:
+                kv_ev[r + 1].record(s)
+        if record:
+            fw_ev[0].record(s)
+        for r in range(D):
+            tsp.layer_forward(dims, sw, r, xs[r], K, V, ys[r], ws)
+            if record:
+                fw_ev[r + 1].record(s)
+        return kv_ev, fw_ev
+
+    for _ in range(args.warmup):
+        one_layer(False)
+    torch.cuda.synchronize()
+    assert tsp.get_device_status(ws) == tsp.TSP_OK, "device wait timed out during warm-up"
+    steps = max(1, min(args.steps, 5))
+    clocks = ClockSampler(0)
+    time.sleep(0.3)
+    recs = [one_layer(True) for _ in range(steps)]
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    assert tsp.get_device_status(ws) == tsp.TSP_OK, "device wait timed out"
+    kv_ms = [statistics.median(k[r].elapsed_time(k[r + 1]) for k, _ in recs) for r in range(D)]
+    fw_ms = [statistics.median(f[r].elapsed_time(f[r + 1]) for _, f in recs) for r in range(D)]
+    total = sum(kv_ms) + sum(fw_ms)
+    mean = statistics.mean(fw_ms)
+    line = {"metric": "TSP whole-layer fwd tokens/s, all 8 ranks back to back on 1 B200 (7B layer, 128K, D=8)",
+            "value": T / (total * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": steps, "warmup": args.warmup,
+            "ms_per_step": total, "higher_is_better": True, "dtype": "fp16", "data": "synthetic",
+            "config": {"workload": "7B dense layer, T=131072, D=8, every rank in turn (seed 3)",
+                       "l2": "inputs larger than L2; no flush"},
+            "kv_project_ms": [round(t, 4) for t in kv_ms], "layer_forward_ms": [round(t, 4) for t in fw_ms],
+            "layer_spread": (max(fw_ms) - min(fw_ms)) / mean, "clocks": clk}
+    print(json.dumps(line), flush=True)
+
+
+def run_sweep_shards(args):
+    """Rank 0 of the 7B layer at T = 32768 for D = 1, 2, 4, 8, 16 (seed 4):
+    per-kernel times and rates as the shards shrink (h/D Q columns, F/D FFN
+    columns per shard)."""
+    import torch
+    from folded_tensor_sequence_rank_b200 import tsp
+    T, h, H, F = 32768, 4096, 32, 16384
+    torch.cuda.set_device(0)
+    dims = tsp.make_dims(T, h, H, F)
+    rnd, w_full = _synthetic(T, h, F, 4)
+    kv_std = 0.02 * math.sqrt(h)
+    K = rnd(T, h, std=kv_std, dtype=torch.float16)
+    V = rnd(T, h, std=kv_std, dtype=torch.float16)
+    out = {}
+    steps = max(1, min(args.steps, 10))
+    for D in (1, 2, 4, 8, 16):
+        L = T // D
+        sw = tsp.pack_shards(dims, D, w_full)
+        x = rnd(L, h)
+        y = torch.empty(L, h, dtype=torch.bfloat16, device="cuda")
+        ws = tsp.alloc_workspace(dims, D)
+        for _ in range(args.warmup):
+            tsp.rank_step(dims, sw, 0, x, K, V, y, ws)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(tsp.N_STEP_EVENTS)] for _ in range(steps)]
+        for i in range(steps):
+            tsp.rank_step(dims, sw, 0, x, K, V, y, ws, events=evs[i])
+        torch.cuda.synchronize()
+        assert tsp.get_device_status(ws) == tsp.TSP_OK, "device wait timed out"
+        ms = {n: statistics.median(e[j].elapsed_time(e[j + 1]) for e in evs) for j, n in enumerate(STEP_NAMES)}
+        fl = rank_flops(T, h, F, D, 0)
+        step = sum(ms.values())
+        out[str(D)] = {"tokens_per_s": L / (step * 1e-3), "step_ms": round(step, 4),
+                       "kernel_ms": {k: round(v, 4) for k, v in ms.items()},
+                       "tflops": {"attention": fl["attention"] / (ms["attention"] * 1e-3) / 1e12,
+                                  "qkv": fl["qkv"] / (ms["qkv"] * 1e-3) / 1e12,
+                                  "o": fl["o"] / (ms["o"] * 1e-3) / 1e12,
+                                  "w1": fl["mlp"] / 2 / (ms["w1"] * 1e-3) / 1e12,
+                                  "w2": fl["mlp"] / 2 / (ms["w2"] * 1e-3) / 1e12}}
+        del sw, x, y, ws
+        torch.cuda.empty_cache()
+    line = {"metric": "TSP rank-0 layer fwd tokens/s vs shard count D on 1 B200 (7B layer, 32K)",
+            "value": out["8"]["tokens_per_s"], "unit": UNIT, "n_gpus": 1, "steps": steps, "warmup": args.warmup,
+            "higher_is_better": True, "dtype": "fp16", "data": "synthetic",
+            "config": {"workload": "7B dense layer, T=32768, rank 0, D in {1,2,4,8,16} (seed 4); value is D=8"},
+            "by_D": out}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -341,11 +471,18 @@ def main():
     ap.add_argument("--impl", default="tsp", choices=["tsp", "reference"])
     ap.add_argument("--workload", default="7b-128k-d8", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", choices=["ranks", "shards"], default=None,
+                    help="ranks: all 8 ranks of the 128K layer in turn (per-rank spread, whole-layer tokens/s); "
+                         "shards: rank 0 at T=32768 for D=1..16")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     wl = WORKLOADS[args.workload]
-    if args.impl == "reference":
+    if args.sweep == "ranks":
+        run_sweep_ranks(args)
+    elif args.sweep == "shards":
+        run_sweep_shards(args)
+    elif args.impl == "reference":
         run_reference(args, wl)
     else:
         run_tsp(args, wl)
