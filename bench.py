@@ -277,23 +277,41 @@ def run_tsp(args, wl):
             step_ms[n] += ev[j].elapsed_time(ev[j + 1]) / args.steps
     kern_ms = sum(step_ms.values())
 
-    # --- end to end: host (pinned) tokens in, host result out, through the C ABI
-    hx = x_local.cpu().pin_memory()
-    hy = torch.empty(L, h, dtype=torch.bfloat16).pin_memory()
-    xs = torch.empty_like(x_local)
-    ys = torch.empty_like(y)
-    for _ in range(2):
-        tsp.rank_step_host(dims, sw, trank, hx, xs, K, V, ys, hy, ws)
+    # --- end to end: host (pinned) tokens in, host result out, through the C ABI.
+    # Consecutive steps alternate between two streams ("lanes"), each with its
+    # own staging buffers, workspace and K/V, so the copy engines move one
+    # step's tokens while the SMs compute the other's; every step still does
+    # its own host->device and device->host copy.
+    lanes = []
+    for li in range(2):
+        lanes.append(dict(stream=torch.cuda.Stream(), hx=x_local.cpu().pin_memory(),
+                          hy=torch.empty(L, h, dtype=torch.bfloat16).pin_memory(),
+                          xs=torch.empty_like(x_local), ys=torch.empty_like(y),
+                          ws=ws if li == 0 else tsp.alloc_workspace(dims, D),
+                          K=K if li == 0 else K.clone(), V=V if li == 0 else V.clone()))
+    torch.cuda.synchronize()
+
+    def host_step(ln):
+        with torch.cuda.stream(ln["stream"]):
+            tsp.rank_step_host(dims, sw, trank, ln["hx"], ln["xs"], ln["K"], ln["V"], ln["ys"], ln["hy"], ln["ws"],
+                               stream=ln["stream"])
+    for i in range(4):
+        host_step(lanes[i % 2])
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
-        tsp.rank_step_host(dims, sw, trank, hx, xs, K, V, ys, hy, ws)
+    for ln in lanes:
+        ln["stream"].wait_event(e0)
+    for i in range(args.steps):
+        host_step(lanes[i % 2])
+    for ln in lanes:
+        stream.wait_stream(ln["stream"])
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / args.steps
-    assert tsp.get_device_status(ws) == tsp.TSP_OK, "device wait timed out"
+    for ln in lanes:
+        assert tsp.get_device_status(ln["ws"]) == tsp.TSP_OK, "device wait timed out"
 
     ms, e2e_ms, attn_ms = tdist.max_over_ranks([ms, e2e_ms, step_ms["attention"]], device="cuda")
 

@@ -300,6 +300,41 @@ def test_7b_layer_T32768_shard_sweep_sampled(D):
     sampled_rank_check(32768, D, 0, 4, n_sample=30)
 
 
+@pytest.mark.parametrize("T,h,H,F,D,ramp,n_sample", [
+    (512, 256, 4, 1024, 2, 60.0, None),       # head_dim 64, every row of both ranks
+    (8192, 4096, 32, 16384, 8, 3.0, 62),      # head_dim 128, sampled rows of ranks 0 and 5
+])
+def test_growing_logits_force_rescales(T, h, H, F, D, ramp, n_sample):
+    """K rows scaled by 1 + ramp * position / T: the logits grow along the
+    sequence, so a row's running maximum grows by 17-25 in log2 units after
+    its first key tile (about 0 at these sizes without the ramp), and the
+    attention kernel's lazy rescale of O (growth beyond 2^8), including a
+    growth of more than 2^16 inside one tile, runs many times.  The oracle
+    takes the same fp16 K."""
+    L = T // D
+    raw = inputs.rank_inputs(L, T, h, F, 7)
+    g = 1.0 + ramp * torch.arange(T, dtype=torch.float32) / T
+    k_ramp = (raw["k_full"].float() * g[:, None]).to(torch.float16)
+    assert torch.isfinite(k_ramp).all()
+    dev = to_cuda({n: raw[n] for n in inputs.WEIGHT_NAMES})
+    dims = tsp.make_dims(T, h, H, F)
+    sw = tsp.pack_shards(dims, D, dev)
+    ws = tsp.alloc_workspace(dims, D)
+    Kd, Vd = k_ramp.cuda(), raw["v_full"].cuda()
+    w = weights_f64(raw)
+    Kf = k_ramp.double().numpy()
+    Vf = raw["v_full"].double().numpy()
+    x_all = f64(raw["x_local"])
+    for r in (0, D - 3 if D > 2 else 1):
+        y = torch.empty(L, h, dtype=torch.float32, device="cuda")
+        tsp.layer_forward(dims, sw, r, raw["x_local"].cuda(), Kd, Vd, y, ws)
+        assert tsp.get_device_status(ws) == tsp.TSP_OK
+        pos = O.zigzag_index(T, D, r)
+        rows = np.arange(L) if n_sample is None else inputs.sample_rows(L, n_sample, 7 + r, must=(0, L // 2, L - 1))
+        ref = O.rank_rows_forward(x_all[rows], pos[rows], Kf, Vf, w, H)
+        assert_layer_close(f64(y)[rows], ref["y"], f"growing logits T={T} D={D} rank {r}", x_all[rows])
+
+
 # --------------------------------------------------------------------------
 # failure detection without a GPU fault
 # --------------------------------------------------------------------------
