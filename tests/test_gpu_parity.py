@@ -138,6 +138,10 @@ def run_full_sequence(T, h, H, F, D, seed, y_dtype=torch.float32):
     (800, 256, 4, 1024, 2, 7),     # ragged chunks: c = 200
     (288, 256, 2, 512, 2, 8),      # head_dim 128, c = 72 (< one tile)
     (2048, 512, 4, 2048, 2, 9),    # head_dim 128, several tiles per chunk
+    (768, 384, 6, 1536, 3, 10),    # D = 3 (not a power of two), h/D = 128
+    (960, 320, 5, 1280, 5, 11),    # D = 5, h/D = 64, ragged chunks c = 96
+    (1536, 384, 3, 1536, 3, 13),   # head_dim 128 with one head per shard, D = 3
+    (8, 256, 4, 1024, 4, 12),      # degenerate chunks: c = 1, two local rows per rank
 ])
 def test_full_sequence_all_ranks(T, h, H, F, D, seed):
     raw, K, V, Y, idx, inter = run_full_sequence(T, h, H, F, D, seed)

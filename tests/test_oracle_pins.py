@@ -299,9 +299,11 @@ def test_layer_matches_torch_composition(cfg, seed, storage):
 # --------------------------------------------------------------------------
 # the TSP schedule equals the plain layer  (sum over shards = full contraction)
 # --------------------------------------------------------------------------
-@pytest.mark.parametrize("D", [1, 2, 4])
-def test_sharded_schedule_equals_unsharded_layer(D):
-    cfg = TINY
+ODD = dict(T=120, h=120, H=15, F=480)      # d = 8; divisible by D = 3, 5, 15
+
+
+@pytest.mark.parametrize("cfg,D", [(TINY, 1), (TINY, 2), (TINY, 4), (ODD, 3), (ODD, 5), (ODD, 15)])
+def test_sharded_schedule_equals_unsharded_layer(cfg, D):
     x, w = tiny_inputs(cfg, 21 + D)
     full = O.layer_forward(x, w, cfg["H"])
     K, V = O.kv_all_gather_sharded(x, D, w)
