@@ -93,6 +93,68 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, uint6
   }
 }
 
+// One 32-column chunk of an output tile's epilogue: accumulator values r for
+// local row m (global zigzag row grow) and output columns n .. n+31.
+__device__ __forceinline__ void gemm_epilogue_chunk(const GemmParams& p, int m, int64_t grow, int n,
+                                                    const uint32_t (&r)[32]) {
+  if (p.epi == kEpiResidual) {
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+    const int64_t off = static_cast<int64_t>(m) * p.ldo + n;
+    if (p.resid_f32) {
+      const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.resid) + off);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 q = src[i];
+        v[4 * i] += q.x; v[4 * i + 1] += q.y; v[4 * i + 2] += q.z; v[4 * i + 3] += q.w;
+      }
+    } else {
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.resid) + off);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 q = src[i];
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&w[j]);
+          const float2 f = __bfloat1622float2(b2);
+          v[8 * i + 2 * j] += f.x;
+          v[8 * i + 2 * j + 1] += f.y;
+        }
+      }
+    }
+    if (p.out_f32) {
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out[0]) + off);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    } else {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out[0]) + off);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        dst[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                            pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+    }
+  } else {
+    const int seg = n / p.seg_n;
+    const int col = n - seg * p.seg_n;
+    const int64_t orow = p.remap[seg] ? grow : m;
+    uint32_t packed[16];
+    if (p.epi == kEpiGeluBf16) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        packed[i] = pack_half2(gelu_tanh_f(__uint_as_float(r[2 * i])), gelu_tanh_f(__uint_as_float(r[2 * i + 1])));
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) packed[i] = pack_half2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+    }
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<__half*>(p.out[seg]) + orow * p.ldo + col);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+  }
+}
+
 template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_f16_tcgen05(const __grid_constant__ GemmParams p) {
   using S = GemmShape<BN>;
@@ -230,64 +292,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_f16_tcgen05(const __grid
         tmem_ld32(tmem_base + lane_off + buf * BN + ch * 32, r);
         tmem_ld_wait();
         const int n = nb * BN + ch * 32;
-        if (!valid) {
-        } else if (p.epi == kEpiResidual) {
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-          const int64_t off = static_cast<int64_t>(m) * p.ldo + n;
-          if (p.resid_f32) {
-            const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.resid) + off);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float4 q = src[i];
-              v[4 * i] += q.x; v[4 * i + 1] += q.y; v[4 * i + 2] += q.z; v[4 * i + 3] += q.w;
-            }
-          } else {
-            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.resid) + off);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const uint4 q = src[i];
-              const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&w[j]);
-                const float2 f = __bfloat1622float2(b2);
-                v[8 * i + 2 * j] += f.x;
-                v[8 * i + 2 * j + 1] += f.y;
-              }
-            }
-          }
-          if (p.out_f32) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out[0]) + off);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out[0]) + off);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
-                                  pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
-          }
-        } else {
-          const int seg = n / p.seg_n;
-          const int col = n - seg * p.seg_n;
-          const int64_t orow = p.remap[seg] ? grow : m;
-          uint32_t packed[16];
-          if (p.epi == kEpiGeluBf16) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              packed[i] = pack_half2(gelu_tanh_f(__uint_as_float(r[2 * i])), gelu_tanh_f(__uint_as_float(r[2 * i + 1])));
-          } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              packed[i] = pack_half2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-          }
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__half*>(p.out[seg]) + orow * p.ldo + col);
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
-        }
+        if (valid) gemm_epilogue_chunk(p, m, grow, n, r);
       }
       tc_fence_before();
       __syncwarp();

@@ -17,6 +17,7 @@
 
 #include "tsp.h"
 #include "attn_sm100.cuh"
+#include "gemm_pair_sm100.cuh"
 #include "gemm_sm100.cuh"
 #include "misc_kernels.cuh"
 
@@ -188,16 +189,65 @@ int launch_gemm_bn(GemmParams& p, cudaStream_t st) {
   return TSP_OK;
 }
 
+// 256-column tiles run on CTA pairs (clusters of two, 256 x 256 tiles).
+int launch_gemm_pair(GemmParams& p, cudaStream_t st) {
+  using S = GemmPairShape;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  static int max_clusters = 0;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(gemm_pair_f16_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes);
+    if (attr_err != cudaSuccess) return;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = S::kSmemBytes;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    attr_err = cudaOccupancyMaxActiveClusters(&max_clusters, gemm_pair_f16_tcgen05, &cfg);
+  });
+  TSP_CUDA(attr_err);
+  if (max_clusters <= 0) {
+    std::snprintf(g_cuda_err, sizeof(g_cuda_err), "no CTA pair of the GEMM kernel fits on this GPU");
+    return TSP_ERR_CUDA;
+  }
+  const int tiles = ((p.M + kPairBM - 1) / kPairBM) * (p.N / kPairBN);
+  const int pairs = tiles < max_clusters ? tiles : max_clusters;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = S::kSmemBytes;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  TSP_CUDA(cudaLaunchKernelEx(&cfg, gemm_pair_f16_tcgen05, p));
+  TSP_CUDA(cudaGetLastError());
+  return TSP_OK;
+}
+
 int pick_bn(int n_block) {
   if (n_block % 256 == 0) return 256;
   if (n_block % 128 == 0) return 128;
   return 64;
 }
 
+// Rows of a B tile each CTA loads: half of a pair tile for 256 columns.
+int b_box_rows(int bn) { return bn == 256 ? 128 : bn; }
+
 int launch_gemm(GemmParams& p, int bn, cudaStream_t st) {
   if (p.M == 0) return TSP_OK;
   switch (bn) {
-    case 256: return launch_gemm_bn<256>(p, st);
+    case 256: return launch_gemm_pair(p, st);
     case 128: return launch_gemm_bn<128>(p, st);
     default: return launch_gemm_bn<64>(p, st);
   }
@@ -223,7 +273,7 @@ int launch_proj(const Sizes& s, int rank, const __half* xn, const void* const* f
   const int bn = pick_bn(shard_n);
   for (int seg = 0; seg < nseg; ++seg)
     for (int k = 0; k < s.D; ++k) {
-      rc = make_map(&p.map_b[seg * s.D + k], fam[seg][k], shard_n, s.h, s.h, bn);
+      rc = make_map(&p.map_b[seg * s.D + k], fam[seg][k], shard_n, s.h, s.h, b_box_rows(bn));
       if (rc) return rc;
     }
   p.M = static_cast<int>(s.L);
@@ -253,7 +303,7 @@ int launch_ksplit(const Sizes& s, int rank, const __half* a, int Kdim, const voi
   int rc = make_map(&p.map_a, a, s.L, Kdim, Kdim, kGemmBM);
   if (rc) return rc;
   for (int k = 0; k < s.D; ++k) {
-    rc = make_map(&p.map_b[k], fam[k], s.h, shard_k, shard_k, bn);
+    rc = make_map(&p.map_b[k], fam[k], s.h, shard_k, shard_k, b_box_rows(bn));
     if (rc) return rc;
   }
   p.M = static_cast<int>(s.L);
