@@ -481,6 +481,58 @@ def run_sweep_shards(args):
     print(json.dumps(line), flush=True)
 
 
+def run_sweep_stack(args):
+    """A 32-layer stack of the 7B layer at T = 131072 on one GPU, all D = 8
+    ranks in turn per layer (K/V projections, then layer forwards), random
+    weights per layer.  Reports whole-stack tokens/s = T / forward time, the
+    time per layer, the peak device memory of this one-GPU simulation, and
+    the per-GPU memory account of the same forward on 8 GPUs."""
+    import torch
+    from folded_tensor_sequence_rank_b200 import stack, tsp
+    T, h, H, F, D, n_layers = 131072, 4096, 32, 16384, 8, 32
+    torch.cuda.set_device(0)
+    dims = tsp.make_dims(T, h, H, F)
+    layers = []
+    for i in range(n_layers):
+        rnd, w_full = _synthetic(T, h, F, 100 + i)
+        layers.append(tsp.pack_shards(dims, D, w_full))
+        del w_full
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    x = rnd(T, h)
+    xs = [x.index_select(0, tsp.zigzag_index(T, D, r).long()).contiguous() for r in range(D)]
+    del x
+    K = torch.empty(T, h, dtype=torch.float16, device="cuda")
+    V = torch.empty_like(K)
+    ws = tsp.alloc_workspace(dims, D)
+    torch.cuda.reset_peak_memory_stats()
+    stack.stack_forward(dims, layers[:2], xs, K, V, ws)  # warm-up
+    torch.cuda.synchronize()
+    assert tsp.get_device_status(ws) == tsp.TSP_OK, "device wait timed out during warm-up"
+    steps = max(1, min(args.steps, 2))
+    clocks = ClockSampler(0)
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        ys = stack.stack_forward(dims, layers, xs, K, V, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    assert tsp.get_device_status(ws) == tsp.TSP_OK, "device wait timed out"
+    assert all(torch.isfinite(y.float()).all() for y in ys)
+    ms = e0.elapsed_time(e1) / steps
+    acc = stack.memory_account(dims, D, n_layers)
+    line = {"metric": "TSP 32-layer stack fwd tokens/s, all 8 ranks in turn on 1 B200 (7B layers, 128K, D=8)",
+            "value": T / (ms * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": steps, "warmup": 1,
+            "ms_per_step": ms, "ms_per_layer": ms / n_layers, "higher_is_better": True, "dtype": "fp16",
+            "data": "synthetic",
+            "config": {"workload": "32 x 7B dense layer (random weights per layer), T=131072, D=8, every rank in turn"},
+            "peak_device_bytes_this_run": torch.cuda.max_memory_allocated(),
+            "per_gpu_bytes_on_8_gpus": acc, "clocks": clk}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -489,9 +541,9 @@ def main():
     ap.add_argument("--impl", default="tsp", choices=["tsp", "reference"])
     ap.add_argument("--workload", default="7b-128k-d8", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--sweep", choices=["ranks", "shards"], default=None,
+    ap.add_argument("--sweep", choices=["ranks", "shards", "stack"], default=None,
                     help="ranks: all 8 ranks of the 128K layer in turn (per-rank spread, whole-layer tokens/s); "
-                         "shards: rank 0 at T=32768 for D=1..16")
+                         "shards: rank 0 at T=32768 for D=1..16; stack: a 32-layer forward at 128K")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -500,6 +552,8 @@ def main():
         run_sweep_ranks(args)
     elif args.sweep == "shards":
         run_sweep_shards(args)
+    elif args.sweep == "stack":
+        run_sweep_stack(args)
     elif args.impl == "reference":
         run_reference(args, wl)
     else:

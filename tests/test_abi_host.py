@@ -136,3 +136,21 @@ def test_binding_refuses_cpu_tensors(L):
     d = dims()
     with pytest.raises(ValueError):
         tsp.pack_shards(d, 2, {n: torch.zeros(1, dtype=torch.bfloat16) for n in tsp.WEIGHT_NAMES})
+
+
+def test_memory_account_7b_forward():
+    """Per-GPU bytes of a 32-layer forward of the 7B layer at 128K on D = 8
+    GPUs, against the formula written out here: 384 MiB of fp16 weights per
+    layer, 1/D of them owned, one layer's other shards in flight, the rank's
+    tokens in and out, the all-gathered K/V, and the layer workspace."""
+    from folded_tensor_sequence_rank_b200 import stack
+    dims = tsp.make_dims(131072, 4096, 32, 16384)
+    acc = stack.memory_account(dims, 8, 32)
+    MiB = 1 << 20
+    assert acc["weights_own_shards"] == 32 * 384 * MiB // 8
+    assert acc["weights_receive_buffer"] == 384 * MiB * 7 // 8
+    assert acc["tokens_in_out"] == 2 * 16384 * 4096 * 2
+    assert acc["kv_all_gathered"] == 2 * 131072 * 4096 * 2
+    assert acc["workspace"] == tsp.workspace_bytes(dims, 8) > 0
+    assert acc["total"] == sum(v for k, v in acc.items() if k != "total")
+    assert 5.0 < acc["total"] / 2**30 < 6.0
