@@ -26,21 +26,21 @@
 //   warp 1     TMEM allocator + single-thread tcgen05.mma issuer
 //   warps 2-5  softmax, correction and epilogue of query tile A (thread = row)
 //   warps 6-9  the same for query tile B
-// Each SM sub-partition runs one warp of each tile.  The tensor core is fed
-// in the order S_A0 S_B0 | PV_A0 S_A1 PV_B0 S_B1 | PV_A1 S_A2 PV_B1 S_B2 ...,
-// so while one tile's softmax runs, the tensor core works on the other
-// tile's PV and next S, and the two softmax warps of a sub-partition work
-// out of phase.
-// Tensor memory (512 columns): [S_A / P_A | O_A | S_B / P_B | O_B], 128
-// columns each.  The softmax writes the fp16 probabilities P (64 columns, in
-// pairs) over the first half of its own score tile once the scores are in
-// registers; the next score tile of that query tile is issued after the
-// PV that reads P, and tcgen05.mma executes in issue order.  A finished
-// S_X(j) therefore also means PV_X(j-1) has finished, so the softmax may
-// rescale O_X with no further wait.
-// Online softmax in base 2 with a lazily updated row maximum: the running
-// output is rescaled only when the maximum grows by more than 2^8, which is
-// exact (the final division by the row sum cancels the common factor).
+// Each SM sub-partition runs one warp of each tile.
+// Tensor memory (512 columns): [S | P_A | P_B | O_A | O_B] = 128 + 64 + 64 +
+// 128 + 128.  The score buffer S is shared by the two query tiles and used in
+// turn: S_A(j), S_B(j), S_A(j+1), ...  A softmax warp reads its whole score
+// tile into registers and at once hands S back to the issuer, which computes
+// the other tile's scores while the softmax turns its registers into fp16
+// probabilities P in the tile's own P region.  The tensor core is fed in the
+// order S_A(j+1) PV_A(j) S_B(j+1) PV_B(j) ..., so the next scores of a tile
+// never wait for its PV, and a softmax warp never waits for the tensor core
+// except for its next score tile.  P_x is rewritten only after the PV that
+// read it has finished (one commit per PV).
+// Online softmax in base 2 with a lazily updated row maximum: the tile's
+// maximum is found first; the running output is rescaled only when the
+// maximum grows by more than 2^8, which is exact (the final division by the
+// row sum cancels the common factor).
 // Q, K, V, P and the output are fp16; scores, softmax statistics and O are
 // fp32.
 #pragma once
@@ -137,11 +137,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
   uint64_t* k_empty = k_full + KST;         // [KST]
   uint64_t* v_full = k_empty + KST;         // [VST]
   uint64_t* v_empty = v_full + VST;         // [VST]
-  uint64_t* s_full = v_empty + VST;         // [2] score tile of query tile x ready
+  uint64_t* s_full = v_empty + VST;         // [2] S holds the scores of query tile x
   uint64_t* p_full = s_full + 2;            // [2] probabilities of tile x written
   uint64_t* o_full = p_full + 2;            // [2] last PV of tile x done
   uint64_t* o_free = o_full + 2;            // [2] epilogue of tile x has read O
-  uint64_t* it_full = o_free + 2;           // [2]
+  uint64_t* pv_done = o_free + 2;           // [2] a PV of tile x (not its last) done
+  uint64_t* s_free = pv_done + 2;           // the scores in S have been read
+  uint64_t* it_full = s_free + 1;           // [2]
   uint64_t* it_empty = it_full + 2;         // [2]
   uint64_t* drain = it_empty + 2;
   int* it_slot = reinterpret_cast<int*>(drain + 1);  // [2]
@@ -159,6 +161,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
       mbar_init(&p_full[x], 4);
       mbar_init(&o_full[x], 1);
       mbar_init(&o_free[x], 4);
+      mbar_init(&pv_done[x], 1);
       mbar_init(&it_full[x], 1);
       mbar_init(&it_empty[x], 9);
     }
@@ -170,6 +173,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
+    mbar_init(s_free, 4);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -248,6 +252,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
       uint32_t kph = 0, vph = 0, qph[2] = {0, 0};
       uint32_t pcnt[2] = {0, 0};  // probability tiles consumed, per query-tile slot
       uint32_t icnt[2] = {0, 0};  // items finished, per query-tile slot
+      uint32_t scnt = 0;          // score tiles issued (S is reused after each is read)
       bool ok = true;
       // Shared-memory descriptors of every Q and K/V stage, built once; an MMA
       // group then only adds immediate offsets (see mma_ss_x8 / mma_ts_x8).
@@ -259,18 +264,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
       auto vdesc = [&]() { return vdesc0 + static_cast<uint64_t>(vs * (S::kKVBytes >> 4)); };
       // S_x = Q_x K^T for the K tile in slot ks (K = head_dim in 16-column steps:
       // +32 bytes inside a 128-byte swizzle row, +16 KiB to the next 64 columns)
-      auto issue_s = [&](int x, bool last_s) {
+      auto issue_s = [&](int x, bool last_s) -> bool {
+        if (scnt > 0 && !mbar_wait(s_free, (scnt - 1) & 1, ctl)) return false;
+        ++scnt;
+        tc_fence_after();
         if constexpr (HD == 128) {
-          mma_ss_x8<0, 2, 4, 6, 1024, 1026, 1028, 1030>(tmem + x * 256, qdesc(x), kdesc(), idesc_s, 0);
+          mma_ss_x8<0, 2, 4, 6, 1024, 1026, 1028, 1030>(tmem, qdesc(x), kdesc(), idesc_s, 0);
         } else {
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk) {
             const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-            mma_ss(tmem + x * 256, qdesc(x) + off, kdesc() + off, idesc_s, kk != 0);
+            mma_ss(tmem, qdesc(x) + off, kdesc() + off, idesc_s, kk != 0);
           }
         }
         mma_commit(&s_full[x]);
         if (last_s) mma_commit(&q_empty[x]);
+        return true;
       };
       // O_x += P_x V for the V tile in slot vs (K = 128 keys in 16-key steps:
       // P advances 8 TMEM columns, V 2 KiB = 128 units)
@@ -279,8 +288,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
         if (!mbar_wait(&p_full[x], pcnt[x] & 1, ctl)) return false;
         ++pcnt[x];
         tc_fence_after();
-        mma_ts_x8<128>(tmem + x * 256 + 128, tmem + x * 256, vdesc(), idesc_o, first ? 0u : 1u);
-        if (last) mma_commit(&o_full[x]);
+        mma_ts_x8<128>(tmem + 256 + x * 128, tmem + 128 + x * 64, vdesc(), idesc_o, first ? 0u : 1u);
+        mma_commit(last ? &o_full[x] : &pv_done[x]);
         return true;
       };
       auto wait_k = [&]() -> bool {
@@ -310,29 +319,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
         tc_fence_after();
         // scores of K tile 0 for both query tiles
         if (!wait_k()) break;
-        if (na > 0) issue_s(0, na == 1);
-        if (nb > 0) issue_s(1, nb == 1);
+        if (na > 0 && !issue_s(0, na == 1)) break;
+        if (nb > 0 && !issue_s(1, nb == 1)) break;
         release_k();
+        // per key tile: S_A(kt+1) PV_A(kt) S_B(kt+1) PV_B(kt)
         for (int kt = 0; ok && kt < nkv; ++kt) {
           if (!mbar_wait(&v_full[vs], vph, ctl)) { ok = false; break; }
           bool k_waited = false;
           if (kt < na) {
-            if (!issue_pv(0, kt == 0, kt == na - 1)) { ok = false; break; }
             if (kt + 1 < na) {
               if (!wait_k()) { ok = false; break; }
               k_waited = true;
-              issue_s(0, kt + 1 == na - 1);
+              if (!issue_s(0, kt + 1 == na - 1)) { ok = false; break; }
             }
+            if (!issue_pv(0, kt == 0, kt == na - 1)) { ok = false; break; }
           }
           if (kt < nb) {
-            if (!issue_pv(1, kt == 0, kt == nb - 1)) { ok = false; break; }
             if (kt + 1 < nb) {
               if (!k_waited) {
                 if (!wait_k()) { ok = false; break; }
                 k_waited = true;
               }
-              issue_s(1, kt + 1 == nb - 1);
+              if (!issue_s(1, kt + 1 == nb - 1)) { ok = false; break; }
             }
+            if (!issue_pv(1, kt == 0, kt == nb - 1)) { ok = false; break; }
           }
           if (k_waited) release_k();
           mma_commit(&v_empty[vs]);
@@ -351,10 +361,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
     const int quarter = warp & 3;      // TMEM lane quarter = rows 32*quarter ..
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t t_s = tmem + lane_off + x * 256;        // S / P of this tile
-    const uint32_t t_o = tmem + lane_off + x * 256 + 128;  // O of this tile
+    const uint32_t t_s = tmem + lane_off;                  // S (shared by both tiles)
+    const uint32_t t_p = tmem + lane_off + 128 + x * 64;   // P of this tile
+    const uint32_t t_o = tmem + lane_off + 256 + x * 128;  // O of this tile
     const float sl2 = p.scale_log2;
-    uint32_t scnt = 0, icnt = 0;
+    uint32_t scnt = 0, icnt = 0, pvcnt = 0;
     for (int n = 0;; ++n) {
       const int slot = n & 1;
       if (!warp_wait(&it_full[slot], (n >> 1) & 1, ctl)) break;
@@ -374,70 +385,75 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
         if (!warp_wait(&s_full[x], scnt & 1, ctl)) { ok = false; break; }
         ++scnt;
         tc_fence_after();
+        // the whole score tile into registers, then S goes back to the issuer
+        uint32_t sr[128];
+        tmem_ld32p(t_s, &sr[0]);
+        tmem_ld32p(t_s + 32, &sr[32]);
+        tmem_ld32p(t_s + 64, &sr[64]);
+        tmem_ld32p(t_s + 96, &sr[96]);
+        tmem_ld_wait();
+        reg_fence32(&sr[0]);
+        reg_fence32(&sr[32]);
+        reg_fence32(&sr[64]);
+        reg_fence32(&sr[96]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
+        float* sv = reinterpret_cast<float*>(sr);
         const int kbase = kt * kAttnBN;
-        const bool diag = kbase + kAttnBN - 1 > T.p0;  // some key may lie past this row
-        // Loads scores [64 hh, 64 hh + 64) and returns their maximum (masked
-        // keys -> -inf); with `exps`, also writes the probabilities
-        // 2^(s*scale*log2e - m) as fp16 pairs into P (one pair in four by the
-        // polynomial on the FMA pipes, the rest on MUFU) and adds them to la/lb.
-        auto half_tile = [&](int hh, bool exps, float neg_m, uint32_t (&P)[32], float2& la, float2& lb) -> float {
-          uint32_t sr[64];
-          tmem_ld32p(t_s + hh * 64, &sr[0]);
-          tmem_ld32p(t_s + hh * 64 + 32, &sr[32]);
-          tmem_ld_wait();
-          reg_fence32(&sr[0]);
-          reg_fence32(&sr[32]);
-          float* sv = reinterpret_cast<float*>(sr);
-          if (diag) {
+        if (kbase + kAttnBN - 1 > T.p0) {  // some key may lie past this row
 #pragma unroll
-            for (int i = 0; i < 64; ++i)
-              if (kbase + hh * 64 + i > qpos) sv[i] = -INFINITY;
-          }
-          float m4[4];
+          for (int i = 0; i < 128; ++i)
+            if (kbase + i > qpos) sv[i] = -INFINITY;
+        }
+        float m4[4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) m4[k] = fmaxf(sv[k], sv[k + 4]);
+        for (int k = 0; k < 4; ++k) m4[k] = fmaxf(sv[k], sv[k + 4]);
 #pragma unroll
-          for (int i = 8; i < 64; i += 8)
+        for (int i = 8; i < 128; i += 8)
 #pragma unroll
-            for (int k = 0; k < 4; ++k) m4[k] = fmax3(m4[k], sv[i + k], sv[i + k + 4]);
-          if (exps) {
-            const float2 sl2v = make_float2(sl2, sl2), negm = make_float2(neg_m, neg_m);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float2 xv = ffma2(make_float2(sv[2 * i], sv[2 * i + 1]), sl2v, negm);
-              float2 pr;
-              if ((i & 3) == 3) {
-                pr = exp2_poly2(xv);
-              } else {
-                pr.x = ex2_approx(xv.x);
-                pr.y = ex2_approx(xv.y);
-              }
-              if (i & 1) lb = fadd2(lb, pr); else la = fadd2(la, pr);
-              P[i] = pack_half2(pr.x, pr.y);
-            }
-          }
-          return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-        };
-        uint32_t P0[32], P1[32];
-        float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
+          for (int k = 0; k < 4; ++k) m4[k] = fmax3(m4[k], sv[i + k], sv[i + k + 4]);
+        const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+        // lazy maximum: move to the new one only if it grew by more than 2^8
+        float f = 1.0f;
+        bool need = false;
         if (kt == 0) {
-          // first key tile of the item: row maximum first, then probabilities
-          const float mx = fmaxf(half_tile(0, false, 0.f, P0, la, lb), half_tile(1, false, 0.f, P1, la, lb));
-          m_used = mx * sl2;
-          half_tile(0, true, -m_used, P0, la, lb);
-          half_tile(1, true, -m_used, P1, la, lb);
+          m_used = mt;
         } else {
-          // Speculate that the row maximum did not grow by more than 2^8 and
-          // compute P with the current one; P stays in registers (the scores
-          // stay intact in TMEM) until the check below.
-          const float mx = fmaxf(half_tile(0, true, -m_used, P0, la, lb), half_tile(1, true, -m_used, P1, la, lb));
-          const float m_new = fmaxf(m_used, mx * sl2);
-          const bool need = m_new > m_used + 8.0f;
-          if (__any_sync(0xffffffffu, need)) {
-            // rare: rescale O and l to the new maximum, then recompute P.
-            // S_x(kt) finished, so PV_x(kt-1) has too: O may be rescaled now.
-            const float f = need ? ex2_approx(m_used - m_new) : 1.0f;
+          need = mt > m_used + 8.0f;
+          if (need) {
+            f = ex2_approx(m_used - mt);
+            m_used = mt;
+          }
+        }
+        // P = 2^(s*scale*log2e - m) as fp16 pairs (one pair in four by the
+        // polynomial on the FMA pipes, the rest on MUFU), and its row sum
+        uint32_t P[64];
+        float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
+        {
+          const float2 sl2v = make_float2(sl2, sl2), negm = make_float2(-m_used, -m_used);
 #pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const float2 xv = ffma2(make_float2(sv[2 * i], sv[2 * i + 1]), sl2v, negm);
+            float2 pr;
+            if ((i & 3) == 3) {
+              pr = exp2_poly2(xv);
+            } else {
+              pr.x = ex2_approx(xv.x);
+              pr.y = ex2_approx(xv.y);
+            }
+            if (i & 1) lb = fadd2(lb, pr); else la = fadd2(la, pr);
+            P[i] = pack_half2(pr.x, pr.y);
+          }
+        }
+        // P_x and O_x are free once the previous PV of this tile has finished
+        if (kt > 0) {
+          if (!warp_wait(&pv_done[x], pvcnt & 1, ctl)) { ok = false; break; }
+          ++pvcnt;
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, need)) {
+            // rare: rescale O to the new maximum before the next PV adds to it
+#pragma unroll 1
             for (int j = 0; j < HD / 32; ++j) {
               uint32_t r[32];
               tmem_ld32(t_o + j * 32, r);
@@ -446,20 +462,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
               for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
               tmem_st32(t_o + j * 32, r);
             }
-            l *= f;
-            if (need) m_used = m_new;
-            la = make_float2(0.f, 0.f);
-            lb = make_float2(0.f, 0.f);
-            half_tile(0, true, -m_used, P0, la, lb);
-            half_tile(1, true, -m_used, P1, la, lb);
           }
         }
-        // keys 0..63 -> columns 0..31, keys 64..127 -> columns 32..63, over
-        // scores already consumed
-        tmem_st32(t_s, P0);
-        tmem_st32(t_s + 32, P1);
+        // keys 2c, 2c+1 -> column c of P
+        tmem_st32p(t_p, &P[0]);
+        tmem_st32p(t_p + 32, &P[32]);
         const float2 lab = fadd2(la, lb);
-        l += lab.x + lab.y;
+        l = l * f + (lab.x + lab.y);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
