@@ -50,7 +50,9 @@ Zigzag partition: the sequence is cut into 2D equal chunks of c = T/(2D)
 tokens, and rank r holds chunks r and 2D-1-r, in that order.
 
 Parity status: every function here is pinned by tests/test_oracle_pins.py
-(closed forms, invariants, brute force and independent library routines).
+and, for the MLP-half backward, tests/test_oracle_backward_pins.py (closed
+forms, invariants, brute force, finite differences and independent library
+routines).
 """
 from __future__ import annotations
 
@@ -293,3 +295,104 @@ def rank_forward_sharded(rank: int, D: int, x_local, k_full, v_full, w: dict,
 def causal_pairs(T: int, D: int, rank: int) -> int:
     """Number of (query, key) pairs rank `rank` scores: sum over its tokens of pos+1."""
     return int((zigzag_index(T, D, rank) + 1).sum())
+
+
+# ----------------------------------------------------------------------------
+# backward of the MLP half of the layer  [TSP ¶1: the validated workload is
+# training; ¶2, ¶4: the MLP is a sum over weight shards with no all-reduce]
+# ----------------------------------------------------------------------------
+# The pages give no backward; it is the chain rule applied to the forward
+# above.  For rows Y1 of the residual stream the MLP half is
+#     Xn2 = LN(Y1),  U = Xn2 W1,  H = GELU(U),  Y = Y1 + H W2,
+# and for a loss gradient dY the gradients are
+#     dH = dY W2^T,  dU = dH * GELU'(U),  dXn2 = dU W1^T,
+#     dY1 = dY + LN'(Y1)^T dXn2,  dW1 = Xn2^T dU,  dW2 = H^T dY.
+# Over shards, dW1 and dW2 split by FFN columns / rows exactly as W1 and W2
+# do, and dXn2 = sum_k dU_k W1_k^T is again a sum over shards.
+
+def gelu_tanh_grad(x) -> np.ndarray:
+    """Derivative of gelu_tanh: with s = sqrt(2/pi), a = 0.044715 and
+    t = tanh(s (x + a x^3)),  0.5 (1 + t) + 0.5 x (1 - t^2) s (1 + 3 a x^2)."""
+    x = np.asarray(x, dtype=np.float64)
+    s = np.sqrt(2.0 / np.pi)
+    t = np.tanh(s * (x + 0.044715 * x * x * x))
+    return 0.5 * (1.0 + t) + 0.5 * x * (1.0 - t * t) * s * (1.0 + 3.0 * 0.044715 * x * x)
+
+
+def layer_norm_backward(x, g, eps: float = LN_EPS) -> np.ndarray:
+    """Gradient with respect to x of sum(g * layer_norm(x)), row-wise:
+    rstd * (g - mean(g) - xhat * mean(g * xhat)), xhat = layer_norm(x),
+    rstd = 1 / sqrt(var + eps) (biased variance, gamma=1, beta=0)."""
+    x = np.asarray(x, dtype=np.float64)
+    g = np.asarray(g, dtype=np.float64)
+    mean = x.mean(axis=-1, keepdims=True)
+    centred = x - mean
+    var = (centred * centred).mean(axis=-1, keepdims=True)
+    rstd = 1.0 / np.sqrt(var + eps)
+    xhat = centred * rstd
+    return rstd * (g - g.mean(axis=-1, keepdims=True) - xhat * (g * xhat).mean(axis=-1, keepdims=True))
+
+
+def mlp_backward(y1, dy, w: dict, eps: float = LN_EPS, storage="fp16", grad_storage="bf16") -> dict:
+    """Gradients of the MLP half for rows y1 [n, h] given dY [n, h]:
+    {"dy1": [n, h], "dw1": [h, F], "dw2": [F, h]} (weights in the math
+    orientation [in, out]).
+
+    Precision model (the values the layer keeps in 16 bits, rounded to
+    nearest even; every product and sum in fp64):
+    * forward part, as in rank_rows_forward with `storage`: the weights, the
+      LN2 output Xn2 and the pre-activation U = Xn2 W1 are stored in
+      `storage`;
+    * backward part, in `grad_storage`: dU, and the copies of Xn2 and
+      H = GELU(U) that feed the weight-gradient products, are stored in
+      `grad_storage`; dY and the bf16 weights enter as given.  dH, dXn2, dY1,
+      dW1 and dW2 stay unrounded.
+    storage=None and grad_storage=None give the plain fp64 chain rule.
+    """
+    rnd, grnd = _rounder(storage), _rounder(grad_storage)
+    y1 = np.asarray(y1, dtype=np.float64)
+    dy = np.asarray(dy, dtype=np.float64)
+    w1 = np.asarray(w["w1"], dtype=np.float64)
+    w2 = np.asarray(w["w2"], dtype=np.float64)
+    xn2 = rnd(layer_norm(y1, eps))
+    u = rnd(xn2 @ rnd(w1))
+    hh = grnd(gelu_tanh(u))
+    dh = dy @ w2.T
+    du = grnd(dh * gelu_tanh_grad(u))
+    dxn2 = du @ w1.T
+    dy1 = dy + layer_norm_backward(y1, dxn2, eps)
+    dw1 = grnd(xn2).T @ du
+    dw2 = hh.T @ dy
+    return {"dy1": dy1, "dw1": dw1, "dw2": dw2, "du": du, "u": u}
+
+
+def mlp_backward_sampled(y1, dy, w: dict, rows, w1_cols, w2_rows, eps: float = LN_EPS,
+                         storage="fp16", grad_storage="bf16") -> dict:
+    """The outputs of mlp_backward at sampled places, each computed alone
+    with the same precision model: dY1 at rows `rows` (row-local), dW1 at
+    columns `w1_cols` (column j needs U[:, j] and dU[:, j] over all rows) and
+    dW2 at rows `w2_rows` (row f needs H[:, f]).  For sizes where the full
+    products are too slow on a CPU."""
+    rnd, grnd = _rounder(storage), _rounder(grad_storage)
+    y1 = np.asarray(y1, dtype=np.float64)
+    dy = np.asarray(dy, dtype=np.float64)
+    w1 = np.asarray(w["w1"], dtype=np.float64)
+    w2 = np.asarray(w["w2"], dtype=np.float64)
+    w1r = rnd(w1)
+    xn2 = rnd(layer_norm(y1, eps))
+    out = {}
+    # dY1 rows
+    r = np.asarray(rows)
+    u_r = rnd(xn2[r] @ w1r)
+    du_r = grnd((dy[r] @ w2.T) * gelu_tanh_grad(u_r))
+    out["dy1"] = dy[r] + layer_norm_backward(y1[r], du_r @ w1.T, eps)
+    # dW1 columns
+    c = np.asarray(w1_cols)
+    u_c = rnd(xn2 @ w1r[:, c])
+    du_c = grnd((dy @ w2[c, :].T) * gelu_tanh_grad(u_c))
+    out["dw1"] = grnd(xn2).T @ du_c
+    # dW2 rows
+    f = np.asarray(w2_rows)
+    h_f = grnd(gelu_tanh(rnd(xn2 @ w1r[:, f])))
+    out["dw2"] = h_f.T @ dy
+    return out
