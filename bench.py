@@ -481,6 +481,59 @@ def run_sweep_shards(args):
     print(json.dumps(line), flush=True)
 
 
+BWD_NAMES = ["ln2_u", "du", "dxn2", "ln2_bwd", "transposes", "dw1", "dw2"]
+
+
+def run_sweep_mlp_bwd(args):
+    """Backward of the MLP half for rank 0 of the 7B layer at T = 131072,
+    D = 8 (16384 tokens, seed 5): dY1, dW1, dW2 from Y1 and dY.  tokens/s =
+    L / backward time; the five matmuls (U recomputed, dU, dXn2, dW1, dW2)
+    are 2 L h F FLOPs each."""
+    import torch
+    from folded_tensor_sequence_rank_b200 import tsp
+    T, h, H, F, D = 131072, 4096, 32, 16384, 8
+    L = T // D
+    torch.cuda.set_device(0)
+    dims = tsp.make_dims(T, h, H, F)
+    rnd, w_full = _synthetic(T, h, F, 5)
+    sw = tsp.pack_shards(dims, D, w_full)
+    y1 = rnd(L, h, dtype=torch.float32)
+    dy = rnd(L, h)
+    dy1 = torch.empty(L, h, dtype=torch.float32, device="cuda")
+    dw1 = torch.empty(h, F, dtype=torch.float32, device="cuda")
+    dw2 = torch.empty(F, h, dtype=torch.float32, device="cuda")
+    bws = tsp.alloc_mlp_backward_workspace(dims, D)
+    for _ in range(args.warmup):
+        tsp.mlp_backward(dims, sw, w_full["w1"], w_full["w2"], y1, dy, dy1, dw1, dw2, bws)
+    steps = max(1, min(args.steps, 20))
+    clocks = ClockSampler(0)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(tsp.N_STEP_EVENTS)] for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(steps):
+        tsp.mlp_backward(dims, sw, w_full["w1"], w_full["w2"], y1, dy, dy1, dw1, dw2, bws, events=evs[i])
+    t1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    assert tsp.get_device_status(bws) == tsp.TSP_OK, "device wait timed out"
+    ms = t0.elapsed_time(t1) / steps
+    part = {n: statistics.median(e[j].elapsed_time(e[j + 1]) for e in evs) for j, n in enumerate(BWD_NAMES)}
+    gf = 2.0 * L * h * F
+    rate = {n: gf / (part[n] * 1e-3) / 1e12 for n in ("du", "dxn2", "dw1", "dw2")}
+    line = {"metric": "TSP MLP-half backward tokens/s on 1 B200 (7B layer, 128K, D=8, rank 0)",
+            "value": L / (ms * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "MLP half of the 7B layer, backward (dY1, dW1, dW2), T=131072, D=8, rank 0: "
+                                   "16384 tokens, Y1 ~ N(0,1) fp32, dY ~ N(0,1) bf16 (seed 5)",
+                       "l2": "inputs larger than L2; no flush"},
+            "tflop_per_step": 5 * gf / 1e12, "tflops": 5 * gf / (ms * 1e-3) / 1e12,
+            "part_ms": {k: round(v, 4) for k, v in part.items()},
+            "gemm_tflops": {k: round(v, 1) for k, v in rate.items()},
+            "clocks": clk}
+    print(json.dumps(line), flush=True)
+
+
 def run_sweep_stack(args):
     """A 32-layer stack of the 7B layer at T = 131072 on one GPU, all D = 8
     ranks in turn per layer (K/V projections, then layer forwards), random
@@ -541,9 +594,10 @@ def main():
     ap.add_argument("--impl", default="tsp", choices=["tsp", "reference"])
     ap.add_argument("--workload", default="7b-128k-d8", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--sweep", choices=["ranks", "shards", "stack"], default=None,
+    ap.add_argument("--sweep", choices=["ranks", "shards", "stack", "mlp_bwd"], default=None,
                     help="ranks: all 8 ranks of the 128K layer in turn (per-rank spread, whole-layer tokens/s); "
-                         "shards: rank 0 at T=32768 for D=1..16; stack: a 32-layer forward at 128K")
+                         "shards: rank 0 at T=32768 for D=1..16; stack: a 32-layer forward at 128K; "
+                         "mlp_bwd: the MLP-half backward of rank 0 at 128K")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -552,6 +606,8 @@ def main():
         run_sweep_ranks(args)
     elif args.sweep == "shards":
         run_sweep_shards(args)
+    elif args.sweep == "mlp_bwd":
+        run_sweep_mlp_bwd(args)
     elif args.sweep == "stack":
         run_sweep_stack(args)
     elif args.impl == "reference":

@@ -131,7 +131,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_pair_f16_tcgen05(const _
     }
   } else if (warp == 1) {
     if (cta == 0 && elect_one()) {
-      constexpr uint32_t idesc = idesc_f32acc(kPairBM, kPairBN, 0, 0, kFmtF16);
+      const uint32_t idesc = p.fmt_bf16 ? idesc_f32acc(kPairBM, kPairBN, 0, 0, kFmtBF16)
+                                        : idesc_f32acc(kPairBM, kPairBN, 0, 0, kFmtF16);
       constexpr uint16_t kBoth = 3;
       int stage = 0;
       uint32_t phase = 0;

@@ -1,7 +1,8 @@
 // gemm_sm100.cuh - persistent tcgen05 GEMM C = A * B^T for the TSP shard loops.
 //
-// A [M, K] fp16 K-major (one tensor map), B given as a list of per-shard
-// fp16 K-major tensor maps; fp32 accumulation in tensor memory.  Two ways the shard list is walked, both without any
+// A [M, K] K-major (one tensor map), B given as a list of per-shard K-major
+// tensor maps, both fp16 or both bf16 (fmt_bf16); fp32 accumulation in
+// tensor memory.  Two ways the shard list is walked, both without any
 // reduction kernel:
 //   N-split (Q/K/V and W1 shards: each shard owns a block of output columns):
 //     output column block n belongs to map n / shard_n.
@@ -30,7 +31,11 @@ constexpr int kGemmThreads = 192;
 constexpr int kGemmMaxMaps = 48;  // 3 segments x 16 shards
 constexpr int kGemmGroupM = 16;   // M tiles per raster group (L2 reuse of A)
 
-enum GemmEpi : int { kEpiStoreBf16 = 0, kEpiGeluBf16 = 1, kEpiResidual = 2 };
+// Epilogues.  kEpiStoreBf16 / kEpiGeluBf16 write fp16 operands for the next
+// matmul (the names keep the 16-bit operand role); kEpiResidual adds the
+// residual stream; kEpiGeluBwd writes the bf16 gradient acc * GELU'(U) with U
+// (fp16, [M, ldo]) at `resid`; kEpiStoreF32 writes acc as fp32.
+enum GemmEpi : int { kEpiStoreBf16 = 0, kEpiGeluBf16 = 1, kEpiResidual = 2, kEpiGeluBwd = 3, kEpiStoreF32 = 4 };
 
 struct __align__(64) GemmParams {
   CUtensorMap map_a;
@@ -41,6 +46,7 @@ struct __align__(64) GemmParams {
   int shard_k;    // K-split: reduction length per B map
   int seg_n;      // N-split: output columns per output segment
   int epi;        // GemmEpi
+  int fmt_bf16;   // operands: 0 fp16, 1 bf16
   void* out[3];   // per segment (N-split, fp16) or out[0] (K-split, fp32 / bf16)
   int remap[3];   // per segment: 1 = write local row m at its global zigzag row
   int64_t ldo;    // output row stride, elements
@@ -83,6 +89,18 @@ __device__ __forceinline__ float gelu_tanh_f(float x) {
   return x / (1.0f + ex2_approx(k * u));
 }
 
+// d/dx GELU (tanh form).  With p = 1 / (1 + e^(-2u)) = 0.5 (1 + tanh(u)),
+// 1 - tanh(u)^2 = 4 p (1 - p), so
+//   GELU'(x) = p + 2 x p (1 - p) sqrt(2/pi) (1 + 3 * 0.044715 x^2).
+__device__ __forceinline__ float gelu_tanh_grad_f(float x) {
+  const float s = 0.7978845608028654f;
+  const float k = -2.0f * 0.7978845608028654f * 1.4426950408889634f;  // -2 sqrt(2/pi) log2(e)
+  const float x2 = x * x;
+  const float u = fmaf(0.044715f * x, x2, x);
+  const float pr = 1.0f / (1.0f + ex2_approx(k * u));
+  return fmaf(2.0f * x * pr * (1.0f - pr) * s, fmaf(3.0f * 0.044715f, x2, 1.0f), pr);
+}
+
 // Bounded wait that ignores the abort flag: used only to drain copies and
 // MMAs this thread itself started, before the CTA exits.
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
@@ -97,6 +115,33 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, uint6
 // local row m (global zigzag row grow) and output columns n .. n+31.
 __device__ __forceinline__ void gemm_epilogue_chunk(const GemmParams& p, int m, int64_t grow, int n,
                                                     const uint32_t (&r)[32]) {
+  if (p.epi == kEpiStoreF32) {
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out[0]) + static_cast<int64_t>(m) * p.ldo + n);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]), __uint_as_float(r[4 * i + 2]),
+                           __uint_as_float(r[4 * i + 3]));
+    return;
+  }
+  if (p.epi == kEpiGeluBwd) {
+    const int64_t off = static_cast<int64_t>(m) * p.ldo + n;
+    const uint4* us = reinterpret_cast<const uint4*>(static_cast<const __half*>(p.resid) + off);
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out[0]) + off);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 q = us[i];
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 uf = __half22float2(*reinterpret_cast<const __half2*>(&w[j]));
+        o[j] = pack_bf16x2(__uint_as_float(r[8 * i + 2 * j]) * gelu_tanh_grad_f(uf.x),
+                           __uint_as_float(r[8 * i + 2 * j + 1]) * gelu_tanh_grad_f(uf.y));
+      }
+      dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    return;
+  }
   if (p.epi == kEpiResidual) {
     float v[32];
 #pragma unroll
@@ -239,7 +284,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_f16_tcgen05(const __grid
     }
   } else if (warp == 1) {
     if (elect_one()) {
-      constexpr uint32_t idesc = idesc_f32acc(kGemmBM, BN, 0, 0, kFmtF16);
+      const uint32_t idesc = p.fmt_bf16 ? idesc_f32acc(kGemmBM, BN, 0, 0, kFmtBF16)
+                                        : idesc_f32acc(kGemmBM, BN, 0, 0, kFmtF16);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;

@@ -2,6 +2,7 @@
 // zigzag index map, pre-LayerNorm with fp16 output, weight shard packing, and
 // the bounded-wait self test.
 #pragma once
+#include "gemm_sm100.cuh"
 #include "ptx.cuh"
 
 namespace tsp {
@@ -119,6 +120,146 @@ __global__ void pack_transpose_kernel(const __nv_bfloat16* __restrict__ w, int64
       uint16_t hbits;
       asm("cvt.rn.satfinite.f16.f32 %0, %1;" : "=h"(hbits) : "f"(tile[tx][k]));
       reinterpret_cast<uint16_t*>(out)[static_cast<int64_t>(o) * n_in + i] = hbits;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- backward helpers
+template <typename T>
+__device__ __forceinline__ float to_f32(T v);
+template <>
+__device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// out[c][r] = bf16(f(in[r][c])) for r < rows, c < cols, f = identity or GELU
+// (tanh form): the K-major [cols, rows] operand of a weight-gradient matmul
+// that reduces over the rows (tokens).  32 x 32 tiles staged through shared
+// memory so that both the reads and the writes are coalesced.
+template <typename Tin, bool GELU>
+__global__ void transpose_bf16_kernel(const Tin* __restrict__ in, int64_t rows, int cols, int64_t ldi,
+                                      __nv_bfloat16* __restrict__ out, int64_t ldo) {
+  __shared__ float tile[32][33];
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * 32;
+  const int c0 = blockIdx.y * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
+  for (int k = ty; k < 32; k += 8) {
+    const int64_t r = r0 + k;
+    const int c = c0 + tx;
+    if (r < rows && c < cols) {
+      float v = to_f32<Tin>(in[r * ldi + c]);
+      if (GELU) v = gelu_tanh_f(v);
+      tile[k][tx] = v;
+    }
+  }
+  __syncthreads();
+  for (int k = ty; k < 32; k += 8) {
+    const int c = c0 + k;
+    const int64_t r = r0 + tx;
+    if (r < rows && c < cols) out[static_cast<int64_t>(c) * ldo + r] = __float2bfloat16_rn(tile[tx][k]);
+  }
+}
+
+// Block-wide sum of `n` values per thread (n <= 2), 256 threads.
+__device__ __forceinline__ void block_sum2(float& a, float& b, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+    b += __shfl_xor_sync(0xffffffffu, b, o);
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) {
+    red[2 * warp] = a;
+    red[2 * warp + 1] = b;
+  }
+  __syncthreads();
+  a = 0.f;
+  b = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    a += red[2 * w];
+    b += red[2 * w + 1];
+  }
+}
+
+// LayerNorm backward with the residual, one row per 256-thread block:
+//   dy1 = dy + rstd * (g - mean(g) - xhat * mean(g * xhat)),
+//   xhat = (y1 - mean(y1)) * rstd, rstd = 1 / sqrt(var(y1) + eps)
+// (biased variance, gamma = 1, beta = 0), statistics in fp32 from the row
+// held in registers (VPT values per thread, as float4 groups).
+template <int VPT>
+__global__ void __launch_bounds__(256) ln_backward_rows_kernel(const float* __restrict__ y1,
+                                                               const float* __restrict__ g,
+                                                               const __nv_bfloat16* __restrict__ dy,
+                                                               float* __restrict__ dy1, int h, float eps) {
+  __shared__ float red[16];
+  const int64_t row = blockIdx.x;
+  const float* yr = y1 + row * h;
+  const float* gr = g + row * h;
+  float yv[VPT], gv[VPT];
+  float sum = 0.f, dummy = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPT / 4; ++i) {
+    const int col = (i * 256 + threadIdx.x) * 4;
+    if (col < h) {
+      const float4 a = *reinterpret_cast<const float4*>(yr + col);
+      const float4 b = *reinterpret_cast<const float4*>(gr + col);
+      yv[4 * i] = a.x; yv[4 * i + 1] = a.y; yv[4 * i + 2] = a.z; yv[4 * i + 3] = a.w;
+      gv[4 * i] = b.x; gv[4 * i + 1] = b.y; gv[4 * i + 2] = b.z; gv[4 * i + 3] = b.w;
+      sum += (a.x + a.y) + (a.z + a.w);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) yv[4 * i + j] = gv[4 * i + j] = 0.f;
+    }
+  }
+  block_sum2(sum, dummy, red);
+  const float mean = sum / h;
+  float sq = 0.f;
+  dummy = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPT / 4; ++i) {
+    const int col = (i * 256 + threadIdx.x) * 4;
+    if (col < h) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float d = yv[4 * i + j] - mean;
+        sq = fmaf(d, d, sq);
+      }
+    }
+  }
+  block_sum2(sq, dummy, red);
+  const float rstd = rsqrtf(sq / h + eps);
+  float sg = 0.f, sgx = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPT / 4; ++i) {
+    const int col = (i * 256 + threadIdx.x) * 4;
+    if (col < h) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        yv[4 * i + j] = (yv[4 * i + j] - mean) * rstd;  // xhat
+        sg += gv[4 * i + j];
+        sgx = fmaf(gv[4 * i + j], yv[4 * i + j], sgx);
+      }
+    }
+  }
+  block_sum2(sg, sgx, red);
+  const float mg = sg / h, mgx = sgx / h;
+  const __nv_bfloat16* dr = dy + row * h;
+  float* outr = dy1 + row * h;
+#pragma unroll
+  for (int i = 0; i < VPT / 4; ++i) {
+    const int col = (i * 256 + threadIdx.x) * 4;
+    if (col < h) {
+      const uint2 q = *reinterpret_cast<const uint2*>(dr + col);
+      const float2 d01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.x));
+      const float2 d23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.y));
+      float4 o;
+      o.x = d01.x + rstd * (gv[4 * i] - mg - yv[4 * i] * mgx);
+      o.y = d01.y + rstd * (gv[4 * i + 1] - mg - yv[4 * i + 1] * mgx);
+      o.z = d23.x + rstd * (gv[4 * i + 2] - mg - yv[4 * i + 2] * mgx);
+      o.w = d23.y + rstd * (gv[4 * i + 3] - mg - yv[4 * i + 3] * mgx);
+      *reinterpret_cast<float4*>(outr + col) = o;
     }
   }
 }

@@ -60,9 +60,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D fp16 row-major [rows, cols] with row stride ld elements; box = 64
-// columns (128 bytes, 128B swizzle) x box_rows rows.
-int make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld, int box_rows) {
+// 2-D fp16 (or bf16) row-major [rows, cols] with row stride ld elements;
+// box = 64 columns (128 bytes, 128B swizzle) x box_rows rows.
+int make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld, int box_rows,
+             bool bf16 = false) {
   auto fn = encode_fn();
   if (!fn) {
     std::snprintf(g_cuda_err, sizeof(g_cuda_err), "cuTensorMapEncodeTiled unavailable");
@@ -72,7 +73,8 @@ int make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
   cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
@@ -434,6 +436,79 @@ int layer_tail(Ctx& c, const tsp_dims* dims, const tsp_weights* w, int rank, con
   return record(ev, 7, st);
 }
 
+// ---------------------------------------------------------------- MLP backward
+struct BwdLayout {
+  size_t status, xn2, u, du, dxn2, xn2t, dut, ht, dyt, total;
+};
+
+BwdLayout bwd_layout(const Sizes& s) {
+  BwdLayout b;
+  const size_t Lh = static_cast<size_t>(s.L) * s.h, LF = static_cast<size_t>(s.L) * s.F;
+  size_t o = 0;
+  b.status = o; o += align_up(256);
+  b.xn2 = o; o += align_up(Lh * 2);
+  b.u = o; o += align_up(LF * 2);
+  b.du = o; o += align_up(LF * 2);
+  b.dxn2 = o; o += align_up(Lh * 4);
+  b.xn2t = o; o += align_up(Lh * 2);
+  b.dut = o; o += align_up(LF * 2);
+  b.ht = o; o += align_up(LF * 2);
+  b.dyt = o; o += align_up(Lh * 2);
+  b.total = o;
+  return b;
+}
+
+// C [M, N] = A [M, K] * B [N, K]^T with one B map: A and B K-major with row
+// strides lda / ldb, both fp16 or both bf16; epilogue kEpiStoreF32 (out fp32)
+// or kEpiGeluBwd (out bf16, aux = U fp16), row stride ldo.
+int launch_plain(const void* a, int M, int K, int64_t lda, const void* b, int N, int64_t ldb, bool bf16, int epi,
+                 void* out, int64_t ldo, const void* aux, int* status, cudaStream_t st) {
+  static thread_local GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  const int bn = pick_bn(N);
+  int rc = make_map(&p.map_a, a, M, K, lda, kGemmBM, bf16);
+  if (rc) return rc;
+  rc = make_map(&p.map_b[0], b, N, K, ldb, b_box_rows(bn), bf16);
+  if (rc) return rc;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.ksplit = 0;
+  p.shard_n = N;
+  p.shard_k = K;
+  p.seg_n = N;
+  p.epi = epi;
+  p.fmt_bf16 = bf16 ? 1 : 0;
+  p.out[0] = out;
+  p.ldo = ldo;
+  p.resid = aux;
+  p.status = status;
+  p.timeout_ns = kDefaultTimeoutNs;
+  return launch_gemm(p, bn, st);
+}
+
+template <typename Tin, bool GELU>
+int launch_transpose(const Tin* in, int64_t rows, int cols, __nv_bfloat16* out, cudaStream_t st) {
+  if (rows == 0) return TSP_OK;
+  const dim3 grid(static_cast<unsigned>((rows + 31) / 32), static_cast<unsigned>((cols + 31) / 32));
+  transpose_bf16_kernel<Tin, GELU><<<grid, dim3(32, 8), 0, st>>>(in, rows, cols, cols, out, rows);
+  TSP_CUDA(cudaGetLastError());
+  return TSP_OK;
+}
+
+int launch_ln_backward(const float* y1, const float* g, const __nv_bfloat16* dy, float* dy1, int64_t rows, int h,
+                       float eps, cudaStream_t st) {
+  if (rows == 0) return TSP_OK;
+  const int groups = (h + 1023) / 1024;  // float4 groups per thread
+  const dim3 grid(static_cast<unsigned>(rows));
+  if (groups <= 1) ln_backward_rows_kernel<4><<<grid, 256, 0, st>>>(y1, g, dy, dy1, h, eps);
+  else if (groups <= 2) ln_backward_rows_kernel<8><<<grid, 256, 0, st>>>(y1, g, dy, dy1, h, eps);
+  else if (groups <= 4) ln_backward_rows_kernel<16><<<grid, 256, 0, st>>>(y1, g, dy, dy1, h, eps);
+  else ln_backward_rows_kernel<32><<<grid, 256, 0, st>>>(y1, g, dy, dy1, h, eps);
+  TSP_CUDA(cudaGetLastError());
+  return TSP_OK;
+}
+
 // ---------------------------------------------------------------- allocation-free K/V projection
 // Scratch for tsp_kv_project_noalloc: a file-scope device array, so the call
 // needs no device allocation.  Layout: status word (256 B), 768 B spare, then
@@ -688,6 +763,85 @@ int tsp_rank_step_host(const tsp_dims* dims, const tsp_weights* w, int rank, con
   if (rc) return rc;
   TSP_CUDA(cudaMemcpyAsync(h_y_local, d_y_staging, yb, cudaMemcpyDeviceToHost, stream));
   return TSP_OK;
+}
+
+size_t tsp_mlp_backward_workspace_bytes(const tsp_dims* dims, int D) {
+  if (check_dims(dims, D) != TSP_OK) return 0;
+  return bwd_layout(sizes_of(dims, D)).total;
+}
+
+int tsp_mlp_backward(const tsp_dims* dims, const tsp_weights* w, const void* w1_full, const void* w2_full,
+                     const void* y1, const void* dy, void* dy1, void* dw1, void* dw2, void* bws, size_t bws_bytes,
+                     cudaStream_t stream, cudaEvent_t* ev) {
+  const int D = w ? w->D : 0;
+  int rc = check_dims(dims, D);
+  if (rc) return rc;
+  rc = check_weights(w, D);
+  if (rc) return rc;
+  const Sizes s = sizes_of(dims, D);
+  // with no tokens only the weight gradients (zeros) are written
+  const void* ptrs[7] = {w1_full, w2_full, dw1, dw2, y1, dy, dy1};
+  for (int i = 0; i < (s.L == 0 ? 4 : 7); ++i)
+    if (!ptrs[i] || !aligned16(ptrs[i])) return TSP_ERR_INVALID_ARG;
+  if (!bws || (reinterpret_cast<uintptr_t>(bws) & 255)) return TSP_ERR_INVALID_ARG;
+  if (s.h % 256 || s.F % 256) return TSP_ERR_UNSUPPORTED;
+  const BwdLayout b = bwd_layout(s);
+  if (bws_bytes < b.total) return TSP_ERR_WORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(bws);
+  int* status = reinterpret_cast<int*>(base + b.status);
+  if ((rc = record(ev, 0, stream))) return rc;
+  if (s.L == 0) {  // no tokens: zero weight gradients
+    TSP_CUDA(cudaMemsetAsync(dw1, 0, static_cast<size_t>(s.h) * s.F * 4, stream));
+    TSP_CUDA(cudaMemsetAsync(dw2, 0, static_cast<size_t>(s.F) * s.h * 4, stream));
+    for (int i = 1; i < TSP_N_STEP_EVENTS; ++i)
+      if ((rc = record(ev, i, stream))) return rc;
+    return TSP_OK;
+  }
+  __half* xn2 = reinterpret_cast<__half*>(base + b.xn2);
+  __half* u = reinterpret_cast<__half*>(base + b.u);
+  __nv_bfloat16* du = reinterpret_cast<__nv_bfloat16*>(base + b.du);
+  float* dxn2 = reinterpret_cast<float*>(base + b.dxn2);
+  __nv_bfloat16* xn2t = reinterpret_cast<__nv_bfloat16*>(base + b.xn2t);
+  __nv_bfloat16* dut = reinterpret_cast<__nv_bfloat16*>(base + b.dut);
+  __nv_bfloat16* ht = reinterpret_cast<__nv_bfloat16*>(base + b.ht);
+  __nv_bfloat16* dyt = reinterpret_cast<__nv_bfloat16*>(base + b.dyt);
+  const int L = static_cast<int>(s.L);
+  // Xn2 = LN2(Y1), U = Xn2 W1 (fp16 shards, as in the forward)
+  rc = launch_layernorm<float>(static_cast<const float*>(y1), xn2, s.L, s.h, dims->ln_eps, stream);
+  if (rc) return rc;
+  const void* const* w1fam[3] = {reinterpret_cast<const void* const*>(w->w1), nullptr, nullptr};
+  void* uout[3] = {u, nullptr, nullptr};
+  const int noremap[3] = {0, 0, 0};
+  rc = launch_proj(s, 0, xn2, w1fam, uout, noremap, 1, kEpiStoreBf16, s.F, status, stream);
+  if (rc) return rc;
+  if ((rc = record(ev, 1, stream))) return rc;
+  // dU = (dY W2^T) * GELU'(U): B = W2 [F, h] is K-major over h
+  rc = launch_plain(dy, L, s.h, s.h, w2_full, s.F, s.h, true, kEpiGeluBwd, du, s.F, u, status, stream);
+  if (rc) return rc;
+  if ((rc = record(ev, 2, stream))) return rc;
+  // dXn2 = dU W1^T: B = W1 [h, F] is K-major over F
+  rc = launch_plain(du, L, s.F, s.F, w1_full, s.h, s.F, true, kEpiStoreF32, dxn2, s.h, nullptr, status, stream);
+  if (rc) return rc;
+  if ((rc = record(ev, 3, stream))) return rc;
+  // dY1 = dY + LN2'(Y1)^T dXn2
+  rc = launch_ln_backward(static_cast<const float*>(y1), dxn2, static_cast<const __nv_bfloat16*>(dy),
+                          static_cast<float*>(dy1), s.L, s.h, dims->ln_eps, stream);
+  if (rc) return rc;
+  if ((rc = record(ev, 4, stream))) return rc;
+  // token-major operands of the weight gradients (reduction over the tokens)
+  if ((rc = launch_transpose<__half, false>(xn2, s.L, s.h, xn2t, stream))) return rc;
+  if ((rc = launch_transpose<__nv_bfloat16, false>(du, s.L, s.F, dut, stream))) return rc;
+  if ((rc = launch_transpose<__half, true>(u, s.L, s.F, ht, stream))) return rc;
+  if ((rc = launch_transpose<__nv_bfloat16, false>(static_cast<const __nv_bfloat16*>(dy), s.L, s.h, dyt, stream)))
+    return rc;
+  if ((rc = record(ev, 5, stream))) return rc;
+  // dW1 [h, F] = Xn2^T dU ; dW2 [F, h] = GELU(U)^T dY
+  rc = launch_plain(xn2t, s.h, L, L, dut, s.F, L, true, kEpiStoreF32, dw1, s.F, nullptr, status, stream);
+  if (rc) return rc;
+  if ((rc = record(ev, 6, stream))) return rc;
+  rc = launch_plain(ht, s.F, L, L, dyt, s.h, L, true, kEpiStoreF32, dw2, s.h, nullptr, status, stream);
+  if (rc) return rc;
+  return record(ev, 7, stream);
 }
 
 int tsp_selftest_wait_timeout(void* ws, uint64_t timeout_ns, cudaStream_t stream) {

@@ -17,6 +17,9 @@ each tensor rounded once to bf16 round-to-nearest-even):
   K and V in) instead of bf16.  ``kv_std`` defaults to 0.02*sqrt(h), the
   standard deviation of LayerNorm(x) @ W for such weights, so attention
   logits have the spread the real projection gives.
+* ``mlp_backward_inputs``: the rank's residual rows Y1 [L, h] ~ N(0, 1) kept
+  in fp32 (the residual stream is fp32), the six weights as above, then the
+  loss gradient dY [L, h] ~ N(0, 1) rounded to bf16.
 """
 from __future__ import annotations
 
@@ -61,6 +64,16 @@ def rank_inputs(L: int, T: int, h: int, F: int, seed: int,
     out.update(_weights(gen, h, F))
     out["k_full"] = _draw(gen, (T, h), kv_std, torch.float16)
     out["v_full"] = _draw(gen, (T, h), kv_std, torch.float16)
+    return out
+
+
+def mlp_backward_inputs(L: int, h: int, F: int, seed: int) -> dict:
+    """Residual rows Y1 (fp32), the weights (bf16) and a loss gradient dY (bf16); CPU."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(seed)
+    out = {"y1": _draw(gen, (L, h), 1.0, torch.float32)}
+    out.update(_weights(gen, h, F))
+    out["dy"] = _draw(gen, (L, h), 1.0)
     return out
 
 

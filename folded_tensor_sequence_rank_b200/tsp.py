@@ -75,6 +75,8 @@ def lib() -> ctypes.CDLL:
         "tsp_rank_step": (i32, [pd, pw, i32, vp, vp, vp, vp, i32, vp, sz, vp, ctypes.POINTER(vp)]),
         "tsp_rank_step_host": (i32, [pd, pw, i32, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]),
         "tsp_selftest_wait_timeout": (i32, [vp, ctypes.c_uint64, vp]),
+        "tsp_mlp_backward_workspace_bytes": (sz, [pd, i32]),
+        "tsp_mlp_backward": (i32, [pd, pw, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, ctypes.POINTER(vp)]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -262,6 +264,31 @@ def rank_step(dims: Dims, w: ShardedWeights, rank: int, x_local, k_full, v_full,
     yd = OUT_F32 if y_local.dtype == torch.float32 else OUT_BF16
     _check(lib().tsp_rank_step(ctypes.byref(dims), ctypes.byref(w.struct), rank, px, pk, pv, py, yd, pws,
                                ws.numel(), _stream(stream), _events(events)), "tsp_rank_step")
+
+
+def mlp_backward_workspace_bytes(dims: Dims, D: int) -> int:
+    return lib().tsp_mlp_backward_workspace_bytes(ctypes.byref(dims), D)
+
+
+def alloc_mlp_backward_workspace(dims: Dims, D: int, device="cuda") -> torch.Tensor:
+    n = mlp_backward_workspace_bytes(dims, D)
+    if n == 0:
+        _check(check_dims(dims, D) or TSP_ERR_INVALID_ARG, "tsp_mlp_backward_workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def mlp_backward(dims: Dims, w: ShardedWeights, w1_full, w2_full, y1, dy, dy1, dw1, dw2, bws,
+                 stream=None, events=None):
+    """Backward of the MLP half for one rank's rows: dy1 = dL/dY1, dw1 = dL/dW1 [h, F],
+    dw2 = dL/dW2 [F, h] (fp32), from y1 (fp32) and dy (bf16) [T/D, h], rank-local order.
+    w1_full [h, F] and w2_full [F, h] are the full bf16 weights in the math orientation."""
+    L, h, F = dims.T // w.D, dims.h, dims.ffn
+    args = [_ptr(w1_full, "w1_full", torch.bfloat16, (h, F)), _ptr(w2_full, "w2_full", torch.bfloat16, (F, h)),
+            _ptr(y1, "y1", torch.float32, (L, h)) if L else None, _ptr(dy, "dy", torch.bfloat16, (L, h)) if L else None,
+            _ptr(dy1, "dy1", torch.float32, (L, h)) if L else None, _ptr(dw1, "dw1", torch.float32, (h, F)),
+            _ptr(dw2, "dw2", torch.float32, (F, h))]
+    _check(lib().tsp_mlp_backward(ctypes.byref(dims), ctypes.byref(w.struct), *args, _ptr(bws, "bws", torch.uint8),
+                                  bws.numel(), _stream(stream), _events(events)), "tsp_mlp_backward")
 
 
 def rank_step_host(dims: Dims, w: ShardedWeights, rank: int, h_x_local, x_staging, k_full, v_full,

@@ -227,6 +227,39 @@ int tsp_rank_step_host(const tsp_dims* dims, const tsp_weights* w, int rank,
                        void* h_y_local, int y_dtype, void* ws, size_t ws_bytes,
                        cudaStream_t stream);
 
+/* Workspace bytes of tsp_mlp_backward at this D (its own status word first,
+ * then the recomputed and transposed activations); 0 on a bad argument. */
+size_t tsp_mlp_backward_workspace_bytes(const tsp_dims* dims, int D);
+
+/* Backward of the MLP half of the layer for one rank's tokens [zubnet.ai
+ * TSP item, paragraph 1: the validated workload is training; paragraphs
+ * 2 and 4: the MLP is a sum over FFN shards with no all-reduce].  For the
+ * rank's residual rows Y1 and the loss gradient dY of Y = Y1 + GELU(LN2(Y1)
+ * W1) W2 (the chain rule; the pages give no backward):
+ *   Xn2 = LN2(Y1) and U = Xn2 W1 are recomputed (fp16, as in the forward;
+ *   U by the fp16 shards in `w`),
+ *   dU = (dY W2^T) * GELU'(U)        (bf16),
+ *   dY1 = dY + LN2'(Y1)^T (dU W1^T)  (fp32),
+ *   dW1 = Xn2^T dU,  dW2 = GELU(U)^T dY  (fp32, summed over the rank's
+ *   tokens; Xn2 and GELU(U) enter these two products as bf16).
+ * The products with dY, dU and their transposes run on bf16 tensor-core
+ * operands: W1 and W2 are read from the caller's full bf16 weights in the
+ * math orientation, w1_full [h, F] and w2_full [F, h] row-major.  Shard k's
+ * gradient is columns k*F/D .. (k+1)*F/D-1 of dW1 and the same rows of dW2.
+ * y1: fp32 [T/D, h] and dy: bf16 [T/D, h], both rank-local order (read
+ * only); dy1: fp32 [T/D, h]; dw1: fp32 [h, F]; dw2: fp32 [F, h]; every
+ * pointer 16-byte aligned.  With T = 0 only dw1 and dw2 are written (zeros)
+ * and y1, dy, dy1 may be NULL.  bws: tsp_mlp_backward_workspace_bytes(dims, D)
+ * bytes, also the status word that tsp_get_device_status reads.  h and F
+ * must be multiples of 256.  step_events: NULL, or TSP_N_STEP_EVENTS
+ * caller-created events recorded on `stream` before the first launch and
+ * after LN2 + U, dU, dXn2, the LN2 backward, the transposes, dW1 and dW2. */
+int tsp_mlp_backward(const tsp_dims* dims, const tsp_weights* w,
+                     const void* w1_full, const void* w2_full,
+                     const void* y1, const void* dy, void* dy1, void* dw1, void* dw2,
+                     void* bws, size_t bws_bytes, cudaStream_t stream,
+                     cudaEvent_t* step_events);
+
 /* Fault-detection self test: launches one block that waits on a barrier
  * nothing will ever complete, with a limit of `timeout_ns` nanoseconds
  * (at most 2e9).  The wait gives up, the kernel records TSP_ERR_TIMEOUT in

@@ -154,3 +154,36 @@ def test_memory_account_7b_forward():
     assert acc["workspace"] == tsp.workspace_bytes(dims, 8) > 0
     assert acc["total"] == sum(v for k, v in acc.items() if k != "total")
     assert 5.0 < acc["total"] / 2**30 < 6.0
+
+
+def test_mlp_backward_argument_checks(L):
+    d = dims()
+    w = tsp.Weights()
+    w.D = 2
+    for name in tsp.WEIGHT_NAMES:
+        arr = getattr(w, name)
+        for k in range(2):
+            arr[k] = 0x10000 * (k + 1)
+    n = L.tsp_mlp_backward_workspace_bytes(ctypes.byref(d), 2)
+    L_tok, h, F = 256, 256, 1024
+    # the backward workspace holds at least the recomputed and transposed activations
+    assert n >= L_tok * (h * 2 + F * 2 * 4 + h * 4 + h * 2 * 2)
+    assert L.tsp_mlp_backward_workspace_bytes(ctypes.byref(dims(T=510)), 2) == 0
+    ok = [16] * 7
+    # a null or misaligned pointer
+    for i in range(7):
+        args = list(ok)
+        args[i] = None
+        assert L.tsp_mlp_backward(ctypes.byref(d), ctypes.byref(w), *args, 256, n, None, None) == tsp.TSP_ERR_INVALID_ARG
+        args[i] = 24
+        assert L.tsp_mlp_backward(ctypes.byref(d), ctypes.byref(w), *args, 256, n, None, None) == tsp.TSP_ERR_INVALID_ARG
+    # workspace: misaligned, then too small
+    assert L.tsp_mlp_backward(ctypes.byref(d), ctypes.byref(w), *ok, 272, n, None, None) == tsp.TSP_ERR_INVALID_ARG
+    assert L.tsp_mlp_backward(ctypes.byref(d), ctypes.byref(w), *ok, 256, n - 1, None, None) == tsp.TSP_ERR_WORKSPACE
+    # h not a multiple of 256
+    d2 = dims(T=768, h=192, H=3, F=768)
+    w.D = 3
+    for name in tsp.WEIGHT_NAMES:
+        getattr(w, name)[2] = 0x30000
+    n2 = L.tsp_mlp_backward_workspace_bytes(ctypes.byref(d2), 3)
+    assert L.tsp_mlp_backward(ctypes.byref(d2), ctypes.byref(w), *ok, 256, n2, None, None) == tsp.TSP_ERR_UNSUPPORTED

@@ -1,0 +1,99 @@
+"""Parity of tsp_mlp_backward (the MLP half of the layer's backward) against
+the fp64 oracle, through the C ABI.
+
+Tolerance: the oracle stores in 16 bits exactly the values the CUDA path
+stores (Xn2 and U in fp16; dU and the weight-gradient copies of Xn2 and
+GELU(U) in bf16), so what remains is fp32 accumulation order over K = h, F or
+the L tokens (relative ~sqrt(K) * 2^-24, about 1e-5), the ex2-based GELU'
+(2^-22), and rare one-ulp flips of a stored 16-bit value where fp32 and fp64
+round differently.  Bound: rel-L2 <= 1e-3 and max-abs <= 1e-2 * max |ref|
+per output, about 100x the measured errors.
+"""
+import numpy as np
+import pytest
+import torch
+
+from folded_tensor_sequence_rank_b200 import inputs, tsp
+from oracle import tsp_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+REL_L2 = 1e-3
+REL_MAX = 1e-2
+
+
+def _run(T, h, H, F, D, seed, zero_dy=False):
+    L = T // D
+    raw = inputs.mlp_backward_inputs(L, h, F, seed)
+    if zero_dy:
+        raw["dy"] = torch.zeros_like(raw["dy"])
+    dims = tsp.make_dims(T, h, H, F)
+    dev = {n: raw[n].cuda() for n in inputs.WEIGHT_NAMES}
+    sw = tsp.pack_shards(dims, D, dev)
+    y1, dy = raw["y1"].cuda(), raw["dy"].cuda()
+    dy1 = torch.full((L, h), float("nan"), device="cuda")
+    dw1 = torch.full((h, F), float("nan"), device="cuda")
+    dw2 = torch.full((F, h), float("nan"), device="cuda")
+    bws = tsp.alloc_mlp_backward_workspace(dims, D)
+    tsp.mlp_backward(dims, sw, dev["w1"], dev["w2"], y1, dy, dy1, dw1, dw2, bws)
+    assert tsp.get_device_status(bws) == tsp.TSP_OK
+    got = {k: v.double().cpu().numpy() for k, v in (("dy1", dy1), ("dw1", dw1), ("dw2", dw2))}
+    return raw, got
+
+
+def _close(name, got, ref):
+    assert np.isfinite(got).all(), name
+    err = float(np.abs(got - ref).max())
+    scale = float(np.abs(ref).max())
+    rel = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+    assert err <= REL_MAX * scale and rel <= REL_L2, f"{name}: max-abs {err:.3e} (scale {scale:.3e}) rel-L2 {rel:.3e}"
+
+
+@pytest.mark.parametrize("T,h,H,F,D,seed", [
+    (512, 256, 4, 1024, 2, 21),      # L = 256: one 256-row tile
+    (1024, 512, 4, 2048, 4, 22),     # D = 4
+    (3072, 256, 4, 1024, 2, 23),     # L = 1536: several M tiles
+])
+def test_mlp_backward_matches_oracle(T, h, H, F, D, seed):
+    raw, got = _run(T, h, H, F, D, seed)
+    w = {n: raw[n].double().numpy() for n in ("w1", "w2")}
+    ref = O.mlp_backward(raw["y1"].double().numpy(), raw["dy"].double().numpy(), w)
+    for k in ("dy1", "dw1", "dw2"):
+        _close(k, got[k], ref[k])
+
+
+def test_mlp_backward_7b_128k_sampled():
+    """The 7B layer at 128K, D = 8 (one rank: 16384 tokens): sampled rows of
+    dY1, columns of dW1 and rows of dW2, each computed alone by the oracle."""
+    T, h, H, F, D, seed = 131072, 4096, 32, 16384, 8, 24
+    raw, got = _run(T, h, H, F, D, seed)
+    L = T // D
+    rows = inputs.sample_rows(L, 14, seed, must=(0, L - 1))
+    cols = inputs.sample_rows(F, 14, seed + 1, must=(0, F - 1))
+    frows = inputs.sample_rows(F, 14, seed + 2, must=(0, F - 1))
+    w = {n: raw[n].double().numpy() for n in ("w1", "w2")}
+    ref = O.mlp_backward_sampled(raw["y1"].double().numpy(), raw["dy"].double().numpy(), w, rows, cols, frows)
+    _close("dy1", got["dy1"][rows], ref["dy1"])
+    _close("dw1", got["dw1"][:, cols], ref["dw1"])
+    _close("dw2", got["dw2"][frows, :], ref["dw2"])
+
+
+def test_zero_gradient_gives_zeros():
+    """dY = 0: every gradient is exactly zero (no term survives)."""
+    _, got = _run(512, 256, 4, 1024, 2, 25, zero_dy=True)
+    for k in ("dy1", "dw1", "dw2"):
+        assert not np.any(got[k]), k
+
+
+def test_empty_sequence_zeroes_weight_gradients():
+    dims = tsp.make_dims(0, 256, 4, 1024)
+    raw = inputs.mlp_backward_inputs(0, 256, 1024, 26)
+    dev = {n: raw[n].cuda() for n in inputs.WEIGHT_NAMES}
+    sw = tsp.pack_shards(dims, 2, dev)
+    dw1 = torch.full((256, 1024), 7.0, device="cuda")
+    dw2 = torch.full((1024, 256), 7.0, device="cuda")
+    bws = tsp.alloc_mlp_backward_workspace(dims, 2)
+    empty = torch.empty(0, 256, device="cuda")
+    tsp.mlp_backward(dims, sw, dev["w1"], dev["w2"], empty, empty.bfloat16(), empty, dw1, dw2, bws)
+    torch.cuda.synchronize()
+    assert not dw1.any() and not dw2.any()
