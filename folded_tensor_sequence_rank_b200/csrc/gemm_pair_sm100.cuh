@@ -37,7 +37,7 @@ struct GemmPairShape {
   static constexpr int kStages = 6;
   static constexpr int kTmemCols = 2 * kPairBN;  // two accumulators of 256 columns
   static constexpr int kBarBytes = 256;
-  static constexpr int kSmemBytes = kStages * (kABytes + kBBytes) + kBarBytes + 1024;
+  static constexpr int kSmemBytes = kStages * (kABytes + kBBytes) + kBarBytes + kStageBytes + 1024;
 };
 
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_pair_f16_tcgen05(const __grid_constant__ GemmParams p) {
@@ -164,6 +164,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_pair_f16_tcgen05(const _
   } else {
     // epilogue warps 2..5 -> TMEM lane quarters 2,3,0,1 of this CTA's 128 rows
     const int quarter = warp & 3;
+    uint32_t* stage = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(bars) + S::kBarBytes) +
+                      (warp - 2) * kStageWords;  // this warp's transpose buffer
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     int acc = 0;
@@ -183,7 +185,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_pair_f16_tcgen05(const _
         __syncwarp();
         tmem_ld32(tmem_base + lane_off + buf * kPairBN + ch * 32, r);
         tmem_ld_wait();
-        if (valid) gemm_epilogue_chunk(p, m, grow, nb * kPairBN + ch * 32, r);
+        if (valid) gemm_epilogue_chunk(p, m, grow, nb * kPairBN + ch * 32, r, stage);
       }
       tc_fence_before();
       __syncwarp();

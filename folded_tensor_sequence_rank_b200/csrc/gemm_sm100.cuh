@@ -35,6 +35,12 @@ constexpr int kGemmGroupM = 16;   // M tiles per raster group (L2 reuse of A)
 // matmul (the names keep the 16-bit operand role); kEpiResidual adds the
 // residual stream; kEpiGeluBwd writes the bf16 gradient acc * GELU'(U) with U
 // (fp16, [M, ldo]) at `resid`; kEpiStoreF32 writes acc as fp32.
+// kEpiStoreBf16 and kEpiGeluBwd can also write the tile transposed, as bf16,
+// to out_t [N, ld_t] (row n, column m): kEpiStoreBf16 writes GELU of the
+// fp16-rounded value there, kEpiGeluBwd the gradient itself.  A warp holds 32
+// consecutive rows; it transposes each 32 x 32 chunk through its own slice of
+// shared memory, so every lane writes one 64-byte output row segment.  The
+// transposed store needs every lane of the warp (M a multiple of 128).
 enum GemmEpi : int { kEpiStoreBf16 = 0, kEpiGeluBf16 = 1, kEpiResidual = 2, kEpiGeluBwd = 3, kEpiStoreF32 = 4 };
 
 struct __align__(64) GemmParams {
@@ -47,6 +53,8 @@ struct __align__(64) GemmParams {
   int seg_n;      // N-split: output columns per output segment
   int epi;        // GemmEpi
   int fmt_bf16;   // operands: 0 fp16, 1 bf16
+  void* out_t;    // optional transposed bf16 copy [N, ld_t] (see above)
+  int64_t ld_t;
   void* out[3];   // per segment (N-split, fp16) or out[0] (K-split, fp32 / bf16)
   int remap[3];   // per segment: 1 = write local row m at its global zigzag row
   int64_t ldo;    // output row stride, elements
@@ -59,6 +67,12 @@ struct __align__(64) GemmParams {
   uint64_t timeout_ns;
 };
 
+// Per epilogue warp: 16 words x 32 rows, row stride 36 words (16-byte
+// aligned, and the 128-bit reads of one transposed row spread over banks).
+constexpr int kStageStride = 36;
+constexpr int kStageWords = 16 * kStageStride;
+constexpr int kStageBytes = 4 * kStageWords * 4;
+
 template <int BN>
 struct GemmShape {
   static constexpr int kABytes = kGemmBM * kGemmBK * 2;
@@ -66,7 +80,7 @@ struct GemmShape {
   static constexpr int kStages = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);
   static constexpr int kTmemCols = 2 * BN;  // two accumulators
   static constexpr int kBarBytes = 256;
-  static constexpr int kSmemBytes = kStages * (kABytes + kBBytes) + kBarBytes + 1024;
+  static constexpr int kSmemBytes = kStages * (kABytes + kBBytes) + kBarBytes + kStageBytes + 1024;
 };
 
 __device__ __forceinline__ void gemm_tile_coords(int tile, int num_m, int num_n, int& mb, int& nb) {
@@ -97,7 +111,7 @@ __device__ __forceinline__ float gelu_tanh_grad_f(float x) {
   const float k = -2.0f * 0.7978845608028654f * 1.4426950408889634f;  // -2 sqrt(2/pi) log2(e)
   const float x2 = x * x;
   const float u = fmaf(0.044715f * x, x2, x);
-  const float pr = 1.0f / (1.0f + ex2_approx(k * u));
+  const float pr = __frcp_rn(1.0f + ex2_approx(k * u));
   return fmaf(2.0f * x * pr * (1.0f - pr) * s, fmaf(3.0f * 0.044715f, x2, 1.0f), pr);
 }
 
@@ -111,10 +125,37 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, uint6
   }
 }
 
+// Writes the 32 x 32 bf16 chunk whose row m (this lane) holds w[k] =
+// columns (n + 2k, n + 2k + 1) as rows n .. n+31 of out_t: each lane packs
+// its words into `stage` (word k of row `lane` at k * kStageStride + lane),
+// then reads back the column pair of output row n + lane with 128-bit loads
+// and joins rows 2i, 2i+1 with a byte permute.
+__device__ __forceinline__ void store_transposed_bf16(const GemmParams& p, uint32_t* stage, int m, int n,
+                                                      const uint32_t (&w)[16]) {
+  const int lane = threadIdx.x & 31;
+  __syncwarp();
+#pragma unroll
+  for (int k = 0; k < 16; ++k) stage[k * kStageStride + lane] = w[k];
+  __syncwarp();
+  const uint32_t* col = stage + (lane >> 1) * kStageStride;
+  const uint32_t sel = (lane & 1) ? 0x7632u : 0x5410u;  // high or low halves of two words
+  uint32_t o[16];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const uint4 v = *reinterpret_cast<const uint4*>(col + 4 * q);
+    o[2 * q] = __byte_perm(v.x, v.y, sel);
+    o[2 * q + 1] = __byte_perm(v.z, v.w, sel);
+  }
+  uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out_t) + static_cast<int64_t>(n + lane) * p.ld_t +
+                                        (m - lane));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+}
+
 // One 32-column chunk of an output tile's epilogue: accumulator values r for
 // local row m (global zigzag row grow) and output columns n .. n+31.
 __device__ __forceinline__ void gemm_epilogue_chunk(const GemmParams& p, int m, int64_t grow, int n,
-                                                    const uint32_t (&r)[32]) {
+                                                    const uint32_t (&r)[32], uint32_t* stage) {
   if (p.epi == kEpiStoreF32) {
     float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out[0]) + static_cast<int64_t>(m) * p.ldo + n);
 #pragma unroll
@@ -127,6 +168,7 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const GemmParams& p, int m, 
     const int64_t off = static_cast<int64_t>(m) * p.ldo + n;
     const uint4* us = reinterpret_cast<const uint4*>(static_cast<const __half*>(p.resid) + off);
     uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out[0]) + off);
+    uint32_t tw[16];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const uint4 q = us[i];
@@ -139,7 +181,10 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const GemmParams& p, int m, 
                            __uint_as_float(r[8 * i + 2 * j + 1]) * gelu_tanh_grad_f(uf.y));
       }
       dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) tw[4 * i + j] = o[j];
     }
+    if (p.out_t) store_transposed_bf16(p, stage, m, n, tw);
     return;
   }
   if (p.epi == kEpiResidual) {
@@ -197,6 +242,15 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const GemmParams& p, int m, 
 #pragma unroll
     for (int i = 0; i < 4; ++i)
       dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+    if (p.out_t) {  // bf16(GELU(fp16 value)), transposed
+      uint32_t tw[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&packed[i]));
+        tw[i] = pack_bf16x2(gelu_tanh_f(f.x), gelu_tanh_f(f.y));
+      }
+      store_transposed_bf16(p, stage, m, n, tw);
+    }
   }
 }
 
@@ -318,6 +372,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_f16_tcgen05(const __grid
   } else {
     // epilogue warps 2..5 -> TMEM lane quarters 2,3,0,1
     const int quarter = warp & 3;
+    uint32_t* stage = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(bars) + S::kBarBytes) +
+                      (warp - 2) * kStageWords;  // this warp's transpose buffer
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     int acc = 0;
@@ -338,7 +394,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_f16_tcgen05(const __grid
         tmem_ld32(tmem_base + lane_off + buf * BN + ch * 32, r);
         tmem_ld_wait();
         const int n = nb * BN + ch * 32;
-        if (valid) gemm_epilogue_chunk(p, m, grow, n, r);
+        if (valid) gemm_epilogue_chunk(p, m, grow, n, r, stage);
       }
       tc_fence_before();
       __syncwarp();

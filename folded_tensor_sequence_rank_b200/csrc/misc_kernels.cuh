@@ -132,31 +132,58 @@ __device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(
 template <>
 __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
 
-// out[c][r] = bf16(f(in[r][c])) for r < rows, c < cols, f = identity or GELU
-// (tanh form): the K-major [cols, rows] operand of a weight-gradient matmul
-// that reduces over the rows (tokens).  32 x 32 tiles staged through shared
-// memory so that both the reads and the writes are coalesced.
-template <typename Tin, bool GELU>
-__global__ void transpose_bf16_kernel(const Tin* __restrict__ in, int64_t rows, int cols, int64_t ldi,
-                                      __nv_bfloat16* __restrict__ out, int64_t ldo) {
-  __shared__ float tile[32][33];
-  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * 32;
-  const int c0 = blockIdx.y * 32;
-  const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
-  for (int k = ty; k < 32; k += 8) {
-    const int64_t r = r0 + k;
-    const int c = c0 + tx;
-    if (r < rows && c < cols) {
-      float v = to_f32<Tin>(in[r * ldi + c]);
-      if (GELU) v = gelu_tanh_f(v);
-      tile[k][tx] = v;
+template <typename T>
+__device__ __forceinline__ void unpack8(uint4 v, float (&f)[8]);
+template <>
+__device__ __forceinline__ void unpack8<__half>(uint4 v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&w[j]));
+    f[2 * j] = t.x;
+    f[2 * j + 1] = t.y;
+  }
+}
+template <>
+__device__ __forceinline__ void unpack8<__nv_bfloat16>(uint4 v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+    f[2 * j] = t.x;
+    f[2 * j + 1] = t.y;
+  }
+}
+
+// out[c][r] = bf16(in[r][c]) for r < rows, c < cols (both multiples of 8):
+// the K-major [cols, rows] operand of a weight-gradient matmul that reduces
+// over the rows (tokens).  64 x 64 tiles staged through shared memory, read
+// and written as 16-byte vectors of 8 elements.
+template <typename Tin>
+__global__ void __launch_bounds__(256) transpose_bf16_kernel(const Tin* __restrict__ in, int64_t rows, int cols,
+                                                             __nv_bfloat16* __restrict__ out) {
+  __shared__ float tile[64][65];
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * 64;
+  const int c0 = blockIdx.y * 64;
+  for (int q = threadIdx.x; q < 512; q += 256) {
+    const int rr = q >> 3, cc = (q & 7) * 8;
+    if (r0 + rr < rows && c0 + cc < cols) {
+      float f[8];
+      unpack8<Tin>(*reinterpret_cast<const uint4*>(in + (r0 + rr) * cols + c0 + cc), f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) tile[rr][cc + j] = f[j];
     }
   }
   __syncthreads();
-  for (int k = ty; k < 32; k += 8) {
-    const int c = c0 + k;
-    const int64_t r = r0 + tx;
-    if (r < rows && c < cols) out[static_cast<int64_t>(c) * ldo + r] = __float2bfloat16_rn(tile[tx][k]);
+  for (int q = threadIdx.x; q < 512; q += 256) {
+    const int cc = q >> 3, rr = (q & 7) * 8;
+    if (c0 + cc < cols && r0 + rr < rows) {
+      uint32_t w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) w[j] = pack_bf16x2(tile[rr + 2 * j][cc], tile[rr + 2 * j + 1][cc]);
+      *reinterpret_cast<uint4*>(out + static_cast<int64_t>(c0 + cc) * rows + r0 + rr) =
+          make_uint4(w[0], w[1], w[2], w[3]);
+    }
   }
 }
 

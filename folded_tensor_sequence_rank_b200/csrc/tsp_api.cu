@@ -266,7 +266,8 @@ void gemm_common(GemmParams& p, const Sizes& s, int rank, int* status) {
 // N-split projection of xn [L, h] by nseg weight families (each D shards
 // [h/D, h]) into nseg outputs [*, h]; remap[i] sends rows to global rows.
 int launch_proj(const Sizes& s, int rank, const __half* xn, const void* const* fam[3], void* out[3],
-                const int remap[3], int nseg, int epi, int F_cols, int* status, cudaStream_t st) {
+                const int remap[3], int nseg, int epi, int F_cols, int* status, cudaStream_t st,
+                void* out_t = nullptr) {
   static thread_local GemmParams p;
   std::memset(&p, 0, sizeof(p));
   const int shard_n = F_cols / s.D;
@@ -291,6 +292,9 @@ int launch_proj(const Sizes& s, int rank, const __half* xn, const void* const* f
     p.remap[i] = remap[i];
   }
   p.ldo = F_cols;
+  if (out_t && s.L % kGemmBM) return TSP_ERR_UNSUPPORTED;  // the transposed store needs whole warps
+  p.out_t = out_t;  // transposed GELU copy [N, L] (single segment, no remap)
+  p.ld_t = s.L;
   gemm_common(p, s, rank, status);
   return launch_gemm(p, bn, st);
 }
@@ -462,7 +466,8 @@ BwdLayout bwd_layout(const Sizes& s) {
 // strides lda / ldb, both fp16 or both bf16; epilogue kEpiStoreF32 (out fp32)
 // or kEpiGeluBwd (out bf16, aux = U fp16), row stride ldo.
 int launch_plain(const void* a, int M, int K, int64_t lda, const void* b, int N, int64_t ldb, bool bf16, int epi,
-                 void* out, int64_t ldo, const void* aux, int* status, cudaStream_t st) {
+                 void* out, int64_t ldo, const void* aux, int* status, cudaStream_t st, void* out_t = nullptr,
+                 int64_t ld_t = 0) {
   static thread_local GemmParams p;
   std::memset(&p, 0, sizeof(p));
   const int bn = pick_bn(N);
@@ -482,16 +487,20 @@ int launch_plain(const void* a, int M, int K, int64_t lda, const void* b, int N,
   p.out[0] = out;
   p.ldo = ldo;
   p.resid = aux;
+  if (out_t && M % kGemmBM) return TSP_ERR_UNSUPPORTED;  // the transposed store needs whole warps
+  p.out_t = out_t;
+  p.ld_t = ld_t;
   p.status = status;
   p.timeout_ns = kDefaultTimeoutNs;
   return launch_gemm(p, bn, st);
 }
 
-template <typename Tin, bool GELU>
+template <typename Tin>
 int launch_transpose(const Tin* in, int64_t rows, int cols, __nv_bfloat16* out, cudaStream_t st) {
   if (rows == 0) return TSP_OK;
-  const dim3 grid(static_cast<unsigned>((rows + 31) / 32), static_cast<unsigned>((cols + 31) / 32));
-  transpose_bf16_kernel<Tin, GELU><<<grid, dim3(32, 8), 0, st>>>(in, rows, cols, cols, out, rows);
+  if (rows % 8 || cols % 8) return TSP_ERR_UNSUPPORTED;
+  const dim3 grid(static_cast<unsigned>((rows + 63) / 64), static_cast<unsigned>((cols + 63) / 64));
+  transpose_bf16_kernel<Tin><<<grid, 256, 0, st>>>(in, rows, cols, out);
   TSP_CUDA(cudaGetLastError());
   return TSP_OK;
 }
@@ -806,17 +815,19 @@ int tsp_mlp_backward(const tsp_dims* dims, const tsp_weights* w, const void* w1_
   __nv_bfloat16* ht = reinterpret_cast<__nv_bfloat16*>(base + b.ht);
   __nv_bfloat16* dyt = reinterpret_cast<__nv_bfloat16*>(base + b.dyt);
   const int L = static_cast<int>(s.L);
-  // Xn2 = LN2(Y1), U = Xn2 W1 (fp16 shards, as in the forward)
+  // Xn2 = LN2(Y1), U = Xn2 W1 (fp16 shards, as in the forward); the same
+  // epilogue writes GELU(U)^T (bf16 [F, L]) for dW2
   rc = launch_layernorm<float>(static_cast<const float*>(y1), xn2, s.L, s.h, dims->ln_eps, stream);
   if (rc) return rc;
   const void* const* w1fam[3] = {reinterpret_cast<const void* const*>(w->w1), nullptr, nullptr};
   void* uout[3] = {u, nullptr, nullptr};
   const int noremap[3] = {0, 0, 0};
-  rc = launch_proj(s, 0, xn2, w1fam, uout, noremap, 1, kEpiStoreBf16, s.F, status, stream);
+  rc = launch_proj(s, 0, xn2, w1fam, uout, noremap, 1, kEpiStoreBf16, s.F, status, stream, ht);
   if (rc) return rc;
   if ((rc = record(ev, 1, stream))) return rc;
-  // dU = (dY W2^T) * GELU'(U): B = W2 [F, h] is K-major over h
-  rc = launch_plain(dy, L, s.h, s.h, w2_full, s.F, s.h, true, kEpiGeluBwd, du, s.F, u, status, stream);
+  // dU = (dY W2^T) * GELU'(U): B = W2 [F, h] is K-major over h; the
+  // epilogue also writes dU^T (bf16 [F, L]) for dW1
+  rc = launch_plain(dy, L, s.h, s.h, w2_full, s.F, s.h, true, kEpiGeluBwd, du, s.F, u, status, stream, dut, s.L);
   if (rc) return rc;
   if ((rc = record(ev, 2, stream))) return rc;
   // dXn2 = dU W1^T: B = W1 [h, F] is K-major over F
@@ -829,10 +840,8 @@ int tsp_mlp_backward(const tsp_dims* dims, const tsp_weights* w, const void* w1_
   if (rc) return rc;
   if ((rc = record(ev, 4, stream))) return rc;
   // token-major operands of the weight gradients (reduction over the tokens)
-  if ((rc = launch_transpose<__half, false>(xn2, s.L, s.h, xn2t, stream))) return rc;
-  if ((rc = launch_transpose<__nv_bfloat16, false>(du, s.L, s.F, dut, stream))) return rc;
-  if ((rc = launch_transpose<__half, true>(u, s.L, s.F, ht, stream))) return rc;
-  if ((rc = launch_transpose<__nv_bfloat16, false>(static_cast<const __nv_bfloat16*>(dy), s.L, s.h, dyt, stream)))
+  if ((rc = launch_transpose<__half>(xn2, s.L, s.h, xn2t, stream))) return rc;
+  if ((rc = launch_transpose<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(dy), s.L, s.h, dyt, stream)))
     return rc;
   if ((rc = record(ev, 5, stream))) return rc;
   // dW1 [h, F] = Xn2^T dU ; dW2 [F, h] = GELU(U)^T dY
