@@ -485,13 +485,15 @@ BWD_NAMES = ["ln2_u", "du", "dxn2", "ln2_bwd", "transposes", "dw1", "dw2"]
 
 
 def run_sweep_mlp_bwd(args):
-    """Backward of the MLP half for rank 0 of the 7B layer at T = 131072,
-    D = 8 (16384 tokens, seed 5): dY1, dW1, dW2 from Y1 and dY.  tokens/s =
+    """Backward of the MLP half for rank 0 of the 7B layer (T and D from
+    --workload; 128K, D = 8 by default: 16384 tokens, seed 5): dY1, dW1, dW2
+    from Y1 and dY.  tokens/s =
     L / backward time; the five matmuls (U recomputed, dU, dXn2, dW1, dW2)
     are 2 L h F FLOPs each."""
     import torch
     from folded_tensor_sequence_rank_b200 import tsp
-    T, h, H, F, D = 131072, 4096, 32, 16384, 8
+    wl = WORKLOADS[args.workload]
+    T, h, H, F, D = wl["T"], wl["h"], wl["H"], wl["F"], wl["D"]
     L = T // D
     torch.cuda.set_device(0)
     dims = tsp.make_dims(T, h, H, F)
@@ -521,11 +523,11 @@ def run_sweep_mlp_bwd(args):
     part = {n: statistics.median(e[j].elapsed_time(e[j + 1]) for e in evs) for j, n in enumerate(BWD_NAMES)}
     gf = 2.0 * L * h * F
     rate = {n: gf / (part[n] * 1e-3) / 1e12 for n in ("du", "dxn2", "dw1", "dw2")}
-    line = {"metric": "TSP MLP-half backward tokens/s on 1 B200 (7B layer, 128K, D=8, rank 0)",
+    line = {"metric": f"TSP MLP-half backward tokens/s on 1 B200 (7B layer, T={T}, D={D}, rank 0)",
             "value": L / (ms * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "MLP half of the 7B layer, backward (dY1, dW1, dW2), T=131072, D=8, rank 0: "
-                                   "16384 tokens, Y1 ~ N(0,1) fp32, dY ~ N(0,1) bf16 (seed 5)",
+            "config": {"workload": f"MLP half of the 7B layer, backward (dY1, dW1, dW2), T={T}, D={D}, rank 0: "
+                                   f"{L} tokens, Y1 ~ N(0,1) fp32, dY ~ N(0,1) bf16 (seed 5)",
                        "l2": "inputs larger than L2; no flush"},
             "tflop_per_step": 5 * gf / 1e12, "tflops": 5 * gf / (ms * 1e-3) / 1e12,
             "part_ms": {k: round(v, 4) for k, v in part.items()},

@@ -179,13 +179,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_pair_f16_tcgen05(const _
       const int m = mb * kPairBM + 128 * static_cast<int>(cta) + row;
       const bool valid = m < p.M;
       const int64_t grow = (m < p.c) ? (p.off0 + m) : (p.off1 + m);
+      // Software-pipelined over the 32-column chunks: the next chunk's
+      // accumulators (and, for kEpiGeluBwd, its U values) are loaded while
+      // this chunk is processed.
+      constexpr int kChunks = kPairBN / 32;
+      const bool aux_on = valid && p.epi == kEpiGeluBwd;
+      uint32_t r[32], rn[32];
+      uint4 aux[4] = {}, auxn[4] = {};
+      __syncwarp();
+      tmem_ld32(tmem_base + lane_off + buf * kPairBN, r);
+      if (aux_on) load_epilogue_aux(p, m, nb * kPairBN, aux);
+      tmem_ld_wait();
+      reg_fence32(r);
 #pragma unroll 1
-      for (int ch = 0; ch < kPairBN / 32; ++ch) {
-        uint32_t r[32];
-        __syncwarp();
-        tmem_ld32(tmem_base + lane_off + buf * kPairBN + ch * 32, r);
-        tmem_ld_wait();
-        if (valid) gemm_epilogue_chunk(p, m, grow, nb * kPairBN + ch * 32, r, stage);
+      for (int ch = 0; ch < kChunks; ++ch) {
+        if (ch + 1 < kChunks) {
+          __syncwarp();
+          tmem_ld32(tmem_base + lane_off + buf * kPairBN + (ch + 1) * 32, rn);
+          if (aux_on) load_epilogue_aux(p, m, nb * kPairBN + (ch + 1) * 32, auxn);
+        }
+        if (valid) gemm_epilogue_chunk(p, m, grow, nb * kPairBN + ch * 32, r, aux, stage);
+        if (ch + 1 < kChunks) {
+          tmem_ld_wait();
+          reg_fence32(rn);  // no use of rn before the wait
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = rn[i];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) aux[i] = auxn[i];
+        }
       }
       tc_fence_before();
       __syncwarp();

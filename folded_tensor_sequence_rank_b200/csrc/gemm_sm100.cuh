@@ -152,10 +152,19 @@ __device__ __forceinline__ void store_transposed_bf16(const GemmParams& p, uint3
   for (int i = 0; i < 4; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
 }
 
+// kEpiGeluBwd's U values for row m, columns n .. n+31 (the epilogue loop
+// loads them one chunk ahead).
+__device__ __forceinline__ void load_epilogue_aux(const GemmParams& p, int m, int n, uint4 (&a)[4]) {
+  const uint4* us = reinterpret_cast<const uint4*>(static_cast<const __half*>(p.resid) + static_cast<int64_t>(m) * p.ldo + n);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) a[i] = us[i];
+}
+
 // One 32-column chunk of an output tile's epilogue: accumulator values r for
 // local row m (global zigzag row grow) and output columns n .. n+31.
 __device__ __forceinline__ void gemm_epilogue_chunk(const GemmParams& p, int m, int64_t grow, int n,
-                                                    const uint32_t (&r)[32], uint32_t* stage) {
+                                                    const uint32_t (&r)[32], const uint4 (&aux)[4],
+                                                    uint32_t* stage) {
   if (p.epi == kEpiStoreF32) {
     float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out[0]) + static_cast<int64_t>(m) * p.ldo + n);
 #pragma unroll
@@ -166,12 +175,11 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const GemmParams& p, int m, 
   }
   if (p.epi == kEpiGeluBwd) {
     const int64_t off = static_cast<int64_t>(m) * p.ldo + n;
-    const uint4* us = reinterpret_cast<const uint4*>(static_cast<const __half*>(p.resid) + off);
     uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out[0]) + off);
     uint32_t tw[16];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint4 q = us[i];
+      const uint4 q = aux[i];
       const uint32_t w[4] = {q.x, q.y, q.z, q.w};
       uint32_t o[4];
 #pragma unroll
@@ -393,8 +401,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_f16_tcgen05(const __grid
         __syncwarp();
         tmem_ld32(tmem_base + lane_off + buf * BN + ch * 32, r);
         tmem_ld_wait();
+        reg_fence32(r);
         const int n = nb * BN + ch * 32;
-        if (valid) gemm_epilogue_chunk(p, m, grow, n, r, stage);
+        uint4 aux[4] = {};
+        if (valid && p.epi == kEpiGeluBwd) load_epilogue_aux(p, m, n, aux);
+        if (valid) gemm_epilogue_chunk(p, m, grow, n, r, aux, stage);
       }
       tc_fence_before();
       __syncwarp();
