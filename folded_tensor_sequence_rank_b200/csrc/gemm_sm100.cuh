@@ -15,9 +15,9 @@
 //   warp 0     TMA producer: A and B tiles into a STAGES-deep shared ring
 //   warp 1     TMEM allocator + single-thread tcgen05.mma issuer
 //   warps 2-5  epilogue: tcgen05.ld the 128 x BN fp32 accumulator (thread =
-//              row), apply store / GELU / residual, write to global memory
-//              (fp16 operands for the next matmul, or the fp32 / bf16
-//              residual stream).
+//              row), apply store / GELU / residual / GELU', write to global
+//              memory (fp16 operands for the next matmul, the fp32 / bf16
+//              residual stream, bf16 gradients, fp32 weight gradients).
 // Two TMEM accumulators let the epilogue of tile i overlap the K loop of
 // tile i+1.
 #pragma once

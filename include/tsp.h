@@ -1,6 +1,6 @@
 /*
  * tsp.h - C ABI of the TSP (Tensor + Sequence Parallelism) per-rank layer
- * forward for NVIDIA B200 (sm_100a).
+ * forward, and the backward of its MLP half, for NVIDIA B200 (sm_100a).
  *
  * The method (zubnet.ai news item "Zyphra TSP folds TP+SP onto one GPU
  * axis", paragraphs 1-2): tensor parallelism (weights split) and sequence
