@@ -50,7 +50,8 @@ Zigzag partition: the sequence is cut into 2D equal chunks of c = T/(2D)
 tokens, and rank r holds chunks r and 2D-1-r, in that order.
 
 Parity status: every function here is pinned by tests/test_oracle_pins.py
-and, for the MLP-half backward, tests/test_oracle_backward_pins.py (closed
+and, for the backward, tests/test_oracle_backward_pins.py (MLP half) and
+tests/test_oracle_attention_backward_pins.py (causal attention) (closed
 forms, invariants, brute force, finite differences and independent library
 routines).
 """
@@ -396,3 +397,43 @@ def mlp_backward_sampled(y1, dy, w: dict, rows, w1_cols, w2_rows, eps: float = L
     h_f = grnd(gelu_tanh(rnd(xn2 @ w1r[:, f])))
     out["dw2"] = h_f.T @ dy
     return out
+
+
+# ----------------------------------------------------------------------------
+# backward of causal attention  [TSP ¶1 (training), ¶2 (each rank's queries
+# against the all-gathered K/V)]
+# ----------------------------------------------------------------------------
+def causal_attention_backward(q, k, v, q_pos, dout, n_heads: int, scale: float):
+    """Gradients of sum(dout * causal_attention(q, k, v, q_pos)) with respect
+    to q [n, H*d] and to the full-sequence k, v [T, H*d], per head:
+        S = scale q k^T (keys past q_pos masked), P = softmax(S), O = P v,
+        dV = P^T dO,  dP = dO v^T,  dS = P * (dP - rowsum(dP * P)),
+        dQ = scale dS k,  dK = scale dS^T q.
+    Keys no query row reaches get zero gradient.  A rank's dK, dV are its
+    queries' contributions; summed over the ranks they give the gradients of
+    the whole sequence (what a reduce-scatter back to the key owners adds)."""
+    q = np.asarray(q, dtype=np.float64)
+    dout = np.asarray(dout, dtype=np.float64)
+    q_pos = np.asarray(q_pos, dtype=np.int64)
+    n, hd = q.shape
+    T = np.asarray(k).shape[0]
+    d = hd // n_heads
+    dq = np.zeros((n, hd))
+    dk = np.zeros((T, hd))
+    dv = np.zeros((T, hd))
+    if n == 0:
+        return dq, dk, dv
+    _, probs = causal_attention(q, k, v, q_pos, n_heads, scale, return_probs=True)
+    kmax = probs[0].shape[1]
+    for j in range(n_heads):
+        cols = slice(j * d, (j + 1) * d)
+        kj = np.asarray(k[:kmax, cols], dtype=np.float64)
+        vj = np.asarray(v[:kmax, cols], dtype=np.float64)
+        p = probs[j]
+        do = dout[:, cols]
+        dv[:kmax, cols] = p.T @ do
+        dp = do @ vj.T
+        ds = p * (dp - (dp * p).sum(axis=1, keepdims=True))
+        dq[:, cols] = scale * (ds @ kj)
+        dk[:kmax, cols] = scale * (ds.T @ q[:, cols])
+    return dq, dk, dv

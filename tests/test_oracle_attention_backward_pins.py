@@ -1,0 +1,123 @@
+"""Pins for the oracle's causal-attention backward (the attention half of the
+layer's backward is not built in CUDA yet; its oracle comes first).
+
+Sources of truth: central finite differences, torch autograd in fp64 through
+F.scaled_dot_product_attention with an explicit position mask, the softmax's
+invariances, and the sum over zigzag ranks against the whole sequence."""
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as Fn
+
+from oracle import tsp_oracle as O
+
+
+def _inputs(seed, n, T, H, d, pos=None):
+    rng = np.random.default_rng(seed)
+    q = rng.normal(size=(n, H * d))
+    k = rng.normal(size=(T, H * d))
+    v = rng.normal(size=(T, H * d))
+    dout = rng.normal(size=(n, H * d))
+    if pos is None:
+        pos = np.sort(rng.choice(T, size=n, replace=False))
+    return q, k, v, np.asarray(pos), dout
+
+
+def _loss(q, k, v, pos, dout, H, scale):
+    return float((dout * O.causal_attention(q, k, v, pos, H, scale)).sum())
+
+
+def _central(f, x, step=1e-6):
+    g = np.zeros_like(x)
+    it = np.nditer(x, flags=["multi_index"])
+    for _ in it:
+        i = it.multi_index
+        a = x.copy(); a[i] += step
+        b = x.copy(); b[i] -= step
+        g[i] = (f(a) - f(b)) / (2 * step)
+    return g
+
+
+def test_attention_backward_matches_finite_differences():
+    H, d, T = 2, 3, 7
+    q, k, v, pos, dout = _inputs(0, 4, T, H, d, pos=[0, 2, 5, 6])
+    s = 0.6
+    dq, dk, dv = O.causal_attention_backward(q, k, v, pos, dout, H, s)
+    np.testing.assert_allclose(dq, _central(lambda a: _loss(a, k, v, pos, dout, H, s), q), atol=1e-7)
+    np.testing.assert_allclose(dk, _central(lambda a: _loss(q, a, v, pos, dout, H, s), k), atol=1e-7)
+    np.testing.assert_allclose(dv, _central(lambda a: _loss(q, k, a, pos, dout, H, s), v), atol=1e-7)
+
+
+def test_attention_backward_matches_torch_autograd():
+    H, d, T = 3, 8, 40
+    q, k, v, pos, dout = _inputs(1, 12, T, H, d)
+    s = 1.0 / np.sqrt(d)
+    dq, dk, dv = O.causal_attention_backward(q, k, v, pos, dout, H, s)
+    qt, kt, vt = (torch.tensor(a, requires_grad=True) for a in (q, k, v))
+    mask = torch.tensor(np.arange(T)[None, :] <= pos[:, None])
+    split = lambda t: t.view(t.shape[0], H, d).transpose(0, 1)
+    o = Fn.scaled_dot_product_attention(split(qt), split(kt), split(vt), attn_mask=mask, scale=s)
+    (o.transpose(0, 1).reshape(len(pos), H * d) * torch.tensor(dout)).sum().backward()
+    np.testing.assert_allclose(dq, qt.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dk, kt.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dv, vt.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_attention_backward_invariants():
+    """Rows of P sum to 1, so the key-summed dV equals the query-summed dO;
+    softmax ignores a common shift of the scores, so the key-summed dK of each
+    head is zero; keys past the last query position get no gradient."""
+    H, d, T = 2, 4, 30
+    q, k, v, pos, dout = _inputs(2, 9, T, H, d)
+    dq, dk, dv = O.causal_attention_backward(q, k, v, pos, dout, H, 0.5)
+    np.testing.assert_allclose(dv.sum(axis=0), dout.sum(axis=0), atol=1e-12)
+    np.testing.assert_allclose(dk.sum(axis=0), 0.0, atol=1e-12)
+    assert not dk[pos.max() + 1:].any() and not dv[pos.max() + 1:].any()
+    # position 0 attends only to key 0: its query gets no gradient
+    q0, k0, v0, p0, do0 = _inputs(3, 3, 10, 1, 4, pos=[0, 4, 9])
+    g0 = O.causal_attention_backward(q0, k0, v0, p0, do0, 1, 0.5)[0]
+    assert not g0[0].any()
+
+
+@pytest.mark.parametrize("T,D", [(16, 2), (24, 3)])
+def test_zigzag_ranks_sum_to_the_whole_sequence(T, D):
+    """Each rank back-propagates its own zigzag rows against the full K/V; the
+    sum of the ranks' dK, dV is the whole sequence's, and the ranks' dQ rows
+    are the whole sequence's rows at their positions."""
+    H, d = 2, 4
+    q, k, v, _, dout = _inputs(4, T, T, H, d, pos=np.arange(T))
+    s = 0.4
+    full = O.causal_attention_backward(q, k, v, np.arange(T), dout, H, s)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for r in range(D):
+        idx = O.zigzag_index(T, D, r)
+        dq_r, dk_r, dv_r = O.causal_attention_backward(q[idx], k, v, idx, dout[idx], H, s)
+        np.testing.assert_allclose(dq_r, full[0][idx], atol=1e-12)
+        dk += dk_r
+        dv += dv_r
+    np.testing.assert_allclose(dk, full[1], atol=1e-12)
+    np.testing.assert_allclose(dv, full[2], atol=1e-12)
+
+
+def test_planted_softmax_backward_mistake_is_caught(monkeypatch):
+    """A backward that drops the row-sum term of dS (dS = P * dP) must break
+    the autograd pin."""
+    def bad(q, k, v, q_pos, dout, n_heads, scale):
+        q = np.asarray(q, dtype=np.float64)
+        n, hd = q.shape
+        d = hd // n_heads
+        dq, dk, dv = np.zeros((n, hd)), np.zeros(k.shape), np.zeros(v.shape)
+        _, probs = O.causal_attention(q, k, v, q_pos, n_heads, scale, return_probs=True)
+        km = probs[0].shape[1]
+        for j in range(n_heads):
+            c = slice(j * d, (j + 1) * d)
+            p = probs[j]
+            ds = p * (dout[:, c] @ v[:km, c].T)
+            dv[:km, c] = p.T @ dout[:, c]
+            dq[:, c] = scale * (ds @ k[:km, c])
+            dk[:km, c] = scale * (ds.T @ q[:, c])
+        return dq, dk, dv
+    monkeypatch.setattr(O, "causal_attention_backward", bad)
+    with pytest.raises(AssertionError):
+        test_attention_backward_matches_torch_autograd()
