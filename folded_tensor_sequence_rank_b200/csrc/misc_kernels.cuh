@@ -210,6 +210,74 @@ __device__ __forceinline__ void block_sum2(float& a, float& b, float* red) {
   }
 }
 
+// LayerNorm forward for wide rows (h >= 1024), one row per 256-thread block:
+// the same arithmetic as layernorm_rows_kernel (fp32 statistics over the row
+// held in registers: mean, then the centred sum of squares; fp16 output,
+// round to nearest even), with 4 G values per thread.  Small blocks with few
+// registers keep many rows in flight per SM, which the one-warp-per-row
+// kernel cannot at h = 4096.
+template <typename Tin>
+__device__ __forceinline__ void load4(const Tin* src, float* v);
+template <>
+__device__ __forceinline__ void load4<float>(const float* src, float* v) {
+  const float4 a = *reinterpret_cast<const float4*>(src);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+}
+template <>
+__device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* src, float* v) {
+  const uint2 q = *reinterpret_cast<const uint2*>(src);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.y));
+  v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+}
+
+template <typename Tin, int G>
+__global__ void __launch_bounds__(256) layernorm_block_kernel(const Tin* __restrict__ x, __half* __restrict__ y, int h,
+                                                              float eps) {
+  __shared__ float red[16];
+  const int64_t row = blockIdx.x;
+  const Tin* xr = x + row * h;
+  float v[4 * G];
+  float sum = 0.f, dummy = 0.f;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const int col = (g * 256 + threadIdx.x) * 4;
+    if (col < h) {
+      load4<Tin>(xr + col, &v[4 * g]);
+      sum += (v[4 * g] + v[4 * g + 1]) + (v[4 * g + 2] + v[4 * g + 3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[4 * g + j] = 0.f;
+    }
+  }
+  block_sum2(sum, dummy, red);
+  const float mean = sum / h;
+  float sq = 0.f;
+  dummy = 0.f;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const int col = (g * 256 + threadIdx.x) * 4;
+    if (col < h) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float d = v[4 * g + j] - mean;
+        sq = fmaf(d, d, sq);
+      }
+    }
+  }
+  block_sum2(sq, dummy, red);
+  const float rstd = rsqrtf(sq / h + eps);
+  __half* yr = y + row * h;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const int col = (g * 256 + threadIdx.x) * 4;
+    if (col < h)
+      *reinterpret_cast<uint2*>(yr + col) =
+          make_uint2(pack_half2((v[4 * g] - mean) * rstd, (v[4 * g + 1] - mean) * rstd),
+                     pack_half2((v[4 * g + 2] - mean) * rstd, (v[4 * g + 3] - mean) * rstd));
+  }
+}
+
 // LayerNorm backward with the residual, one row per 256-thread block:
 //   dy1 = dy + rstd * (g - mean(g) - xhat * mean(g * xhat)),
 //   xhat = (y1 - mean(y1)) * rstd, rstd = 1 / sqrt(var(y1) + eps)

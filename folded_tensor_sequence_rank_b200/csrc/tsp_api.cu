@@ -162,6 +162,16 @@ int check_weights(const tsp_weights* w, int D) {
 template <typename Tin>
 int launch_layernorm(const Tin* x, __half* y, int64_t rows, int h, float eps, cudaStream_t st) {
   if (rows == 0) return TSP_OK;
+  if (h >= 1024 && h <= 8192) {  // one row per block
+    const dim3 grid(static_cast<unsigned>(rows));
+    const int g = (h + 1023) / 1024;
+    if (g <= 1) layernorm_block_kernel<Tin, 1><<<grid, 256, 0, st>>>(x, y, h, eps);
+    else if (g <= 2) layernorm_block_kernel<Tin, 2><<<grid, 256, 0, st>>>(x, y, h, eps);
+    else if (g <= 4) layernorm_block_kernel<Tin, 4><<<grid, 256, 0, st>>>(x, y, h, eps);
+    else layernorm_block_kernel<Tin, 8><<<grid, 256, 0, st>>>(x, y, h, eps);
+    TSP_CUDA(cudaGetLastError());
+    return TSP_OK;
+  }
   const int warps = 8;
   const dim3 grid(static_cast<unsigned>((rows + warps - 1) / warps));
   const int nch = h / 8;
