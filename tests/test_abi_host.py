@@ -187,3 +187,12 @@ def test_mlp_backward_argument_checks(L):
         getattr(w, name)[2] = 0x30000
     n2 = L.tsp_mlp_backward_workspace_bytes(ctypes.byref(d2), 3)
     assert L.tsp_mlp_backward(ctypes.byref(d2), ctypes.byref(w), *ok, 256, n2, None, None) == tsp.TSP_ERR_UNSUPPORTED
+
+
+def test_mlp_backward_binding_checks_shapes_before_the_call(L):
+    import torch
+    d = dims()
+    w = tsp.ShardedWeights(D=2, buf=torch.zeros(1, dtype=torch.uint8), struct=tsp.Weights())
+    cpu = torch.zeros(4, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):  # CPU tensors are refused before the library is called
+        tsp.mlp_backward(d, w, cpu, cpu, cpu, cpu, cpu, cpu, cpu, torch.zeros(16, dtype=torch.uint8))
