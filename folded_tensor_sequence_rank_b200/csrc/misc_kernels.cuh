@@ -1,8 +1,9 @@
-// misc_kernels.cuh - the bandwidth-bound pieces of the TSP rank forward:
-// zigzag index map, pre-LayerNorm with fp16 output, weight shard packing, and
-// the bounded-wait self test.
+// misc_kernels.cuh - the bandwidth-bound pieces of the TSP rank step and of
+// the MLP-half backward: zigzag index map, pre-LayerNorm with fp16 output
+// (one warp per row, or one block per row for wide rows), weight shard
+// packing, the bf16 transposes and the LayerNorm backward of the backward
+// pass, and the bounded-wait self test.
 #pragma once
-#include "gemm_sm100.cuh"
 #include "ptx.cuh"
 
 namespace tsp {
@@ -125,13 +126,6 @@ __global__ void pack_transpose_kernel(const __nv_bfloat16* __restrict__ w, int64
 }
 
 // ---------------------------------------------------------------- backward helpers
-template <typename T>
-__device__ __forceinline__ float to_f32(T v);
-template <>
-__device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
-template <>
-__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
-
 template <typename T>
 __device__ __forceinline__ void unpack8(uint4 v, float (&f)[8]);
 template <>
