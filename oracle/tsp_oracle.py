@@ -437,3 +437,55 @@ def causal_attention_backward(q, k, v, q_pos, dout, n_heads: int, scale: float):
         dq[:, cols] = scale * (ds @ kj)
         dk[:kmax, cols] = scale * (ds.T @ q[:, cols])
     return dq, dk, dv
+
+
+def rank_layer_backward(rank: int, D: int, x_full, w: dict, dy_local, n_heads: int,
+                        eps: float = LN_EPS, scale: float | None = None) -> dict:
+    """One TSP rank's share of the whole layer's backward, in plain fp64 (no
+    16-bit storage), for the loss gradient dy_local [L, h] of its own output
+    rows (rank-local order).  x_full [T, h] is the sequence in natural order.
+
+    The rank computes, from its own rows and the all-gathered K/V:
+      the MLP half (mlp_backward): dY1, and its dW1, dW2 contributions;
+      the attention half: dA = dY1 Wo^T, dWo = A^T dY1, then
+      causal_attention_backward gives dQ for its rows and dK, dV for all T
+      keys; dWq = Xn1^T dQ; dXn1 = dQ Wq^T.
+    What crosses ranks: "dk_full", "dv_full" (every rank's contributions,
+    summed by a reduce-scatter back to the key owners).  After that sum, each
+    owner adds LN1'^T (dK Wk^T + dV Wv^T) to its rows' dX and forms dWk, dWv
+    (kv_backward_rows).  Weight-gradient entries are this rank's
+    contributions over its tokens; summed over ranks they give the layer's."""
+    x_full = np.asarray(x_full, dtype=np.float64)
+    T, h = x_full.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(h // n_heads)
+    w = {n: np.asarray(a, dtype=np.float64) for n, a in w.items()}
+    pos = zigzag_index(T, D, rank)
+    x = x_full[pos]
+    xn_full = layer_norm(x_full, eps)
+    k_full, v_full = xn_full @ w["wk"], xn_full @ w["wv"]
+    xn1 = xn_full[pos]
+    q = xn1 @ w["wq"]
+    a = causal_attention(q, k_full, v_full, pos, n_heads, scale)
+    y1 = x + a @ w["wo"]
+    mlp = mlp_backward(y1, dy_local, w, eps, storage=None, grad_storage=None)
+    dy1 = mlp["dy1"]
+    da = dy1 @ w["wo"].T
+    dwo = a.T @ dy1
+    dq, dk_full, dv_full = causal_attention_backward(q, k_full, v_full, pos, da, n_heads, scale)
+    dwq = xn1.T @ dq
+    dx = dy1 + layer_norm_backward(x, dq @ w["wq"].T, eps)
+    return {"dx_partial": dx, "dwq": dwq, "dwo": dwo, "dw1": mlp["dw1"], "dw2": mlp["dw2"],
+            "dk_full": dk_full, "dv_full": dv_full}
+
+
+def kv_backward_rows(x_rows, dk_rows, dv_rows, w: dict, eps: float = LN_EPS) -> dict:
+    """For rows whose keys/values are K = LN1(x) Wk, V = LN1(x) Wv and whose
+    summed gradients are dK, dV: the rows' extra input gradient
+    LN1'^T (dK Wk^T + dV Wv^T) and their dWk = LN1(x)^T dK, dWv = LN1(x)^T dV."""
+    x_rows = np.asarray(x_rows, dtype=np.float64)
+    xn = layer_norm(x_rows, eps)
+    wk = np.asarray(w["wk"], dtype=np.float64)
+    wv = np.asarray(w["wv"], dtype=np.float64)
+    return {"dx": layer_norm_backward(x_rows, dk_rows @ wk.T + dv_rows @ wv.T, eps),
+            "dwk": xn.T @ dk_rows, "dwv": xn.T @ dv_rows}

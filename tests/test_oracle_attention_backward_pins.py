@@ -121,3 +121,47 @@ def test_planted_softmax_backward_mistake_is_caught(monkeypatch):
     monkeypatch.setattr(O, "causal_attention_backward", bad)
     with pytest.raises(AssertionError):
         test_attention_backward_matches_torch_autograd()
+
+
+@pytest.mark.parametrize("T,D", [(8, 2), (12, 3)])
+def test_rank_backwards_sum_to_the_whole_layer_gradient(T, D):
+    """The D ranks' shares, with dK, dV summed over ranks (the reduce-scatter)
+    and each owner's K/V backward added, equal torch autograd of the whole
+    unsharded layer (fp64) for every input row and all six weights."""
+    h, H, F = 8, 2, 16
+    rng = np.random.default_rng(11)
+    x = rng.normal(size=(T, h))
+    w = {n: rng.normal(size=s) * 0.3 for n, s in (("wq", (h, h)), ("wk", (h, h)), ("wv", (h, h)), ("wo", (h, h)),
+                                                    ("w1", (h, F)), ("w2", (F, h)))}
+    dy = rng.normal(size=(T, h))
+    s = 1.0 / np.sqrt(h // H)
+    dx = np.zeros((T, h))
+    grads = {n: np.zeros_like(w[n]) for n in w}
+    dk = np.zeros((T, h))
+    dv = np.zeros((T, h))
+    for r in range(D):
+        idx = O.zigzag_index(T, D, r)
+        g = O.rank_layer_backward(r, D, x, w, dy[idx], H, scale=s)
+        dx[idx] += g["dx_partial"]
+        for n in ("wq", "wo", "w1", "w2"):
+            grads[n] += g["d" + n]
+        dk += g["dk_full"]
+        dv += g["dv_full"]
+    for r in range(D):   # each owner's K/V backward for its own rows
+        idx = O.zigzag_index(T, D, r)
+        kv = O.kv_backward_rows(x[idx], dk[idx], dv[idx], w)
+        dx[idx] += kv["dx"]
+        grads["wk"] += kv["dwk"]
+        grads["wv"] += kv["dwv"]
+    xt = torch.tensor(x, requires_grad=True)
+    wt = {n: torch.tensor(a, requires_grad=True) for n, a in w.items()}
+    xn = Fn.layer_norm(xt, (h,), eps=O.LN_EPS)
+    split = lambda t: t.view(T, H, h // H).transpose(0, 1)
+    att = Fn.scaled_dot_product_attention(split(xn @ wt["wq"]), split(xn @ wt["wk"]), split(xn @ wt["wv"]),
+                                          is_causal=True, scale=s)
+    y1 = xt + att.transpose(0, 1).reshape(T, h) @ wt["wo"]
+    y = y1 + Fn.gelu(Fn.layer_norm(y1, (h,), eps=O.LN_EPS) @ wt["w1"], approximate="tanh") @ wt["w2"]
+    (y * torch.tensor(dy)).sum().backward()
+    np.testing.assert_allclose(dx, xt.grad.numpy(), rtol=1e-9, atol=1e-11)
+    for n in w:
+        np.testing.assert_allclose(grads[n], wt[n].grad.numpy(), rtol=1e-9, atol=1e-11, err_msg=n)
