@@ -147,3 +147,33 @@ def test_planted_backward_mistakes_are_caught(monkeypatch, mistake):
         monkeypatch.setattr(O, "mlp_backward", bad_mlp)
     with pytest.raises(AssertionError):
         test_mlp_backward_matches_torch_autograd()
+
+
+@pytest.mark.parametrize("mistake", ["gelu_grad_first_term_only", "ln_backward_without_mean", "dw2_from_u"])
+def test_gpu_parity_bound_rejects_plausible_mistakes(monkeypatch, mistake):
+    """The GPU parity bound for the backward (rel-L2 <= 1e-3, max-abs <=
+    1e-2 max|ref|) is far tighter than what a plausible bug changes: each
+    planted mistake below moves some output beyond it (CPU only)."""
+    rng = np.random.default_rng(9)
+    n, h, F = 64, 32, 128
+    y1 = rng.normal(size=(n, h))
+    dy = O.round_bf16(rng.normal(size=(n, h)))
+    w = {"w1": O.round_bf16(rng.normal(size=(h, F)) * 0.1), "w2": O.round_bf16(rng.normal(size=(F, h)) * 0.1)}
+    ref = O.mlp_backward(y1, dy, w)
+    if mistake == "gelu_grad_first_term_only":
+        monkeypatch.setattr(O, "gelu_tanh_grad",
+                            lambda x: 0.5 * (1.0 + np.tanh(np.sqrt(2 / np.pi) * (x + 0.044715 * x ** 3))))
+    elif mistake == "ln_backward_without_mean":
+        def bad(x, g, eps=EPS):
+            c = x - x.mean(axis=-1, keepdims=True)
+            rstd = 1.0 / np.sqrt((c * c).mean(axis=-1, keepdims=True) + eps)
+            return rstd * (g - (c * rstd) * (g * c * rstd).mean(axis=-1, keepdims=True))
+        monkeypatch.setattr(O, "layer_norm_backward", bad)
+    else:
+        monkeypatch.setattr(O, "gelu_tanh", lambda x: np.asarray(x, dtype=np.float64))
+    got = O.mlp_backward(y1, dy, w)
+
+    def within(a, b):
+        return (np.abs(a - b).max() <= 1e-2 * np.abs(b).max()
+                and np.linalg.norm(a - b) <= 1e-3 * np.linalg.norm(b))
+    assert not all(within(got[k], ref[k]) for k in ("dy1", "dw1", "dw2"))
