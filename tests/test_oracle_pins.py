@@ -390,3 +390,32 @@ def test_planted_shard_mistakes_are_caught(monkeypatch):
     w_bad = dict(w, wo=w["wo"].T.copy())
     y = O.rank_forward_sharded(1, D, x[idx], K, V, w_bad, cfg["H"])
     assert not np.allclose(y, full["y"][idx], atol=1e-6)
+
+
+def test_gpu_parity_gates_reject_planted_attention_mistakes(monkeypatch):
+    """The forward GPU tests gate the attention output A at rel-L2 <= 2e-3 and
+    the layer's own contribution Y - X at 2e-2 (tests/test_gpu_parity.py).  On
+    the tiny layer, where attention is close to uniform averaging, each
+    plausible attention bug still moves A well beyond its gate (CPU only)."""
+    raw = inputs.layer_inputs(512, 256, 1024, 0)
+    x = raw["x"].double().numpy()
+    w = {n: raw[n].double().numpy() for n in inputs.WEIGHT_NAMES}
+    ref = O.layer_forward(x, w, 4)
+    good = O.causal_attention
+
+    def off_by_one(q, k, v, q_pos, n_heads, scale, return_probs=False):
+        return good(q, k, v, np.maximum(np.asarray(q_pos) - 1, 0), n_heads, scale, return_probs)
+
+    def wrong_scale(q, k, v, q_pos, n_heads, scale, return_probs=False):
+        return good(q, k, v, q_pos, n_heads, scale * 2 ** 0.5, return_probs)
+
+    def no_mask(q, k, v, q_pos, n_heads, scale, return_probs=False):
+        return good(q, k, v, np.full_like(np.asarray(q_pos), np.asarray(k).shape[0] - 1), n_heads, scale,
+                    return_probs)
+
+    def rel(a, b):
+        return float(np.linalg.norm(a - b) / np.linalg.norm(b))
+    for bad in (off_by_one, wrong_scale, no_mask):
+        monkeypatch.setattr(O, "causal_attention", bad)
+        out = O.layer_forward(x, w, 4)
+        assert rel(out["a"], ref["a"]) > 10 * 2e-3 or rel(out["y"] - x, ref["y"] - x) > 2e-2, bad.__name__
