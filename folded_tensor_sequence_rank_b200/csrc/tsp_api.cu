@@ -803,7 +803,9 @@ int tsp_mlp_backward(const tsp_dims* dims, const tsp_weights* w, const void* w1_
   for (int i = 0; i < (s.L == 0 ? 4 : 7); ++i)
     if (!ptrs[i] || !aligned16(ptrs[i])) return TSP_ERR_INVALID_ARG;
   if (!bws || (reinterpret_cast<uintptr_t>(bws) & 255)) return TSP_ERR_INVALID_ARG;
-  if (s.h % 256 || s.F % 256) return TSP_ERR_UNSUPPORTED;
+  // whole 256-column tiles, and whole 128-row tiles of tokens (the
+  // transposed epilogue stores need every lane of a warp)
+  if (s.h % 256 || s.F % 256 || s.L % 128) return TSP_ERR_UNSUPPORTED;
   const BwdLayout b = bwd_layout(s);
   if (bws_bytes < b.total) return TSP_ERR_WORKSPACE;
   uint8_t* base = static_cast<uint8_t*>(bws);

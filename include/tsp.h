@@ -251,7 +251,8 @@ size_t tsp_mlp_backward_workspace_bytes(const tsp_dims* dims, int D);
  * pointer 16-byte aligned.  With T = 0 only dw1 and dw2 are written (zeros)
  * and y1, dy, dy1 may be NULL.  bws: tsp_mlp_backward_workspace_bytes(dims, D)
  * bytes, also the status word that tsp_get_device_status reads.  h and F
- * must be multiples of 256.  step_events: NULL, or TSP_N_STEP_EVENTS
+ * must be multiples of 256 and T/D a multiple of 128 (TSP_ERR_UNSUPPORTED
+ * otherwise, before anything is enqueued).  step_events: NULL, or TSP_N_STEP_EVENTS
  * caller-created events recorded on `stream` before the first launch and
  * after LN2 + U, dU, dXn2, the LN2 backward, the transposes, dW1 and dW2. */
 int tsp_mlp_backward(const tsp_dims* dims, const tsp_weights* w,

@@ -180,6 +180,10 @@ def test_mlp_backward_argument_checks(L):
     # workspace: misaligned, then too small
     assert L.tsp_mlp_backward(ctypes.byref(d), ctypes.byref(w), *ok, 272, n, None, None) == tsp.TSP_ERR_INVALID_ARG
     assert L.tsp_mlp_backward(ctypes.byref(d), ctypes.byref(w), *ok, 256, n - 1, None, None) == tsp.TSP_ERR_WORKSPACE
+    # ragged token count: T/D = 400 is not a multiple of 128
+    d3 = dims(T=800)
+    n3 = L.tsp_mlp_backward_workspace_bytes(ctypes.byref(d3), 2)
+    assert L.tsp_mlp_backward(ctypes.byref(d3), ctypes.byref(w), *ok, 256, n3, None, None) == tsp.TSP_ERR_UNSUPPORTED
     # h not a multiple of 256
     d2 = dims(T=768, h=192, H=3, F=768)
     w.D = 3
