@@ -32,7 +32,9 @@ constexpr int kGemmMaxMaps = 48;  // 3 segments x 16 shards
 constexpr int kGemmGroupM = 16;   // M tiles per raster group (L2 reuse of A)
 
 // Epilogues.  kEpiStoreBf16 / kEpiGeluBf16 write fp16 operands for the next
-// matmul (the names keep the 16-bit operand role); kEpiResidual adds the
+// matmul (the names keep the 16-bit operand role), saturating at +-65504 and
+// setting kFlagFp16Saturated in the flags word after `status` when a value
+// was out of range; kEpiResidual adds the
 // residual stream; kEpiGeluBwd writes the bf16 gradient acc * GELU'(U) with U
 // (fp16, [M, ldo]) at `resid`; kEpiStoreF32 writes acc as fp32.
 // kEpiStoreBf16 and kEpiGeluBwd can also write the tile transposed, as bf16,
@@ -63,7 +65,7 @@ struct __align__(64) GemmParams {
   int out_f32;        // kEpiResidual: output fp32 (1) or bf16 (0)
   int c;              // zigzag: local rows [0,c) -> off0 + m, [c, 2c) -> off1 + m
   int64_t off0, off1;
-  int* status;
+  int* status;        // status word; status[1] is the flags word
   uint64_t timeout_ns;
 };
 
@@ -238,14 +240,23 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const GemmParams& p, int m, 
     const int col = n - seg * p.seg_n;
     const int64_t orow = p.remap[seg] ? grow : m;
     uint32_t packed[16];
+    float mx = 0.f;  // largest magnitude converted: flags a saturation
     if (p.epi == kEpiGeluBf16) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        packed[i] = pack_half2(gelu_tanh_f(__uint_as_float(r[2 * i])), gelu_tanh_f(__uint_as_float(r[2 * i + 1])));
+      for (int i = 0; i < 16; ++i) {
+        const float a = gelu_tanh_f(__uint_as_float(r[2 * i])), b = gelu_tanh_f(__uint_as_float(r[2 * i + 1]));
+        mx = fmax3(mx, fabsf(a), fabsf(b));
+        packed[i] = pack_half2(a, b);
+      }
     } else {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) packed[i] = pack_half2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+      for (int i = 0; i < 16; ++i) {
+        const float a = __uint_as_float(r[2 * i]), b = __uint_as_float(r[2 * i + 1]);
+        mx = fmax3(mx, fabsf(a), fabsf(b));
+        packed[i] = pack_half2(a, b);
+      }
     }
+    note_fp16_saturation(p.status, mx);
     uint4* dst = reinterpret_cast<uint4*>(static_cast<__half*>(p.out[seg]) + orow * p.ldo + col);
 #pragma unroll
     for (int i = 0; i < 4; ++i)

@@ -105,8 +105,9 @@ __global__ void __launch_bounds__(256) layernorm_rows_kernel(const Tin* __restri
 // converted to fp16 (round to nearest even, saturating) in the K-major
 // [n_out, n_in] layout the GEMM's B operand uses.  32x32 tiles staged through
 // shared memory so both sides are coalesced.
+// A weight outside fp16's range sets kFlagFp16Saturated in status[1].
 __global__ void pack_transpose_kernel(const __nv_bfloat16* __restrict__ w, int64_t ld, int64_t row0, int64_t col0,
-                                      __half* __restrict__ out, int n_out, int n_in) {
+                                      __half* __restrict__ out, int n_out, int n_in, int* status) {
   __shared__ float tile[32][33];
   const int i0 = blockIdx.x * 32, o0 = blockIdx.y * 32;
   const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
@@ -115,14 +116,18 @@ __global__ void pack_transpose_kernel(const __nv_bfloat16* __restrict__ w, int64
     if (i < n_in && o < n_out) tile[k][tx] = __bfloat162float(w[(row0 + i) * ld + col0 + o]);
   }
   __syncthreads();
+  float mx = 0.f;
   for (int k = ty; k < 32; k += 8) {
     const int o = o0 + k, i = i0 + tx;
     if (i < n_in && o < n_out) {
       uint16_t hbits;
-      asm("cvt.rn.satfinite.f16.f32 %0, %1;" : "=h"(hbits) : "f"(tile[tx][k]));
+      const float v = tile[tx][k];
+      mx = fmaxf(mx, fabsf(v));
+      asm("cvt.rn.satfinite.f16.f32 %0, %1;" : "=h"(hbits) : "f"(v));
       reinterpret_cast<uint16_t*>(out)[static_cast<int64_t>(o) * n_in + i] = hbits;
     }
   }
+  note_fp16_saturation(status, mx);
 }
 
 // ---------------------------------------------------------------- backward helpers

@@ -10,6 +10,15 @@ namespace tsp {
 
 // Status word values written by kernels (match tsp_status in tsp.h).
 constexpr int kStatusTimeout = 4;
+// Bits of the flags word that follows the status word (status[1]).
+constexpr int kFlagFp16Saturated = 1;
+
+// Records that a value outside fp16's finite range (|x| > 65504) was clamped
+// to +-65504 by a saturating conversion.  `status` is the status word; the
+// flags word is the next int.
+__device__ __forceinline__ void note_fp16_saturation(int* status, float maxabs) {
+  if (maxabs > 65504.0f) atomicOr(status + 1, kFlagFp16Saturated);
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -143,7 +143,9 @@ int check_dims(const tsp_dims* dims, int D) {
   if (!(dims->ln_eps >= 0.f) || !(dims->softmax_scale > 0.f)) return TSP_ERR_INVALID_ARG;
   if (dims->T >= (int64_t(1) << 31)) return TSP_ERR_UNSUPPORTED;
   if (dims->head_dim != 64 && dims->head_dim != 128) return TSP_ERR_UNSUPPORTED;
-  if (dims->h % 64 != 0 || dims->h > 4096) return TSP_ERR_UNSUPPORTED;
+  // h <= 8192: the LayerNorm kernels (forward and backward) hold a row as at
+  // most 8 groups of 4 values per thread of a 256-thread block
+  if (dims->h % 64 != 0 || dims->h > 8192) return TSP_ERR_UNSUPPORTED;
   if ((dims->h / D) % 64 != 0 || (dims->ffn / D) % 64 != 0) return TSP_ERR_UNSUPPORTED;
   return TSP_OK;
 }
@@ -536,24 +538,75 @@ int launch_ln_backward(const float* y1, const float* g, const __nv_bfloat16* dy,
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
 constexpr size_t kNoAllocXnOffset = 1024;
 
+// Device address of the array in the CUDA context current on this thread.
+// The address belongs to a context: after cudaDeviceReset, or if the primary
+// context is released and created again, the module is loaded anew and the
+// array can move.  So the cache is per device AND keyed on the context's
+// unique ID (cuCtxGetId; IDs are never reused within a process), and the
+// address is looked up again whenever the current context is not the one it
+// was found in.  In host code the array's name is only a host-side stand-in:
+// the device address comes from cudaGetSymbolAddress, called with the device
+// current (the first call on a device, or in a new context, does this lookup).
+struct NoAllocEntry {
+  void* addr = nullptr;
+  unsigned long long ctx_id = 0;
+  bool keyed = false;
+};
 std::mutex g_noalloc_mu;
-void* g_noalloc_addr[256] = {};  // device address of the array, per device ordinal
+NoAllocEntry g_noalloc_cache[256];
 
-// In host code the array's name is only a host-side stand-in: the device
-// address comes from cudaGetSymbolAddress, looked up once per device with that
-// device current (the first call on a device does this lookup).
+// ID of the context current on this thread; false if none is current or the
+// driver entry points are unavailable (then every call looks the address up).
+bool current_ctx_id(unsigned long long* id) {
+  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (!get_cur || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_cur(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
 int noalloc_scratch(void** out) {
   int dev = 0;
   TSP_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 256) return TSP_ERR_UNSUPPORTED;
+  unsigned long long id = 0;
+  const bool have_id = current_ctx_id(&id);
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_addr[dev]) {
-    void* p = nullptr;
-    TSP_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch));
-    g_noalloc_addr[dev] = p;
+  NoAllocEntry& e = g_noalloc_cache[dev];
+  if (have_id && e.keyed && e.addr && e.ctx_id == id) {
+    *out = e.addr;
+    return TSP_OK;
   }
-  *out = g_noalloc_addr[dev];
+  void* p = nullptr;
+  TSP_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+  // the lookup makes the device's primary context current if none was
+  unsigned long long id2 = 0;
+  e.keyed = current_ctx_id(&id2);
+  e.ctx_id = id2;
+  e.addr = p;
+  *out = p;
   return TSP_OK;
+}
+
+// The status section's two words -> the status a caller sees: a timeout
+// first, then a saturation; anything else in the status word is unknown.
+int status_of_words(const int (&h)[2]) {
+  if (h[0] == TSP_ERR_TIMEOUT) return TSP_ERR_TIMEOUT;
+  if (h[0] != 0) return TSP_ERR_CUDA;
+  return (h[1] & kFlagFp16Saturated) ? TSP_ERR_SATURATED : TSP_OK;
 }
 
 }  // namespace
@@ -571,6 +624,7 @@ const char* tsp_status_string(int status) {
     case TSP_ERR_CUDA: return "CUDA error";
     case TSP_ERR_TIMEOUT: return "device wait timed out";
     case TSP_ERR_WORKSPACE: return "workspace too small";
+    case TSP_ERR_SATURATED: return "fp16 conversion saturated";
     default: return "unknown status";
   }
 }
@@ -595,8 +649,9 @@ int tsp_zigzag_index(int64_t T, int D, int rank, int32_t* d_idx, cudaStream_t st
 size_t tsp_shard_buffer_bytes(const tsp_dims* dims, int D) {
   if (check_dims(dims, D) != TSP_OK) return 0;
   const size_t h = dims->h, F = dims->ffn;
-  // per shard: 4 attention matrices of h*h/D, 2 FFN matrices of h*F/D
-  return static_cast<size_t>(D) * (4 * align_up(h * (h / D) * 2) + 2 * align_up(h * (F / D) * 2));
+  // a status section, then per shard: 4 attention matrices of h*h/D, 2 FFN
+  // matrices of h*F/D
+  return kAlign + static_cast<size_t>(D) * (4 * align_up(h * (h / D) * 2) + 2 * align_up(h * (F / D) * 2));
 }
 
 int tsp_pack_shards(const tsp_dims* dims, int D, const void* const w_full[6], void* d_buf, size_t buf_bytes,
@@ -608,15 +663,18 @@ int tsp_pack_shards(const tsp_dims* dims, int D, const void* const w_full[6], vo
     if (!w_full[i]) return TSP_ERR_INVALID_ARG;
   if (buf_bytes < tsp_shard_buffer_bytes(dims, D)) return TSP_ERR_WORKSPACE;
   const int h = dims->h, F = dims->ffn, hs = h / D, Fs = F / D;
+  if (!aligned16(d_buf)) return TSP_ERR_INVALID_ARG;
   std::memset(out, 0, sizeof(*out));
   out->D = D;
-  uint8_t* p = static_cast<uint8_t*>(d_buf);
+  int* status = static_cast<int*>(d_buf);  // status section: status word, flags word
+  TSP_CUDA(cudaMemsetAsync(status, 0, 2 * sizeof(int), stream));
+  uint8_t* p = static_cast<uint8_t*>(d_buf) + kAlign;
   const dim3 blk(32, 8);
   auto pack = [&](const void* src, int64_t ld, int64_t row0, int64_t col0, int n_out, int n_in, const void** dst) -> int {
     *dst = p;
     const dim3 grid((n_in + 31) / 32, (n_out + 31) / 32);
     pack_transpose_kernel<<<grid, blk, 0, stream>>>(static_cast<const __nv_bfloat16*>(src), ld, row0, col0,
-                                                    reinterpret_cast<__half*>(p), n_out, n_in);
+                                                    reinterpret_cast<__half*>(p), n_out, n_in, status);
     TSP_CUDA(cudaGetLastError());
     p += align_up(static_cast<size_t>(n_out) * n_in * 2);
     return TSP_OK;
@@ -651,16 +709,16 @@ int tsp_workspace_offsets(const tsp_dims* dims, int D, size_t off[8]) {
 
 int tsp_reset_device_status(void* ws, cudaStream_t stream) {
   if (!ws) return TSP_ERR_INVALID_ARG;
-  TSP_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), stream));
+  TSP_CUDA(cudaMemsetAsync(ws, 0, 2 * sizeof(int), stream));
   return TSP_OK;
 }
 
 int tsp_get_device_status(const void* ws, cudaStream_t stream) {
   if (!ws) return TSP_ERR_INVALID_ARG;
-  int h = 0;
-  TSP_CUDA(cudaMemcpyAsync(&h, ws, sizeof(int), cudaMemcpyDeviceToHost, stream));
+  int h[2] = {0, 0};
+  TSP_CUDA(cudaMemcpyAsync(h, ws, sizeof(h), cudaMemcpyDeviceToHost, stream));
   TSP_CUDA(cudaStreamSynchronize(stream));
-  return h == 0 ? TSP_OK : (h == TSP_ERR_TIMEOUT ? TSP_ERR_TIMEOUT : TSP_ERR_CUDA);
+  return status_of_words(h);
 }
 
 int tsp_kv_project(const tsp_dims* dims, const tsp_weights* w, int rank, const void* x_local, void* k_full,
@@ -704,8 +762,9 @@ int tsp_kv_project_noalloc(const tsp_dims* dims, const tsp_weights* w, int rank,
   uint8_t* base = static_cast<uint8_t*>(scratch);
   int* status = reinterpret_cast<int*>(base);
   __half* xn = reinterpret_cast<__half*>(base + kNoAllocXnOffset);
-  // the array keeps the previous call's contents: the status word starts at zero
-  TSP_CUDA(cudaMemsetAsync(status, 0, sizeof(int), stream));
+  // the array keeps the previous call's contents: the status and flags words
+  // start at zero
+  TSP_CUDA(cudaMemsetAsync(status, 0, 2 * sizeof(int), stream));
   rc = launch_layernorm<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x_local), xn, sz.L, sz.h, dims->ln_eps, stream);
   if (rc) return rc;
   const void* const* fam[3] = {reinterpret_cast<const void* const*>(w->wk),
@@ -713,6 +772,16 @@ int tsp_kv_project_noalloc(const tsp_dims* dims, const tsp_weights* w, int rank,
   void* out[3] = {k_full, v_full, nullptr};
   const int remap[3] = {1, 1, 0};
   return launch_proj(sz, rank, xn, fam, out, remap, 2, kEpiStoreBf16, sz.h, status, stream);
+}
+
+int tsp_kv_project_noalloc_status(cudaStream_t stream) {
+  void* scratch = nullptr;
+  int rc = noalloc_scratch(&scratch);
+  if (rc) return rc;
+  int h[2] = {0, 0};
+  TSP_CUDA(cudaMemcpyAsync(h, scratch, sizeof(h), cudaMemcpyDeviceToHost, stream));
+  TSP_CUDA(cudaStreamSynchronize(stream));
+  return status_of_words(h);
 }
 
 int tsp_layer_forward(const tsp_dims* dims, const tsp_weights* w, int rank, const void* x_local, const void* k_full,
@@ -773,8 +842,12 @@ int tsp_rank_step_host(const tsp_dims* dims, const tsp_weights* w, int rank, con
   Ctx c;
   int rc = make_ctx(c, dims, w, rank, ws, ws_bytes);
   if (rc) return rc;
+  // every argument tsp_rank_step checks, before anything is enqueued
+  if (y_dtype != TSP_OUT_BF16 && y_dtype != TSP_OUT_F32) return TSP_ERR_INVALID_ARG;
   if (c.s.L == 0) return TSP_OK;
-  if (!h_x_local || !d_x_staging || !d_y_staging || !h_y_local) return TSP_ERR_INVALID_ARG;
+  if (!h_x_local || !d_x_staging || !d_y_staging || !h_y_local || !k_full || !v_full) return TSP_ERR_INVALID_ARG;
+  if (!aligned16(d_x_staging) || !aligned16(d_y_staging) || !aligned16(k_full) || !aligned16(v_full))
+    return TSP_ERR_INVALID_ARG;
   const size_t xb = static_cast<size_t>(c.s.L) * c.s.h * 2;
   const size_t yb = static_cast<size_t>(c.s.L) * c.s.h * (y_dtype == TSP_OUT_F32 ? 4 : 2);
   TSP_CUDA(cudaMemcpyAsync(d_x_staging, h_x_local, xb, cudaMemcpyHostToDevice, stream));
@@ -866,7 +939,11 @@ int tsp_mlp_backward(const tsp_dims* dims, const tsp_weights* w, const void* w1_
 }
 
 int tsp_selftest_wait_timeout(void* ws, uint64_t timeout_ns, cudaStream_t stream) {
-  if (!ws || timeout_ns == 0 || timeout_ns > 2000000000ull) return TSP_ERR_INVALID_ARG;
+  if (timeout_ns == 0 || timeout_ns > 2000000000ull) return TSP_ERR_INVALID_ARG;
+  if (!ws) {  // the status word of tsp_kv_project_noalloc's static scratch
+    int rc = noalloc_scratch(&ws);
+    if (rc) return rc;
+  }
   wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(static_cast<int*>(ws), timeout_ns);
   TSP_CUDA(cudaGetLastError());
   return TSP_OK;

@@ -18,8 +18,10 @@ MAX_D = 16
 N_STEP_EVENTS = 8
 OUT_BF16, OUT_F32 = 0, 1
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "CUDA error",
-          4: "device wait timed out", 5: "workspace too small"}
-TSP_OK, TSP_ERR_INVALID_ARG, TSP_ERR_UNSUPPORTED, TSP_ERR_CUDA, TSP_ERR_TIMEOUT, TSP_ERR_WORKSPACE = range(6)
+          4: "device wait timed out", 5: "workspace too small", 6: "fp16 conversion saturated"}
+(TSP_OK, TSP_ERR_INVALID_ARG, TSP_ERR_UNSUPPORTED, TSP_ERR_CUDA, TSP_ERR_TIMEOUT, TSP_ERR_WORKSPACE,
+ TSP_ERR_SATURATED) = range(7)
+DEVICE_STATUSES = (TSP_OK, TSP_ERR_TIMEOUT, TSP_ERR_SATURATED)
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtsp_b200.so")
 WEIGHT_NAMES = ("wq", "wk", "wv", "wo", "w1", "w2")
@@ -71,6 +73,7 @@ def lib() -> ctypes.CDLL:
         "tsp_get_device_status": (i32, [vp, vp]),
         "tsp_kv_project": (i32, [pd, pw, i32, vp, vp, vp, vp, sz, vp]),
         "tsp_kv_project_noalloc": (i32, [pd, pw, i32, vp, vp, vp, vp]),
+        "tsp_kv_project_noalloc_status": (i32, [vp]),
         "tsp_layer_forward": (i32, [pd, pw, i32, vp, vp, vp, vp, i32, vp, sz, vp, ctypes.POINTER(vp)]),
         "tsp_rank_step": (i32, [pd, pw, i32, vp, vp, vp, vp, i32, vp, sz, vp, ctypes.POINTER(vp)]),
         "tsp_rank_step_host": (i32, [pd, pw, i32, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]),
@@ -206,9 +209,19 @@ def reset_device_status(ws: torch.Tensor, stream=None):
 
 
 def get_device_status(ws: torch.Tensor, stream=None) -> int:
+    """Reads a status section (a workspace, an MLP backward workspace or a
+    packed shard buffer): TSP_OK, TSP_ERR_TIMEOUT or TSP_ERR_SATURATED."""
     rc = lib().tsp_get_device_status(_ptr(ws, "ws"), _stream(stream))
-    if rc not in (TSP_OK, TSP_ERR_TIMEOUT):
+    if rc not in DEVICE_STATUSES:
         _check(rc, "tsp_get_device_status")
+    return rc
+
+
+def kv_project_noalloc_status(stream=None) -> int:
+    """Status section of tsp_kv_project_noalloc's static scratch (its last call)."""
+    rc = lib().tsp_kv_project_noalloc_status(_stream(stream))
+    if rc not in DEVICE_STATUSES:
+        _check(rc, "tsp_kv_project_noalloc_status")
     return rc
 
 
@@ -309,6 +322,7 @@ def rank_step_host(dims: Dims, w: ShardedWeights, rank: int, h_x_local, x_stagin
            "tsp_rank_step_host")
 
 
-def selftest_wait_timeout(ws: torch.Tensor, timeout_ns: int, stream=None):
-    _check(lib().tsp_selftest_wait_timeout(_ptr(ws, "ws"), timeout_ns, _stream(stream)),
+def selftest_wait_timeout(ws: torch.Tensor | None, timeout_ns: int, stream=None):
+    """ws=None targets the status section of tsp_kv_project_noalloc's scratch."""
+    _check(lib().tsp_selftest_wait_timeout(None if ws is None else _ptr(ws, "ws"), timeout_ns, _stream(stream)),
            "tsp_selftest_wait_timeout")

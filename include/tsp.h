@@ -43,12 +43,22 @@
  *   - Every device buffer is allocated and freed by the caller.  Functions
  *     that take a stream only enqueue work on it (asynchronous) unless
  *     stated otherwise; the library allocates no device memory and keeps no
- *     state between calls.
+ *     state between calls.  One exception: tsp_kv_project_noalloc's scratch
+ *     is a 64 MiB file-scope device array of this library (held on every
+ *     device that loads it until exit), whose device address the library
+ *     caches per device and CUDA context; that array keeps the last call's
+ *     contents, and calls that overlap on the GPU race on it.
  *   - Host-detectable errors are returned synchronously and nothing is
  *     enqueued.  There is no fallback path: an unsupported shape is an
- *     error.  Device-side timeouts (a bounded wait inside a kernel that ran
- *     out) are recorded in the workspace status word and reported by
- *     tsp_get_device_status.
+ *     error.  Device-side events are recorded in a status section (a status
+ *     word, then a flags word) at the start of the workspace, of the MLP
+ *     backward's workspace and of the packed shard buffer, and reported by
+ *     tsp_get_device_status: a bounded wait inside a kernel that ran out
+ *     (TSP_ERR_TIMEOUT), or a conversion to fp16 that saturated
+ *     (TSP_ERR_SATURATED: a weight beyond +-65504 when packing, or a Q, K,
+ *     V, GELU output or recomputed pre-activation beyond it in a GEMM
+ *     epilogue).  LayerNorm outputs (|y| < sqrt(h)) and attention outputs (a
+ *     convex combination of fp16 V rows) cannot leave the range.
  */
 #ifndef TSP_H_
 #define TSP_H_
@@ -70,7 +80,10 @@ typedef enum {
   TSP_ERR_UNSUPPORTED = 2, /* a shape the kernels do not implement (see tsp_check_dims) */
   TSP_ERR_CUDA = 3,        /* a CUDA runtime call failed; see tsp_last_cuda_error */
   TSP_ERR_TIMEOUT = 4,     /* a bounded wait inside a kernel ran out */
-  TSP_ERR_WORKSPACE = 5    /* workspace or buffer smaller than required */
+  TSP_ERR_WORKSPACE = 5,   /* workspace or buffer smaller than required */
+  TSP_ERR_SATURATED = 6    /* a value outside fp16's range (|x| > 65504) was
+                              clamped to +-65504 on conversion: the results are
+                              finite but may be wrong (device status only) */
 } tsp_status;
 
 /* Layer and sequence sizes. */
@@ -110,8 +123,10 @@ const char* tsp_last_cuda_error(void);
 
 /* Checks sizes against what the kernels implement; returns TSP_OK,
  * TSP_ERR_INVALID_ARG or TSP_ERR_UNSUPPORTED.  Supported: head_dim 64 or
- * 128, h % 64 == 0, h/D % 64 == 0, F/D % 64 == 0, H % D == 0, F % D == 0,
- * 1 <= D <= TSP_MAX_D, T % (2D) == 0, T < 2^31.  Pure host function. */
+ * 128, h % 64 == 0, h <= 8192 (the LayerNorm kernels hold a row as at most
+ * 8 groups of 4 values per thread of a 256-thread block), h/D % 64 == 0,
+ * F/D % 64 == 0, H % D == 0, F % D == 0, 1 <= D <= TSP_MAX_D,
+ * T % (2D) == 0, T < 2^31.  Pure host function. */
 int tsp_check_dims(const tsp_dims* dims, int D);
 
 /* Zigzag index map [zubnet.ai TSP item, paragraph 2: "zigzag partition"]:
@@ -119,15 +134,19 @@ int tsp_check_dims(const tsp_dims* dims, int D);
  * i in [0, T/D).  d_idx: device int32 [T/D].  Bit-exact integer result. */
 int tsp_zigzag_index(int64_t T, int D, int rank, int32_t* d_idx, cudaStream_t stream);
 
-/* Bytes of one packed shard buffer for all six weights at this D. */
+/* Bytes of one packed shard buffer for all six weights at this D: a
+ * 1 KiB status section (read by tsp_get_device_status on the buffer's base
+ * address), then the shards. */
 size_t tsp_shard_buffer_bytes(const tsp_dims* dims, int D);
 
 /* Splits full weights into per-rank shards [zubnet.ai TSP item, paragraph 1:
  * "each GPU holds 1/D of the weights"].  w_full[6] = {Wq, Wk, Wv, Wo, W1, W2}
  * are device bf16 in the math orientation y = x W ([in, out]: Wq/Wk/Wv/Wo
  * [h, h], W1 [h, F], W2 [F, h]).  Writes the K-major fp16 shards into d_buf
- * (tsp_shard_buffer_bytes bytes, caller-owned) and fills *out with
- * pointers into d_buf. */
+ * (tsp_shard_buffer_bytes bytes, caller-owned, 16-byte aligned) and fills
+ * *out with pointers into d_buf.  A weight beyond +-65504 is clamped and
+ * recorded in d_buf's status section (tsp_get_device_status(d_buf, ...)
+ * then returns TSP_ERR_SATURATED). */
 int tsp_pack_shards(const tsp_dims* dims, int D, const void* const w_full[6],
                     void* d_buf, size_t buf_bytes, tsp_weights* out, cudaStream_t stream);
 
@@ -146,11 +165,14 @@ size_t tsp_workspace_bytes(const tsp_dims* dims, int D);
  *   TSP_ERR_INVALID_ARG. */
 int tsp_workspace_offsets(const tsp_dims* dims, int D, size_t off[8]);
 
-/* Clears the workspace status word (enqueued on `stream`). */
+/* Clears a status section - the workspace's, the MLP backward workspace's
+ * or the shard buffer's: its status and flags words (enqueued on `stream`). */
 int tsp_reset_device_status(void* ws, cudaStream_t stream);
 
-/* Synchronises `stream`, then reads the workspace status word: TSP_OK or
- * TSP_ERR_TIMEOUT (sticky until tsp_reset_device_status). */
+/* Synchronises `stream`, then reads a status section (see
+ * tsp_reset_device_status): TSP_ERR_TIMEOUT if a bounded wait ran out, else
+ * TSP_ERR_SATURATED if an fp16 conversion saturated, else TSP_OK.  Both are
+ * sticky until tsp_reset_device_status. */
 int tsp_get_device_status(const void* ws, cudaStream_t stream);
 
 /* K/V projection of one rank's tokens [zubnet.ai TSP item, paragraph 2:
@@ -181,13 +203,22 @@ int tsp_kv_project(const tsp_dims* dims, const tsp_weights* w, int rank,
  * a device looks up the array's device address (cudaGetSymbolAddress) with
  * that device current; make that first call before any stream capture.  All
  * calls share the one array, which keeps the last call's contents (the call
- * clears its status word itself): calls that overlap on the GPU - from
- * different streams or threads - race on it, so order them.  A device-side
- * timeout inside this call is recorded only in the array's status word and is
- * not reported.  No cudaMalloc, cudaFree or allocating library routine is
- * used.  Arguments as in tsp_kv_project. */
+ * clears its status and flags words itself): calls that overlap on the GPU
+ * - from different streams or threads - race on it, so order them.  The
+ * array's device address is cached per device and per CUDA context: after a
+ * cudaDeviceReset, or a primary context released and created again, the
+ * next call looks it up anew in the new context.  A device-side timeout or
+ * an fp16 saturation inside this call is recorded in the array's status
+ * section; tsp_kv_project_noalloc_status reads it.  No cudaMalloc, cudaFree
+ * or allocating library routine is used.  Arguments as in tsp_kv_project. */
 int tsp_kv_project_noalloc(const tsp_dims* dims, const tsp_weights* w, int rank,
                            const void* x_local, void* k_full, void* v_full, cudaStream_t stream);
+
+/* Synchronises `stream`, then reads the status section of
+ * tsp_kv_project_noalloc's static scratch (the last call's, on the current
+ * device): TSP_OK, TSP_ERR_TIMEOUT or TSP_ERR_SATURATED, as
+ * tsp_get_device_status.  The paper has no counterpart. */
+int tsp_kv_project_noalloc_status(cudaStream_t stream);
 
 /* The rank's layer forward given the all-gathered K/V [zubnet.ai TSP item,
  * paragraphs 1-2, 4]:
@@ -265,7 +296,9 @@ int tsp_mlp_backward(const tsp_dims* dims, const tsp_weights* w,
  * nothing will ever complete, with a limit of `timeout_ns` nanoseconds
  * (at most 2e9).  The wait gives up, the kernel records TSP_ERR_TIMEOUT in
  * the workspace status word and returns normally, so the context stays
- * usable.  ws: at least 256 bytes. */
+ * usable.  ws: at least 256 bytes; NULL targets the status section of
+ * tsp_kv_project_noalloc's static scratch (read by
+ * tsp_kv_project_noalloc_status). */
 int tsp_selftest_wait_timeout(void* ws, uint64_t timeout_ns, cudaStream_t stream);
 
 #ifdef __cplusplus

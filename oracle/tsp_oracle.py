@@ -172,15 +172,34 @@ def causal_attention(q, k, v, q_pos, n_heads: int, scale: float,
 # ----------------------------------------------------------------------------
 # the plain (unsharded) layer
 # ----------------------------------------------------------------------------
-def _weights(w: dict, rnd) -> dict:
+class StoredWeights(dict):
+    """Weights already rounded to a storage format (what ``stored_weights``
+    returns).  Rounding to nearest is idempotent, so handing these to the
+    layer functions computes exactly what the raw weights give; it only
+    skips re-rounding every matrix on every call."""
+
+    def __init__(self, w: dict, storage):
+        super().__init__(w)
+        self.storage = storage
+
+
+def stored_weights(w: dict, storage="fp16") -> StoredWeights:
+    """The weights rounded once to `storage` (fp64 arrays), for repeated calls."""
+    rnd = _rounder(storage)
+    return StoredWeights({n: rnd(np.asarray(a, dtype=np.float64)) for n, a in w.items()}, storage)
+
+
+def _weights(w: dict, rnd, storage="fp16") -> dict:
     """The weights as the layer holds them for its matmuls."""
+    if isinstance(w, StoredWeights) and w.storage == storage:
+        return w
     return {n: rnd(np.asarray(a, dtype=np.float64)) for n, a in w.items()}
 
 
 def kv_project(x_rows, w: dict, eps: float = LN_EPS, storage="fp16"):
     """K and V rows of tokens `x_rows`: LN1(x) @ Wk and LN1(x) @ Wv."""
     rnd = _rounder(storage)
-    w = _weights(w, rnd)
+    w = _weights(w, rnd, storage)
     xn = rnd(layer_norm(x_rows, eps))
     return rnd(xn @ w["wk"]), rnd(xn @ w["wv"])
 
@@ -196,7 +215,7 @@ def rank_rows_forward(x_rows, q_pos, k_full, v_full, w: dict, n_heads: int,
     Returns the output and the stored intermediates.
     """
     rnd = _rounder(storage)
-    w = _weights(w, rnd)
+    w = _weights(w, rnd, storage)
     x = np.asarray(x_rows, dtype=np.float64)
     h = x.shape[1]
     if scale is None:
@@ -234,7 +253,7 @@ def kv_all_gather_sharded(x_full, D: int, w: dict, eps: float = LN_EPS,
     places each rank's rows back at their global positions.
     """
     rnd = _rounder(storage)
-    w = _weights(w, rnd)
+    w = _weights(w, rnd, storage)
     x_full = np.asarray(x_full, dtype=np.float64)
     T, h = x_full.shape
     hs = h // D
@@ -263,7 +282,7 @@ def rank_forward_sharded(rank: int, D: int, x_local, k_full, v_full, w: dict,
     local, so no all-reduce is needed.
     """
     rnd = _rounder(storage)
-    w = _weights(w, rnd)
+    w = _weights(w, rnd, storage)
     x = np.asarray(x_local, dtype=np.float64)
     L, h = x.shape
     T = np.asarray(k_full).shape[0]

@@ -45,7 +45,7 @@ def test_struct_layouts_match_header():
 
 
 def test_status_strings(L):
-    for code in range(6):
+    for code in range(7):
         assert L.tsp_status_string(code).decode() == tsp.STATUS[code]
 
 
@@ -68,6 +68,8 @@ def dims(T=512, h=256, H=4, F=1024):
     (dict(T=768, h=192, H=3, F=768), 2, tsp.TSP_ERR_INVALID_ARG),  # H % D
     (dict(h=256, H=4, F=1024), 4, tsp.TSP_OK),   # h/D = 64
     (dict(h=256, H=4, F=96), 2, tsp.TSP_ERR_UNSUPPORTED),  # F/D = 48
+    (dict(T=256, h=8192, H=64, F=16384), 2, tsp.TSP_OK),     # the widest rows the LayerNorm kernels hold
+    (dict(T=256, h=8320, H=65, F=16640), 1, tsp.TSP_ERR_UNSUPPORTED),  # h > 8192
 ])
 def test_check_dims(L, kw, D, expect):
     d = dims(**kw)
@@ -81,8 +83,8 @@ def test_workspace_sizes_and_offsets(L):
     L_tok = 131072 // 8
     assert off[5] + L_tok * 16384 * 2 <= off[7]
     assert all(o % 1024 == 0 for o in off)
-    # shard buffer: all six weights once
-    assert tsp.shard_buffer_bytes(d, 8) == 2 * (4 * 4096 * 4096 + 2 * 4096 * 16384)
+    # shard buffer: a 1 KiB status section, then all six weights once
+    assert tsp.shard_buffer_bytes(d, 8) == 1024 + 2 * (4 * 4096 * 4096 + 2 * 4096 * 16384)
 
 
 def test_bad_arguments_fail_before_any_device_work(L):
@@ -113,8 +115,40 @@ def test_bad_arguments_fail_before_any_device_work(L):
     assert L.tsp_zigzag_index(512, 2, 2, None, None) == tsp.TSP_ERR_INVALID_ARG
     assert L.tsp_zigzag_index(0, 2, 0, None, None) == tsp.TSP_OK
     # self-test limits
-    assert L.tsp_selftest_wait_timeout(None, 1000, None) == tsp.TSP_ERR_INVALID_ARG
+    assert L.tsp_selftest_wait_timeout(256, 0, None) == tsp.TSP_ERR_INVALID_ARG
+    assert L.tsp_selftest_wait_timeout(None, 0, None) == tsp.TSP_ERR_INVALID_ARG
     assert L.tsp_selftest_wait_timeout(256, 3 * 10 ** 9, None) == tsp.TSP_ERR_INVALID_ARG
+
+
+def test_rank_step_host_checks_everything_before_its_first_copy(L):
+    """tsp_rank_step_host validates every argument tsp_rank_step would, before
+    it enqueues the host-to-device copy: without a GPU, any CUDA call would
+    return TSP_ERR_CUDA, so an INVALID_ARG here shows nothing was enqueued."""
+    d = dims()
+    w = tsp.Weights()
+    w.D = 2
+    for name in tsp.WEIGHT_NAMES:
+        arr = getattr(w, name)
+        for k in range(2):
+            arr[k] = 0x10000 * (k + 1)
+    ws, nws = 256, 1 << 30
+    ok = dict(hx=0x1000, xs=0x2000, k=0x3000, v=0x4000, ys=0x5000, hy=0x6000)
+
+    def call(y_dtype=0, **kw):
+        a = dict(ok, **kw)
+        return L.tsp_rank_step_host(ctypes.byref(d), ctypes.byref(w), 0, a["hx"], a["xs"], a["k"], a["v"], a["ys"],
+                                    a["hy"], y_dtype, ws, nws, None)
+    assert call(y_dtype=7) == tsp.TSP_ERR_INVALID_ARG      # output dtype
+    assert call(k=None) == tsp.TSP_ERR_INVALID_ARG         # K
+    assert call(v=0x4008) == tsp.TSP_ERR_INVALID_ARG       # V misaligned
+    assert call(xs=0x2004) == tsp.TSP_ERR_INVALID_ARG      # token staging misaligned
+    assert call(ys=None) == tsp.TSP_ERR_INVALID_ARG        # result staging
+    assert call(hx=None) == tsp.TSP_ERR_INVALID_ARG        # host tokens
+    # with valid arguments the first CUDA call is reached and fails for want
+    # of a GPU (on a GPU machine it would copy from the fake host address)
+    import torch
+    if not torch.cuda.is_available():
+        assert call() == tsp.TSP_ERR_CUDA
 
 
 def test_empty_sequence_is_a_no_op(L):

@@ -8,6 +8,13 @@ the L tokens (relative ~sqrt(K) * 2^-24, about 1e-5), the ex2-based GELU'
 (2^-22), and rare one-ulp flips of a stored 16-bit value where fp32 and fp64
 round differently.  Bound: rel-L2 <= 1e-3 and max-abs <= 1e-2 * max |ref|
 per output, about 100x the measured errors.
+
+Against the plain chain rule (the oracle with no 16-bit storage at all) the
+bf16 gradient operands dominate: each stored value carries a relative
+rounding error of at most 2^-9 (rms 2^-9 / sqrt(3) = 1.1e-3), and dW1, dW2
+take two such operands per product, so rel-L2 ~ 2.4e-3 is expected (the
+oracle's two precision models measure 1.7e-3 to 2.4e-3 apart on these
+shapes).  Bound: rel-L2 <= 1e-2 and max-abs <= 1e-2 * max |ref|.
 """
 import numpy as np
 import pytest
@@ -20,6 +27,7 @@ pytestmark = pytest.mark.gpu
 
 REL_L2 = 1e-3
 REL_MAX = 1e-2
+PLAIN_REL_L2 = 1e-2
 
 
 def _run(T, h, H, F, D, seed, zero_dy=False):
@@ -41,25 +49,30 @@ def _run(T, h, H, F, D, seed, zero_dy=False):
     return raw, got
 
 
-def _close(name, got, ref):
+def _close(name, got, ref, rel_l2=REL_L2):
     assert np.isfinite(got).all(), name
     err = float(np.abs(got - ref).max())
     scale = float(np.abs(ref).max())
     rel = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
-    assert err <= REL_MAX * scale and rel <= REL_L2, f"{name}: max-abs {err:.3e} (scale {scale:.3e}) rel-L2 {rel:.3e}"
+    print(f"{name}: max-abs {err:.3e} (scale {scale:.3e}) rel-L2 {rel:.3e}")
+    assert err <= REL_MAX * scale and rel <= rel_l2, f"{name}: max-abs {err:.3e} (scale {scale:.3e}) rel-L2 {rel:.3e}"
 
 
 @pytest.mark.parametrize("T,h,H,F,D,seed", [
     (512, 256, 4, 1024, 2, 21),      # L = 256: one 256-row tile
     (1024, 512, 4, 2048, 4, 22),     # D = 4
     (3072, 256, 4, 1024, 2, 23),     # L = 1536: several M tiles
+    (2048, 512, 4, 1024, 8, 27),     # F/D = 128: U on the single-SM GEMM with its transposed GELU(U) store
 ])
 def test_mlp_backward_matches_oracle(T, h, H, F, D, seed):
     raw, got = _run(T, h, H, F, D, seed)
     w = {n: raw[n].double().numpy() for n in ("w1", "w2")}
-    ref = O.mlp_backward(raw["y1"].double().numpy(), raw["dy"].double().numpy(), w)
+    y1, dy = raw["y1"].double().numpy(), raw["dy"].double().numpy()
+    ref = O.mlp_backward(y1, dy, w)
+    plain = O.mlp_backward(y1, dy, w, storage=None, grad_storage=None)
     for k in ("dy1", "dw1", "dw2"):
         _close(k, got[k], ref[k])
+        _close(k + " vs plain chain rule", got[k], plain[k], PLAIN_REL_L2)
 
 
 def test_mlp_backward_7b_128k_sampled():
@@ -76,6 +89,11 @@ def test_mlp_backward_7b_128k_sampled():
     _close("dy1", got["dy1"][rows], ref["dy1"])
     _close("dw1", got["dw1"][:, cols], ref["dw1"])
     _close("dw2", got["dw2"][frows, :], ref["dw2"])
+    plain = O.mlp_backward_sampled(raw["y1"].double().numpy(), raw["dy"].double().numpy(), w, rows, cols, frows,
+                                   storage=None, grad_storage=None)
+    _close("dy1 vs plain", got["dy1"][rows], plain["dy1"], PLAIN_REL_L2)
+    _close("dw1 vs plain", got["dw1"][:, cols], plain["dw1"], PLAIN_REL_L2)
+    _close("dw2 vs plain", got["dw2"][frows, :], plain["dw2"], PLAIN_REL_L2)
 
 
 def test_zero_gradient_gives_zeros():

@@ -3,10 +3,14 @@
 Gates (the layer's stated tolerance for bf16 layer outputs): max-abs <= 2e-2
 and relative-L2 <= 5e-3 on the layer output, computed in fp32 by the kernels
 (y_dtype fp32); the bf16 output equals the fp32 output rounded to nearest
-even bit for bit.  The oracle rounds the matmul operands to fp16 where the
-kernels store them (its default storage format).  The zigzag index map and the weight shard packing are
-integer / byte work and must match exactly.  Intermediates get looser
-diagnostic gates that catch errors the residual stream would hide.
+even bit for bit.  Every end-to-end test applies that gate twice: against
+the plain fp64 layer (the oracle with storage=None: no rounding anywhere but
+the bf16 inputs), and against the oracle that rounds the matmul operands to
+fp16 where the kernels store them (storage="fp16"), whose distance to the
+kernels is ~100x smaller and so catches smaller mistakes.  The zigzag index
+map and the weight shard packing are integer / byte work and must match
+exactly.  Intermediates get looser diagnostic gates that catch errors the
+residual stream would hide.
 
 Sizes: the tiny layer (h=256, 4 heads of 64, FFN 1024, T=512, D=2) and
 variants (D=1, D=4, ragged chunks) are compared in full; the 7B layer at
@@ -57,12 +61,19 @@ def assert_layer_close(y_gpu, y_ref, what, x=None):
 
 
 def assert_operand_close(g, e, what):
-    """A stored fp16 operand (K, V): equal up to rounding flips.  An LN output
-    that rounds the other way moves a K entry by up to ulp(xn) * |w| (about
-    2e-4 here), so a rare entry lands two fp16 units away; the bound allows
-    four units of the entry plus a floor of 2^-10 of the tensor's rms, and at
-    most 1e-4 of the entries may differ by more than one unit plus 2^-12 of
-    the rms (near zero a unit is tiny, while these errors are absolute)."""
+    """A stored fp16 operand (K, V): equal up to rounding flips.
+
+    The kernels compute the LayerNorm output in fp32 and the oracle in fp64;
+    about one entry in 2^13 lies so close to an fp16 rounding tie that the two
+    round it differently, i.e. a few entries of every h = 4096 row.  One such
+    flip moves every K entry of the row by ulp(xn) * |w| (2^-9 * 0.08 = 1.6e-4
+    at most for |xn| < 4, |w| < 4 sigma): an ABSOLUTE error, independent of the
+    K entry it lands on, so near zero it is many units of that entry.  Hence
+    the floors, in units of the tensor's rms (1.28 for the 7B layer): 2^-12 *
+    rms = 3.1e-4 covers one flip, 2^-10 * rms covers several in one dot
+    product.  Bound: every entry within four units of itself plus 2^-10 rms;
+    at most 1e-4 of the entries more than one unit plus 2^-12 rms away; and
+    rel-L2 <= 1e-3."""
     scale = float(np.sqrt(np.mean(e * e)))
     diff = np.abs(g - e)
     ulp = np.maximum(2.0 ** (np.floor(np.log2(np.maximum(np.abs(e), 2.0 ** -14))) - 10), 2.0 ** -24)
@@ -142,10 +153,13 @@ def run_full_sequence(T, h, H, F, D, seed, y_dtype=torch.float32):
     (960, 320, 5, 1280, 5, 11),    # D = 5, h/D = 64, ragged chunks c = 96
     (1536, 384, 3, 1536, 3, 13),   # head_dim 128 with one head per shard, D = 3
     (8, 256, 4, 1024, 4, 12),      # degenerate chunks: c = 1, two local rows per rank
+    (256, 8192, 64, 16384, 2, 14),  # the widest rows supported (h = 8192, 64 heads of 128)
 ])
 def test_full_sequence_all_ranks(T, h, H, F, D, seed):
     raw, K, V, Y, idx, inter = run_full_sequence(T, h, H, F, D, seed)
     x = f64(raw["x"])
+    plain = O.layer_forward(x, weights_f64(raw), H, storage=None)
+    assert_layer_close(f64(Y), plain["y"], f"T={T} D={D} vs plain layer", x)
     ref = O.layer_forward(x, weights_f64(raw), H)
     assert_layer_close(f64(Y), ref["y"], f"T={T} D={D}", x)
     for name, got in (("k", K), ("v", V)):
@@ -250,18 +264,26 @@ def test_7b_layer_T8192_rank_in_full():
         ys[r] = y.cpu()
     assert tsp.get_device_status(ws) == tsp.TSP_OK
     x = f64(raw["x"])
-    w = weights_f64(raw)
+    w = O.stored_weights(weights_f64(raw))
+    w0 = O.stored_weights(weights_f64(raw), None)
     Kr, Vr = O.kv_project(x, w)
+    K0, V0 = O.kv_project(x, w0, storage=None)
     for r, y in ys.items():
         idx = O.zigzag_index(T, D, r)
+        plain = O.rank_rows_forward(x[idx], idx, K0, V0, w0, H7, storage=None)
+        assert_layer_close(f64(y), plain["y"], f"7B T=8192 rank {r} vs plain layer", x[idx])
         ref = O.rank_rows_forward(x[idx], idx, Kr, Vr, w, H7)
         assert_layer_close(f64(y), ref["y"], f"7B T=8192 rank {r}", x[idx])
     assert_operand_close(f64(K), Kr, "k")
     assert_operand_close(f64(V), Vr, "v")
 
 
-def sampled_rank_check(T, D, rank, seed, n_sample=62):
-    """Full-size launch (as benchmarked) of one rank, checked on sampled rows."""
+def sampled_rank_check(T, D, ranks, seed, n_sample=62):
+    """Full-size launches (as benchmarked) of the given ranks on one set of
+    inputs - the rank's tokens, the weights and stand-in all-gathered K/V - each
+    checked on sampled rows (the first and last row of both chunks plus a
+    seeded sample) against the plain fp64 layer and the fp16-storage oracle.
+    Each rank's own K/V projection is checked on the same rows."""
     L = T // D
     c = L // 2
     raw = inputs.rank_inputs(L, T, h7, F7, seed)
@@ -269,39 +291,50 @@ def sampled_rank_check(T, D, rank, seed, n_sample=62):
     dims = tsp.make_dims(T, h7, H7, F7)
     sw = tsp.pack_shards(dims, D, dev)
     ws = tsp.alloc_workspace(dims, D)
-    y = torch.empty(L, h7, dtype=torch.float32, device="cuda")
-    tsp.layer_forward(dims, sw, rank, dev["x_local"], dev["k_full"], dev["v_full"], y, ws)
-    # the rank's own K/V projection, into scratch copies
-    Kp = torch.zeros(T, h7, dtype=torch.float16, device="cuda")
-    Vp = torch.zeros_like(Kp)
-    tsp.kv_project(dims, sw, rank, dev["x_local"], Kp, Vp, ws)
-    assert tsp.get_device_status(ws) == tsp.TSP_OK
-    rows = inputs.sample_rows(L, n_sample, seed, must=(0, c - 1, c, L - 1))
-    pos = O.zigzag_index(T, D, rank)
     x = f64(raw["x_local"])
-    w = weights_f64(raw)
+    w = O.stored_weights(weights_f64(raw))
+    w0 = O.stored_weights(weights_f64(raw), None)
     Kf = raw["k_full"].float().numpy()
     Vf = raw["v_full"].float().numpy()
-    ref = O.rank_rows_forward(x[rows], pos[rows], Kf, Vf, w, H7)
-    y_s = f64(y[rows])
-    assert_layer_close(y_s, ref["y"], f"7B T={T} D={D} rank {rank}", x[rows])
-    kr, vr = O.kv_project(x[rows], w)
-    gk, gv = f64(Kp[torch.as_tensor(pos[rows])]), f64(Vp[torch.as_tensor(pos[rows])])
-    assert_operand_close(gk, kr, "k rows")
-    assert_operand_close(gv, vr, "v rows")
+    y = torch.empty(L, h7, dtype=torch.float32, device="cuda")
+    Kp = torch.zeros(T, h7, dtype=torch.float16, device="cuda")
+    Vp = torch.zeros_like(Kp)
+    for rank in ranks:
+        tsp.layer_forward(dims, sw, rank, dev["x_local"], dev["k_full"], dev["v_full"], y, ws)
+        # the rank's own K/V projection, into scratch copies
+        tsp.kv_project(dims, sw, rank, dev["x_local"], Kp, Vp, ws)
+        assert tsp.get_device_status(ws) == tsp.TSP_OK
+        rows = inputs.sample_rows(L, n_sample, seed + rank, must=(0, c - 1, c, L - 1))
+        pos = O.zigzag_index(T, D, rank)
+        y_s = f64(y[rows])
+        plain = O.rank_rows_forward(x[rows], pos[rows], Kf, Vf, w0, H7, storage=None)
+        assert_layer_close(y_s, plain["y"], f"7B T={T} D={D} rank {rank} vs plain layer", x[rows])
+        ref = O.rank_rows_forward(x[rows], pos[rows], Kf, Vf, w, H7)
+        assert_layer_close(y_s, ref["y"], f"7B T={T} D={D} rank {rank}", x[rows])
+        kr, vr = O.kv_project(x[rows], w)
+        gk, gv = f64(Kp[torch.as_tensor(pos[rows])]), f64(Vp[torch.as_tensor(pos[rows])])
+        assert_operand_close(gk, kr, "k rows")
+        assert_operand_close(gv, vr, "v rows")
 
 
 def test_7b_layer_128k_rank0_sampled():
-    sampled_rank_check(131072, 8, 0, 2)
+    sampled_rank_check(131072, 8, [0], 2)
 
 
 def test_7b_layer_128k_last_rank_sampled():
-    sampled_rank_check(131072, 8, 7, 3, n_sample=30)
+    sampled_rank_check(131072, 8, [7], 3, n_sample=30)
+
+
+def test_7b_layer_128k_middle_ranks_sampled():
+    """Ranks 1-6 of the full 128K layer (every rank of the all-ranks
+    configuration is then checked at full size): each holds a different
+    chunk pair, so each walks a different key range and tile mix."""
+    sampled_rank_check(131072, 8, [1, 2, 3, 4, 5, 6], 3, n_sample=16)
 
 
 @pytest.mark.parametrize("D", [1, 2, 4, 8, 16])
 def test_7b_layer_T32768_shard_sweep_sampled(D):
-    sampled_rank_check(32768, D, 0, 4, n_sample=30)
+    sampled_rank_check(32768, D, [0], 4, n_sample=30)
 
 
 @pytest.mark.parametrize("T,h,H,F,D,ramp,n_sample", [
@@ -325,7 +358,8 @@ def test_growing_logits_force_rescales(T, h, H, F, D, ramp, n_sample):
     sw = tsp.pack_shards(dims, D, dev)
     ws = tsp.alloc_workspace(dims, D)
     Kd, Vd = k_ramp.cuda(), raw["v_full"].cuda()
-    w = weights_f64(raw)
+    w = O.stored_weights(weights_f64(raw))
+    w0 = O.stored_weights(weights_f64(raw), None)
     Kf = k_ramp.double().numpy()
     Vf = raw["v_full"].double().numpy()
     x_all = f64(raw["x_local"])
@@ -335,8 +369,56 @@ def test_growing_logits_force_rescales(T, h, H, F, D, ramp, n_sample):
         assert tsp.get_device_status(ws) == tsp.TSP_OK
         pos = O.zigzag_index(T, D, r)
         rows = np.arange(L) if n_sample is None else inputs.sample_rows(L, n_sample, 7 + r, must=(0, L // 2, L - 1))
+        plain = O.rank_rows_forward(x_all[rows], pos[rows], Kf, Vf, w0, H, storage=None)
+        assert_layer_close(f64(y)[rows], plain["y"], f"growing logits T={T} D={D} rank {r} vs plain layer",
+                           x_all[rows])
         ref = O.rank_rows_forward(x_all[rows], pos[rows], Kf, Vf, w, H)
         assert_layer_close(f64(y)[rows], ref["y"], f"growing logits T={T} D={D} rank {r}", x_all[rows])
+
+
+# --------------------------------------------------------------------------
+# fp16 range: saturations are reported, not silent
+# --------------------------------------------------------------------------
+def test_fp16_saturation_is_reported():
+    """Values beyond fp16's range are clamped to +-65504 and recorded in the
+    status section: a weight when the shards are packed, and a Q entry in the
+    QKV GEMM's epilogue.  Wq scaled by 1e5 (entries ~2000, representable)
+    gives Q entries of std 16 * 2000 = 32000, so some exceed 65504; the
+    inputs as drawn give none."""
+    T, h, H, F, D = 512, 256, 4, 1024, 2
+    raw = to_cuda(inputs.layer_inputs(T, h, F, 30))
+    dims = tsp.make_dims(T, h, H, F)
+    ws = tsp.alloc_workspace(dims, D)
+    xs = [raw["x"].index_select(0, tsp.zigzag_index(T, D, r).long()).contiguous() for r in range(D)]
+    y = torch.empty(T // D, h, dtype=torch.float32, device="cuda")
+
+    def run(w_full):
+        sw = tsp.pack_shards(dims, D, w_full)
+        K = torch.zeros(T, h, dtype=torch.float16, device="cuda")
+        V = torch.zeros_like(K)
+        tsp.reset_device_status(ws)
+        for r in range(D):
+            tsp.kv_project(dims, sw, r, xs[r], K, V, ws)
+        tsp.layer_forward(dims, sw, 0, xs[0], K, V, y, ws)
+        return sw
+    sw = run(raw)
+    assert tsp.get_device_status(sw.buf) == tsp.TSP_OK
+    assert tsp.get_device_status(ws) == tsp.TSP_OK
+    big = dict(raw)
+    big["wq"] = (raw["wq"].float() * 1e5).to(torch.bfloat16)
+    sw = run(big)
+    assert tsp.get_device_status(sw.buf) == tsp.TSP_OK          # the weights fit fp16
+    assert tsp.get_device_status(ws) == tsp.TSP_ERR_SATURATED   # some Q entries did not
+    assert torch.isfinite(y).all()
+    tsp.reset_device_status(ws)
+    assert tsp.get_device_status(ws) == tsp.TSP_OK
+    huge = dict(raw)
+    huge["w1"] = raw["w1"].clone()
+    huge["w1"][3, 5] = 1.0e6
+    sw = tsp.pack_shards(dims, D, huge)
+    assert tsp.get_device_status(sw.buf) == tsp.TSP_ERR_SATURATED
+    Fs = F // D
+    assert sw.shard("w1", 5 // Fs, (Fs, h))[5 % Fs, 3].item() == 65504.0
 
 
 # --------------------------------------------------------------------------

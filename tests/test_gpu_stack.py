@@ -1,7 +1,9 @@
 """A stack of TSP layers on one GPU (every rank in turn) against the oracle
-applied layer by layer.  Each layer's output is handed on in bf16, the layer's
-input format, on both sides: the kernels' bf16 output is the fp32 output
-rounded to nearest even, and the oracle's fp64 output is rounded the same way."""
+applied layer by layer: the fp16-storage oracle chained on its own hand-offs,
+and each layer against the plain fp64 layer given the stack's hand-off.
+Each layer's output is handed on in bf16, the layer's input format, on both
+sides: the kernels' bf16 output is the fp32 output rounded to nearest even,
+and the oracle's fp64 output is rounded the same way."""
 import numpy as np
 import pytest
 import torch
@@ -40,7 +42,7 @@ def test_stack_matches_oracle_layer_by_layer(T, h, H, F, D, n_layers):
     Y = torch.zeros(T, h, dtype=torch.float64)
     for r in range(D):
         Y[idx[r].cpu()] = ys[r].double().cpu()
-    # the oracle, layer by layer on the whole sequence
+    # the fp16-storage oracle chained layer by layer on its own bf16 hand-offs
     xr = x.double().numpy()
     for i, raw in enumerate(raws):
         w = {n: raw[n].double().numpy() for n in inputs.WEIGHT_NAMES}
@@ -51,3 +53,20 @@ def test_stack_matches_oracle_layer_by_layer(T, h, H, F, D, n_layers):
     rl = float(np.linalg.norm(got - xr) / np.linalg.norm(xr))
     print(f"stack of {n_layers}, T={T} D={D}: max-abs {err:.3e} rel-L2 {rl:.3e}")
     assert err <= 2e-2 and rl <= 5e-3
+    # every layer of the stack against the plain fp64 layer (storage=None), fed
+    # the stack's own bf16 hand-off: a chained plain oracle would let single
+    # bf16 rounding flips (0.031 at |y| >= 4) compound from layer to layer
+    prev = x.double().numpy()
+    for i, raw in enumerate(raws):
+        ys_i = stack.stack_forward(dims, layers[: i + 1], x_locals, K, V, ws, y_dtype=torch.float32)
+        Yi = torch.zeros(T, h, dtype=torch.float32)
+        for r in range(D):
+            Yi[idx[r].cpu()] = ys_i[r].cpu()
+        w = {n: raw[n].double().numpy() for n in inputs.WEIGHT_NAMES}
+        plain = O.layer_forward(prev, w, H, storage=None)["y"]
+        got_i = Yi.double().numpy()
+        err = float(np.max(np.abs(got_i - plain)))
+        rl = float(np.linalg.norm(got_i - plain) / np.linalg.norm(plain))
+        print(f"  layer {i} vs plain layer: max-abs {err:.3e} rel-L2 {rl:.3e}")
+        assert err <= 2e-2 and rl <= 5e-3, i
+        prev = Yi.to(torch.bfloat16).double().numpy()  # the bf16 hand-off the stack passes on

@@ -316,6 +316,26 @@ def test_sharded_schedule_equals_unsharded_layer(cfg, D):
         assert np.allclose(rows["y"], full["y"][idx], rtol=1e-12, atol=1e-12)
 
 
+@pytest.mark.parametrize("storage", [None, "fp16", "bf16"])
+def test_stored_weights_give_identical_results(storage):
+    """Weights rounded once (stored_weights) and handed to the layer functions
+    give bit-identical outputs: rounding to nearest is idempotent, so the
+    pre-rounding only saves the per-call rounding work."""
+    cfg = TINY
+    x, w = tiny_inputs(cfg, 33)
+    sw = O.stored_weights(w, storage)
+    a = O.layer_forward(x, w, cfg["H"], storage=storage)
+    b = O.layer_forward(x, sw, cfg["H"], storage=storage)
+    for key in ("k", "v", "q", "a", "y1", "h", "y"):
+        assert np.array_equal(a[key], b[key]), key
+    # weights stored for another format are rounded again to this one
+    w_off = {n: a_ * (1.0 + 2.0 ** -20) for n, a_ in w.items()}   # not 16-bit numbers
+    other = O.stored_weights(w_off, None)
+    c = O.layer_forward(x, other, cfg["H"], storage=storage)
+    d = O.layer_forward(x, w_off, cfg["H"], storage=storage)
+    assert np.array_equal(c["y"], d["y"])
+
+
 def test_d1_reduces_to_plain_layer():
     cfg = TINY
     x, w = tiny_inputs(cfg, 31)

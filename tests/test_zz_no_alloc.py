@@ -69,3 +69,20 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(L):
     rc = L.tsp_kv_project_noalloc(ctypes.byref(dims), ctypes.byref(w), 0, 16, 16, 16, None)
     assert rc == tsp.TSP_ERR_WORKSPACE
     assert b"exceeds" in L.tsp_last_cuda_error()
+
+
+def test_noalloc_status_reports_a_timeout_and_the_next_call_clears_it(L):
+    """A device-side timeout inside the allocation-free call lands in the
+    static scratch's status section, which tsp_kv_project_noalloc_status
+    reads.  The bounded-wait self test, aimed at that section, stands in for a
+    wait that runs out (it waits on a barrier nothing completes, then returns
+    normally); the next call starts by clearing the section."""
+    tsp.selftest_wait_timeout(None, 20_000_000)  # 20 ms
+    assert tsp.kv_project_noalloc_status() == tsp.TSP_ERR_TIMEOUT
+    T, h, H, F, D = 1024, 256, 4, 1024, 2
+    dims, sw, xs = _setup(T, h, H, F, D, 22)
+    K = torch.zeros(T, h, dtype=torch.float16, device="cuda")
+    V = torch.zeros_like(K)
+    assert _call_noalloc(L, dims, sw, 1, xs[1], K, V) == tsp.TSP_OK
+    assert tsp.kv_project_noalloc_status() == tsp.TSP_OK
+    assert K.abs().sum() > 0
