@@ -62,7 +62,7 @@ def _close(name, got, ref, rel_l2=REL_L2):
     (512, 256, 4, 1024, 2, 21),      # L = 256: one 256-row tile
     (1024, 512, 4, 2048, 4, 22),     # D = 4
     (3072, 256, 4, 1024, 2, 23),     # L = 1536: several M tiles
-    (2048, 512, 4, 1024, 8, 27),     # F/D = 128: U on the single-SM GEMM with its transposed GELU(U) store
+    (2048, 512, 8, 1024, 8, 27),     # F/D = 128: U on the single-SM GEMM with its transposed GELU(U) store
 ])
 def test_mlp_backward_matches_oracle(T, h, H, F, D, seed):
     raw, got = _run(T, h, H, F, D, seed)
