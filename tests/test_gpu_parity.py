@@ -166,9 +166,14 @@ def test_full_sequence_all_ranks(T, h, H, F, D, seed):
         assert_operand_close(f64(got), ref[name], name)
     for r in range(D):
         rows = idx[r].cpu().numpy()
-        for n, gate in (("q", 1e-3), ("a", 2e-3), ("y1", 1e-4), ("h", 2e-3)):
+        for n, gate in (("q", 1e-3), ("a", 2e-3), ("h", 2e-3)):
             rl = rel_l2(f64(inter[r][n]), ref[n][rows])
             assert rl <= gate, (r, n, rl)
+        # the attention projection Y1 - X = A Wo carries A's relative error, so
+        # it takes A's gate; Y1 itself is dominated by X in small layers (there
+        # |A Wo| ~ 0.01 |X|) and by A Wo at h = 8192 (|A Wo| ~ 2 |X|)
+        rl = rel_l2(f64(inter[r]["y1"]) - x[rows], ref["y1"][rows] - x[rows])
+        assert rl <= 2e-3, (r, "y1 - x", rl)
 
 
 def test_bf16_output_is_rounded_fp32_output():
