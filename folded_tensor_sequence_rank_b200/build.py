@@ -17,7 +17,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "csrc", "tsp_api.cu")
 OUT = os.path.join(HERE, "libtsp_b200.so")
-HEADERS = [os.path.join(HERE, "csrc", f) for f in ("ptx.cuh", "gemm_sm100.cuh", "attn_sm100.cuh", "misc_kernels.cuh")]
+HEADERS = [os.path.join(HERE, "csrc", f) for f in ("ptx.cuh", "gemm_sm100.cuh", "gemm_pair_sm100.cuh", "attn_sm100.cuh",
+                                                   "attn_bwd_sm100.cuh", "misc_kernels.cuh")]
 HEADERS.append(os.path.join(ROOT, "include", "tsp.h"))
 
 

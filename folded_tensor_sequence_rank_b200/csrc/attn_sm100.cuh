@@ -68,6 +68,13 @@ struct __align__(64) AttnParams {
   int* counter;       // work queue head (zeroed before launch)
   int* status;
   uint64_t timeout_ns;
+  // Optional stash for the backward: per row and head the log-sum-exp of the
+  // row's scaled scores in log2 units, lse2 = log2 sum_k 2^(s_k * scale *
+  // log2 e), so that P = 2^(s * scale * log2 e - lse2).  Layout [H][2][c_pad]
+  // fp32: head, local chunk, row within the chunk (c_pad = c rounded up to a
+  // multiple of 128, so every 128-row tile of a chunk starts 512-byte aligned).
+  float* lse;
+  int c_pad;
 };
 
 template <int HD>
@@ -480,6 +487,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
       ++icnt;
       tc_fence_after();
       const float inv = 1.0f / l;
+      if (p.lse != nullptr && row_valid) {
+        const int chunk = T.m0 >= p.c ? 1 : 0;
+        p.lse[(w.head * 2 + chunk) * p.c_pad + (T.m0 - chunk * p.c) + row] = m_used + lg2_approx(l);
+      }
       __half* dst = p.out + static_cast<int64_t>(T.m0 + row) * p.ldo + w.head * HD;
 #pragma unroll
       for (int j = 0; j < HD / 32; ++j) {

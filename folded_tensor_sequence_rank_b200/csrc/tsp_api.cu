@@ -16,6 +16,7 @@
 #include <mutex>
 
 #include "tsp.h"
+#include "attn_bwd_sm100.cuh"
 #include "attn_sm100.cuh"
 #include "gemm_pair_sm100.cuh"
 #include "gemm_sm100.cuh"
@@ -96,6 +97,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 // ---------------------------------------------------------------- sizes
 struct Sizes {
   int64_t T, c, L;
+  int64_t c_pad;  // c rounded up to a whole 128-row tile (rows of the per-chunk stashes)
   int h, H, d, F, D, hs, Fs;
 };
 
@@ -104,6 +106,7 @@ Sizes sizes_of(const tsp_dims* dims, int D) {
   s.T = dims->T;
   s.D = D;
   s.c = dims->T / (2 * D);
+  s.c_pad = (s.c + 127) / 128 * 128;
   s.L = 2 * s.c;
   s.h = dims->h;
   s.H = dims->n_heads;
@@ -115,8 +118,11 @@ Sizes sizes_of(const tsp_dims* dims, int D) {
 }
 
 struct WsLayout {
-  size_t status, xn, q, a, y1, hbuf, counters, total;
+  size_t status, xn, q, a, y1, hbuf, counters, lse, total;
 };
+
+// Bytes of a per-head, per-chunk fp32 stash [H][2][c_pad].
+size_t stash_bytes(const Sizes& s) { return static_cast<size_t>(s.H) * 2 * s.c_pad * 4; }
 
 WsLayout ws_layout(const Sizes& s) {
   WsLayout w;
@@ -128,8 +134,24 @@ WsLayout ws_layout(const Sizes& s) {
   w.a = o; o += align_up(static_cast<size_t>(s.L) * s.h * 2);
   w.y1 = o; o += align_up(static_cast<size_t>(s.L) * s.h * 4);
   w.hbuf = o; o += align_up(static_cast<size_t>(s.L) * s.F * 2);
+  w.lse = o; o += align_up(stash_bytes(s));
   w.total = o;
   return w;
+}
+
+// Workspace of tsp_attn_backward: status section, work-queue counter, Delta.
+struct AbwdLayout {
+  size_t status, counters, delta, total;
+};
+
+AbwdLayout abwd_layout(const Sizes& s) {
+  AbwdLayout b;
+  size_t o = 0;
+  b.status = o; o += align_up(256);
+  b.counters = o; o += align_up(256);
+  b.delta = o; o += align_up(stash_bytes(s));
+  b.total = o;
+  return b;
 }
 
 int check_dims(const tsp_dims* dims, int D) {
@@ -342,7 +364,7 @@ int launch_ksplit(const Sizes& s, int rank, const __half* a, int Kdim, const voi
 }
 
 int launch_attention(const Sizes& s, int rank, const tsp_dims* dims, const __half* q, const void* k_full,
-                     const void* v_full, __half* out, int* counter, int* status, cudaStream_t st) {
+                     const void* v_full, __half* out, float* lse, int* counter, int* status, cudaStream_t st) {
   if (s.L == 0) return TSP_OK;
   static thread_local AttnParams p;
   std::memset(&p, 0, sizeof(p));
@@ -365,6 +387,8 @@ int launch_attention(const Sizes& s, int rank, const tsp_dims* dims, const __hal
   p.counter = counter;
   p.status = status;
   p.timeout_ns = kDefaultTimeoutNs;
+  p.lse = lse;
+  p.c_pad = static_cast<int>(s.c_pad);
   TSP_CUDA(cudaMemsetAsync(counter, 0, sizeof(int), st));
   const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
   if (s.d == 128) {
@@ -397,7 +421,7 @@ struct Ctx {
   int* status;
   int* counters;
   __half *xn, *q, *a, *hbuf;
-  float* y1;
+  float *y1, *lse;
 };
 
 int make_ctx(Ctx& c, const tsp_dims* dims, const tsp_weights* w, int rank, void* ws, size_t ws_bytes) {
@@ -419,6 +443,7 @@ int make_ctx(Ctx& c, const tsp_dims* dims, const tsp_weights* w, int rank, void*
   c.a = reinterpret_cast<__half*>(c.ws + c.lay.a);
   c.y1 = reinterpret_cast<float*>(c.ws + c.lay.y1);
   c.hbuf = reinterpret_cast<__half*>(c.ws + c.lay.hbuf);
+  c.lse = reinterpret_cast<float*>(c.ws + c.lay.lse);
   return TSP_OK;
 }
 
@@ -431,7 +456,7 @@ int record(cudaEvent_t* ev, int i, cudaStream_t st) {
 int layer_tail(Ctx& c, const tsp_dims* dims, const tsp_weights* w, int rank, const void* x_local, const void* k_full,
                const void* v_full, void* y_local, int y_dtype, cudaStream_t st, cudaEvent_t* ev) {
   const Sizes& s = c.s;
-  int rc = launch_attention(s, rank, dims, c.q, k_full, v_full, c.a, c.counters, c.status, st);
+  int rc = launch_attention(s, rank, dims, c.q, k_full, v_full, c.a, c.lse, c.counters, c.status, st);
   if (rc) return rc;
   if ((rc = record(ev, 3, st))) return rc;
   rc = launch_ksplit(s, rank, c.a, s.h, reinterpret_cast<const void* const*>(w->wo), x_local, 0, c.y1, 1, c.status, st);
@@ -450,6 +475,69 @@ int layer_tail(Ctx& c, const tsp_dims* dims, const tsp_weights* w, int rank, con
                      y_dtype == TSP_OUT_F32, c.status, st);
   if (rc) return rc;
   return record(ev, 7, st);
+}
+
+// ---------------------------------------------------------------- attention backward
+template <int HD>
+int launch_attn_bwd_hd(AttnBwdParams& p, cudaStream_t st) {
+  using S = AttnBwdShape<HD>;
+  static std::once_flag once;
+  static cudaError_t e = cudaSuccess;
+  std::call_once(once, [] {
+    e = cudaFuncSetAttribute(attn_bwd_tcgen05<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes);
+  });
+  TSP_CUDA(e);
+  const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
+  attn_bwd_tcgen05<HD><<<grid, kBwdThreads, S::kSmemBytes, st>>>(p);
+  TSP_CUDA(cudaGetLastError());
+  return TSP_OK;
+}
+
+// Delta, then the key-tile-outer backward kernel.  dq is zeroed here (the
+// kernel adds every key tile's contribution); dk, dv are added to.
+int launch_attn_backward(const Sizes& s, int rank, const tsp_dims* dims, const __half* q, const void* k_full,
+                         const void* v_full, const __half* o, const float* lse, const __half* d_o, float* dq,
+                         float* dk, float* dv, float* delta, int* counter, int* status, cudaStream_t st) {
+  if (s.L == 0) return TSP_OK;
+  TSP_CUDA(cudaMemsetAsync(dq, 0, static_cast<size_t>(s.L) * s.h * 4, st));
+  const dim3 grid_rows(static_cast<unsigned>(s.L));
+  if (s.d == 128)
+    attn_bwd_delta_kernel<128><<<grid_rows, 256, 0, st>>>(d_o, o, delta, s.h, static_cast<int>(s.c),
+                                                          static_cast<int>(s.c_pad), dims->softmax_scale);
+  else
+    attn_bwd_delta_kernel<64><<<grid_rows, 256, 0, st>>>(d_o, o, delta, s.h, static_cast<int>(s.c),
+                                                         static_cast<int>(s.c_pad), dims->softmax_scale);
+  TSP_CUDA(cudaGetLastError());
+  static thread_local AttnBwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  int rc = make_map(&p.map_q, q, s.L, s.h, s.h, kBwdTile);
+  if (rc) return rc;
+  if ((rc = make_map(&p.map_do, d_o, s.L, s.h, s.h, kBwdTile))) return rc;
+  if ((rc = make_map(&p.map_k, k_full, s.T, s.h, s.h, kBwdTile))) return rc;
+  if ((rc = make_map(&p.map_v, v_full, s.T, s.h, s.h, kBwdTile))) return rc;
+  p.lse = lse;
+  p.delta = delta;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.ld = s.h;
+  p.T = s.T;
+  p.c = static_cast<int>(s.c);
+  p.c_pad = static_cast<int>(s.c_pad);
+  p.rank = rank;
+  p.D = s.D;
+  p.H = s.H;
+  p.nqt = static_cast<int>((s.c + kBwdTile - 1) / kBwdTile);
+  const int64_t last = (2 * s.D - rank) * s.c;  // last position of the rank + 1
+  p.nkt = static_cast<int>((last + kBwdTile - 1) / kBwdTile);
+  p.n_items = p.nkt * s.H;
+  p.scale_log2 = dims->softmax_scale * 1.4426950408889634f;
+  p.scale = dims->softmax_scale;
+  p.counter = counter;
+  p.status = status;
+  p.timeout_ns = kDefaultTimeoutNs;
+  TSP_CUDA(cudaMemsetAsync(counter, 0, sizeof(int), st));
+  return s.d == 128 ? launch_attn_bwd_hd<128>(p, st) : launch_attn_bwd_hd<64>(p, st);
 }
 
 // ---------------------------------------------------------------- MLP backward
@@ -697,14 +785,43 @@ size_t tsp_workspace_bytes(const tsp_dims* dims, int D) {
   return ws_layout(sizes_of(dims, D)).total;
 }
 
-int tsp_workspace_offsets(const tsp_dims* dims, int D, size_t off[8]) {
+int tsp_workspace_offsets(const tsp_dims* dims, int D, size_t off[TSP_N_WS_OFFSETS]) {
   if (!off) return TSP_ERR_INVALID_ARG;
   int rc = check_dims(dims, D);
   if (rc) return rc;
   const WsLayout w = ws_layout(sizes_of(dims, D));
   off[0] = w.status; off[1] = w.xn; off[2] = w.q; off[3] = w.a;
   off[4] = w.y1; off[5] = w.hbuf; off[6] = w.counters; off[7] = w.total;
+  off[8] = w.lse;
   return TSP_OK;
+}
+
+size_t tsp_attn_backward_workspace_bytes(const tsp_dims* dims, int D) {
+  if (check_dims(dims, D) != TSP_OK) return 0;
+  return abwd_layout(sizes_of(dims, D)).total;
+}
+
+int tsp_attn_backward(const tsp_dims* dims, int D, int rank, const void* q, const void* k_full, const void* v_full,
+                      const void* o, const void* lse, const void* d_o, void* dq, void* dk_full, void* dv_full,
+                      void* ws, size_t ws_bytes, cudaStream_t stream) {
+  int rc = check_dims(dims, D);
+  if (rc) return rc;
+  if (rank < 0 || rank >= D) return TSP_ERR_INVALID_ARG;
+  const Sizes s = sizes_of(dims, D);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return TSP_ERR_INVALID_ARG;
+  const AbwdLayout b = abwd_layout(s);
+  if (ws_bytes < b.total) return TSP_ERR_WORKSPACE;
+  if (s.L == 0) return TSP_OK;
+  const void* ptrs[10] = {q, k_full, v_full, o, lse, d_o, dq, dk_full, dv_full, nullptr};
+  for (int i = 0; i < 9; ++i)
+    if (!ptrs[i] || !aligned16(ptrs[i])) return TSP_ERR_INVALID_ARG;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  return launch_attn_backward(s, rank, dims, static_cast<const __half*>(q), k_full, v_full,
+                              static_cast<const __half*>(o), static_cast<const float*>(lse),
+                              static_cast<const __half*>(d_o), static_cast<float*>(dq), static_cast<float*>(dk_full),
+                              static_cast<float*>(dv_full), reinterpret_cast<float*>(base + b.delta),
+                              reinterpret_cast<int*>(base + b.counters), reinterpret_cast<int*>(base + b.status),
+                              stream);
 }
 
 int tsp_reset_device_status(void* ws, cudaStream_t stream) {

@@ -20,6 +20,8 @@ each tensor rounded once to bf16 round-to-nearest-even):
 * ``mlp_backward_inputs``: the rank's residual rows Y1 [L, h] ~ N(0, 1) kept
   in fp32 (the residual stream is fp32), the six weights as above, then the
   loss gradient dY [L, h] ~ N(0, 1) rounded to bf16.
+* ``attention_grad_inputs``: a gradient of the attention output dA [L, h] ~
+  N(0, (0.02 sqrt(h))^2) rounded to fp16.
 """
 from __future__ import annotations
 
@@ -75,6 +77,15 @@ def mlp_backward_inputs(L: int, h: int, F: int, seed: int) -> dict:
     out.update(_weights(gen, h, F))
     out["dy"] = _draw(gen, (L, h), 1.0)
     return out
+
+
+def attention_grad_inputs(L: int, h: int, seed: int) -> torch.Tensor:
+    """A gradient of the attention output dA [L, h] ~ N(0, (0.02 sqrt(h))^2),
+    the spread dY1 Wo^T has for dY1 ~ N(0, 1) and weights ~ N(0, 0.02^2),
+    rounded to fp16 (the format the attention backward takes it in); CPU."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(seed)
+    return _draw(gen, (L, h), WEIGHT_STD * math.sqrt(h), torch.float16)
 
 
 def sample_rows(n_rows: int, n_sample: int, seed: int, must: tuple = ()) -> list:

@@ -16,6 +16,7 @@ import torch
 
 MAX_D = 16
 N_STEP_EVENTS = 8
+N_WS_OFFSETS = 9
 OUT_BF16, OUT_F32 = 0, 1
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "CUDA error",
           4: "device wait timed out", 5: "workspace too small", 6: "fp16 conversion saturated"}
@@ -78,6 +79,8 @@ def lib() -> ctypes.CDLL:
         "tsp_rank_step": (i32, [pd, pw, i32, vp, vp, vp, vp, i32, vp, sz, vp, ctypes.POINTER(vp)]),
         "tsp_rank_step_host": (i32, [pd, pw, i32, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]),
         "tsp_selftest_wait_timeout": (i32, [vp, ctypes.c_uint64, vp]),
+        "tsp_attn_backward_workspace_bytes": (sz, [pd, i32]),
+        "tsp_attn_backward": (i32, [pd, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "tsp_mlp_backward_workspace_bytes": (sz, [pd, i32]),
         "tsp_mlp_backward": (i32, [pd, pw, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, ctypes.POINTER(vp)]),
     }
@@ -179,7 +182,7 @@ def workspace_bytes(dims: Dims, D: int) -> int:
 
 
 def workspace_offsets(dims: Dims, D: int) -> list:
-    off = (ctypes.c_size_t * 8)()
+    off = (ctypes.c_size_t * N_WS_OFFSETS)()
     _check(lib().tsp_workspace_offsets(ctypes.byref(dims), D, off), "tsp_workspace_offsets")
     return list(off)
 
@@ -198,10 +201,22 @@ def workspace_view(ws: torch.Tensor, dims: Dims, D: int, name: str) -> torch.Ten
     L, h, F = dims.T // D, dims.h, dims.ffn
     table = {"xn": (1, torch.float16, (L, h)), "q": (2, torch.float16, (L, h)),
              "a": (3, torch.float16, (L, h)), "y1": (4, torch.float32, (L, h)),
-             "h": (5, torch.float16, (L, F))}
+             "h": (5, torch.float16, (L, F)), "lse": (8, torch.float32, (dims.n_heads, 2, stash_rows(dims, D)))}
     i, dt, shape = table[name]
     nb = int(torch.tensor(shape).prod()) * (4 if dt == torch.float32 else 2)
     return ws[off[i]: off[i] + nb].view(dt).view(*shape)
+
+
+def stash_rows(dims: Dims, D: int) -> int:
+    """Rows per chunk of the per-head stashes [H][2][c_pad]: c rounded up to 128."""
+    c = dims.T // (2 * D)
+    return (c + 127) // 128 * 128
+
+
+def lse_rows(lse_stash: torch.Tensor, dims: Dims, D: int) -> torch.Tensor:
+    """The forward's log-sum-exp stash [H][2][c_pad] as [T/D, H] in rank-local order."""
+    c = dims.T // (2 * D)
+    return torch.cat([lse_stash[:, 0, :c], lse_stash[:, 1, :c]], dim=1).t()
 
 
 def reset_device_status(ws: torch.Tensor, stream=None):
@@ -277,6 +292,32 @@ def rank_step(dims: Dims, w: ShardedWeights, rank: int, x_local, k_full, v_full,
     yd = OUT_F32 if y_local.dtype == torch.float32 else OUT_BF16
     _check(lib().tsp_rank_step(ctypes.byref(dims), ctypes.byref(w.struct), rank, px, pk, pv, py, yd, pws,
                                ws.numel(), _stream(stream), _events(events)), "tsp_rank_step")
+
+
+def attn_backward_workspace_bytes(dims: Dims, D: int) -> int:
+    return lib().tsp_attn_backward_workspace_bytes(ctypes.byref(dims), D)
+
+
+def alloc_attn_backward_workspace(dims: Dims, D: int, device="cuda") -> torch.Tensor:
+    n = attn_backward_workspace_bytes(dims, D)
+    if n == 0:
+        _check(check_dims(dims, D) or TSP_ERR_INVALID_ARG, "tsp_attn_backward_workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def attn_backward(dims: Dims, D: int, rank: int, q, k_full, v_full, o, lse, d_o, dq, dk_full, dv_full, aws,
+                  stream=None):
+    """Backward of rank `rank`'s causal attention: dq [T/D, h] fp32 (overwritten),
+    dk_full, dv_full [T, h] fp32 (added to), from the forward's Q, A (o) and
+    log-sum-exp stash, the all-gathered K/V and the gradient d_o of A (fp16)."""
+    L, h, T = dims.T // D, dims.h, dims.T
+    args = [_ptr(q, "q", torch.float16, (L, h)), _ptr(k_full, "k_full", torch.float16, (T, h)),
+            _ptr(v_full, "v_full", torch.float16, (T, h)), _ptr(o, "o", torch.float16, (L, h)),
+            _ptr(lse, "lse", torch.float32, (dims.n_heads, 2, stash_rows(dims, D))),
+            _ptr(d_o, "d_o", torch.float16, (L, h)), _ptr(dq, "dq", torch.float32, (L, h)),
+            _ptr(dk_full, "dk_full", torch.float32, (T, h)), _ptr(dv_full, "dv_full", torch.float32, (T, h))]
+    _check(lib().tsp_attn_backward(ctypes.byref(dims), D, rank, *args, _ptr(aws, "aws", torch.uint8), aws.numel(),
+                                   _stream(stream)), "tsp_attn_backward")
 
 
 def mlp_backward_workspace_bytes(dims: Dims, D: int) -> int:

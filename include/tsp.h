@@ -73,6 +73,7 @@ extern "C" {
 
 #define TSP_MAX_D 16
 #define TSP_N_STEP_EVENTS 8
+#define TSP_N_WS_OFFSETS 9
 
 typedef enum {
   TSP_OK = 0,
@@ -156,14 +157,19 @@ int tsp_pack_shards(const tsp_dims* dims, int D, const void* const w_full[6],
 size_t tsp_workspace_bytes(const tsp_dims* dims, int D);
 
 /* Byte offsets inside the workspace of the per-rank intermediates, for
- * inspection after a call (all rank-local order, row-major):
- *   off[0] status word (int32),  off[1] LN output xn fp16 [L, h] (LN2's
- *   output after tsp_layer_forward),  off[2] Q fp16 [L, h],  off[3]
- *   attention output fp16 [L, h],  off[4] Y1 = X + attention projection,
- *   fp32 [L, h],  off[5] H = GELU(LN2(Y1) W1) fp16 [L, F],  off[6]
- *   scheduler counters,  off[7] total bytes.  Returns TSP_OK or
- *   TSP_ERR_INVALID_ARG. */
-int tsp_workspace_offsets(const tsp_dims* dims, int D, size_t off[8]);
+ * inspection after a call and as inputs of the backward (all rank-local
+ * order, row-major):
+ *   off[0] status section,  off[1] LN output xn fp16 [L, h] (LN2's output
+ *   after tsp_layer_forward),  off[2] Q fp16 [L, h],  off[3] attention
+ *   output A fp16 [L, h],  off[4] Y1 = X + attention projection, fp32
+ *   [L, h],  off[5] H = GELU(LN2(Y1) W1) fp16 [L, F],  off[6] scheduler
+ *   counters,  off[7] total bytes,  off[8] the attention's log-sum-exp stash
+ *   fp32 [H][2][c_pad]: per head j, local chunk g (0: chunk r, 1: chunk
+ *   2D-1-r) and row i of the chunk, log2 of sum_k 2^(scale * log2(e) *
+ *   q_i . k_k) over the row's causal keys (c_pad = c rounded up to a
+ *   multiple of 128; rows i >= c are not written).  Returns TSP_OK,
+ *   TSP_ERR_INVALID_ARG or TSP_ERR_UNSUPPORTED. */
+int tsp_workspace_offsets(const tsp_dims* dims, int D, size_t off[TSP_N_WS_OFFSETS]);
 
 /* Clears a status section - the workspace's, the MLP backward workspace's
  * or the shard buffer's: its status and flags words (enqueued on `stream`). */
@@ -257,6 +263,36 @@ int tsp_rank_step_host(const tsp_dims* dims, const tsp_weights* w, int rank,
                        void* k_full, void* v_full, void* d_y_staging,
                        void* h_y_local, int y_dtype, void* ws, size_t ws_bytes,
                        cudaStream_t stream);
+
+/* Workspace bytes of tsp_attn_backward at this D (status section, work
+ * queue counter, Delta); 0 on a bad argument. */
+size_t tsp_attn_backward_workspace_bytes(const tsp_dims* dims, int D);
+
+/* Backward of one rank's causal attention against the all-gathered K/V
+ * [zubnet.ai TSP item, paragraph 1: the validated workload is training;
+ * paragraph 2: every rank attends its own zigzag tokens against the K/V of
+ * the whole sequence, so its dK and dV reach all T keys and are summed over
+ * the ranks - the reduce-scatter back to the key owners].  The chain rule
+ * through the forward (the pages give no backward), per head, for query row i
+ * at global position p(i) and its keys k <= p(i):
+ *   P = 2^(scale * log2(e) * q_i . k_k - lse2_i)  (lse2 from the forward),
+ *   dP = dO V^T,  Delta_i = rowsum(dO_i * O_i),
+ *   dS = scale * P * (dP - Delta),
+ *   dQ = dS K,  dK += dS^T Q,  dV += P^T dO.
+ * q: fp16 [T/D, h] (the forward's Q), o: fp16 [T/D, h] (the forward's
+ * attention output A), d_o: fp16 [T/D, h] (the gradient of A), all
+ * rank-local order; k_full, v_full: fp16 [T, h] natural order; lse: the
+ * forward's stash (tsp_workspace_offsets off[8], same dims, D and rank).
+ * dq: fp32 [T/D, h], overwritten.  dk_full, dv_full: fp32 [T, h] natural
+ * order, ADDED to (zero them before the first rank; running every rank adds
+ * up the whole sequence's gradients); calls that add to the same buffers
+ * must not overlap on the GPU.  P, dS and dO enter the tensor cores as fp16;
+ * scores, Delta and every accumulation are fp32.  ws:
+ * tsp_attn_backward_workspace_bytes(dims, D) bytes, 256-byte aligned, its
+ * status section read by tsp_get_device_status.  Pointers 16-byte aligned. */
+int tsp_attn_backward(const tsp_dims* dims, int D, int rank, const void* q, const void* k_full,
+                      const void* v_full, const void* o, const void* lse, const void* d_o, void* dq,
+                      void* dk_full, void* dv_full, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /* Workspace bytes of tsp_mlp_backward at this D (its own status word first,
  * then the recomputed and transposed activations); 0 on a bad argument. */

@@ -458,6 +458,67 @@ def causal_attention_backward(q, k, v, q_pos, dout, n_heads: int, scale: float):
     return dq, dk, dv
 
 
+def attention_logsumexp(q, k, q_pos, n_heads: int, scale: float) -> np.ndarray:
+    """Per row and head, the log-sum-exp (natural log) of the row's causal
+    scores: lse[i, j] = log sum_{key <= q_pos[i]} exp(scale q_ij . k_j).  The
+    softmax probabilities are exp(scale q.k - lse).  Returns [n, H]."""
+    q = np.asarray(q, dtype=np.float64)
+    q_pos = np.asarray(q_pos, dtype=np.int64)
+    n, hd = q.shape
+    d = hd // n_heads
+    out = np.zeros((n, n_heads))
+    if n == 0:
+        return out
+    kmax = int(q_pos.max()) + 1
+    allowed = np.arange(kmax)[None, :] <= q_pos[:, None]
+    for j in range(n_heads):
+        cols = slice(j * d, (j + 1) * d)
+        sc = scale * (q[:, cols] @ np.asarray(k[:kmax, cols], dtype=np.float64).T)
+        sc = np.where(allowed, sc, -np.inf)
+        m = sc.max(axis=1, keepdims=True)
+        out[:, j] = (m + np.log(np.exp(sc - m).sum(axis=1, keepdims=True)))[:, 0]
+    return out
+
+
+def attention_backward_stored(q, k, v, o, q_pos, dout, n_heads: int, scale: float, storage="fp16"):
+    """causal_attention_backward with the values a 16-bit tensor-core pipeline
+    holds rounded at the points where it stores them.  Per head:
+        dO = rnd(dout),  P = softmax of the causal scores (exact),
+        Delta = rowsum(dO * o)   (o: the stored attention output),
+        dP = dO v^T,  dS = rnd(scale P * (dP - Delta)),
+        dV = rnd(P)^T dO,  dK = dS^T q,  dQ = dS k.
+    With the exact output o = P v, Delta equals rowsum(dP * P), so with
+    storage=None this is causal_attention_backward.  q, k, v and o enter as
+    given (already 16-bit in the layer)."""
+    rnd = _rounder(storage)
+    q = np.asarray(q, dtype=np.float64)
+    o = np.asarray(o, dtype=np.float64)
+    dout = rnd(dout)
+    q_pos = np.asarray(q_pos, dtype=np.int64)
+    n, hd = q.shape
+    T = np.asarray(k).shape[0]
+    d = hd // n_heads
+    dq = np.zeros((n, hd))
+    dk = np.zeros((T, hd))
+    dv = np.zeros((T, hd))
+    if n == 0:
+        return dq, dk, dv
+    _, probs = causal_attention(q, k, v, q_pos, n_heads, scale, return_probs=True)
+    kmax = probs[0].shape[1]
+    for j in range(n_heads):
+        cols = slice(j * d, (j + 1) * d)
+        kj = np.asarray(k[:kmax, cols], dtype=np.float64)
+        vj = np.asarray(v[:kmax, cols], dtype=np.float64)
+        p = probs[j]
+        do = dout[:, cols]
+        delta = (do * o[:, cols]).sum(axis=1, keepdims=True)
+        ds = rnd(scale * p * (do @ vj.T - delta))
+        dv[:kmax, cols] = rnd(p).T @ do
+        dq[:, cols] = ds @ kj
+        dk[:kmax, cols] = ds.T @ q[:, cols]
+    return dq, dk, dv
+
+
 def rank_layer_backward(rank: int, D: int, x_full, w: dict, dy_local, n_heads: int,
                         eps: float = LN_EPS, scale: float | None = None) -> dict:
     """One TSP rank's share of the whole layer's backward, in plain fp64 (no

@@ -234,3 +234,22 @@ def test_mlp_backward_binding_checks_shapes_before_the_call(L):
     cpu = torch.zeros(4, dtype=torch.bfloat16)
     with pytest.raises(ValueError):  # CPU tensors are refused before the library is called
         tsp.mlp_backward(d, w, cpu, cpu, cpu, cpu, cpu, cpu, cpu, torch.zeros(16, dtype=torch.uint8))
+
+
+def test_attn_backward_checks_arguments_first(L):
+    d = dims()
+    n = L.tsp_attn_backward_workspace_bytes(ctypes.byref(d), 2)
+    assert n > 0
+    ok = [0x1000 * (i + 1) for i in range(9)]
+
+    def call(rank=0, D=2, ws=256, nws=n, ptrs=ok):
+        return L.tsp_attn_backward(ctypes.byref(d), D, rank, *ptrs, ws, nws, None)
+    assert call(rank=2) == tsp.TSP_ERR_INVALID_ARG                 # rank out of range
+    assert call(D=3) == tsp.TSP_ERR_INVALID_ARG                    # H % D
+    assert call(ws=257) == tsp.TSP_ERR_INVALID_ARG                 # misaligned workspace
+    assert call(nws=n - 1) == tsp.TSP_ERR_WORKSPACE
+    for i in range(9):                                             # each pointer: null, then misaligned
+        assert call(ptrs=ok[:i] + [None] + ok[i + 1:]) == tsp.TSP_ERR_INVALID_ARG, i
+        assert call(ptrs=ok[:i] + [ok[i] + 8] + ok[i + 1:]) == tsp.TSP_ERR_INVALID_ARG, i
+    e = dims(T=0)
+    assert L.tsp_attn_backward(ctypes.byref(e), 2, 0, *ok, 256, 1 << 20, None) == tsp.TSP_OK  # no tokens

@@ -165,3 +165,80 @@ def test_rank_backwards_sum_to_the_whole_layer_gradient(T, D):
     np.testing.assert_allclose(dx, xt.grad.numpy(), rtol=1e-9, atol=1e-11)
     for n in w:
         np.testing.assert_allclose(grads[n], wt[n].grad.numpy(), rtol=1e-9, atol=1e-11, err_msg=n)
+
+
+# --------------------------------------------------------------------------
+# the stored-value form (what a 16-bit tensor-core pipeline computes)
+# --------------------------------------------------------------------------
+def test_logsumexp_closed_form_and_library():
+    """attention_logsumexp against torch.logsumexp of the masked scores, and
+    exp(score - lse) against the oracle's own probabilities."""
+    H, d, T = 2, 4, 25
+    q, k, v, pos, _ = _inputs(5, 7, T, H, d)
+    s = 0.7
+    lse = O.attention_logsumexp(q, k, pos, H, s)
+    _, probs = O.causal_attention(q, k, v, pos, H, s, return_probs=True)
+    for j in range(H):
+        cols = slice(j * d, (j + 1) * d)
+        sc = torch.tensor(s * q[:, cols] @ k[:, cols].T)
+        sc = sc.masked_fill(torch.tensor(np.arange(T)[None, :] > pos[:, None]), -np.inf)
+        np.testing.assert_allclose(lse[:, j], torch.logsumexp(sc, dim=1).numpy(), rtol=1e-13)
+        kmax = probs[j].shape[1]
+        p = np.exp(s * q[:, cols] @ k[:kmax, cols].T - lse[:, j:j + 1]) * (np.arange(kmax)[None, :] <= pos[:, None])
+        np.testing.assert_allclose(p, probs[j], atol=1e-14)
+    # one key: lse is that key's score
+    one = O.attention_logsumexp(q[:1], k, [0], H, s)
+    np.testing.assert_allclose(one[0], [s * q[0, :d] @ k[0, :d], s * q[0, d:] @ k[0, d:]], rtol=1e-13)
+
+
+def test_stored_backward_without_rounding_is_the_plain_backward():
+    """storage=None with the exact output o = P v: Delta = rowsum(dO * o)
+    equals rowsum(dP * P), so the stored form reduces to the pinned plain
+    backward (the scale folded into dS changes nothing either)."""
+    H, d, T = 3, 8, 40
+    q, k, v, pos, dout = _inputs(6, 12, T, H, d)
+    s = 1.0 / np.sqrt(d)
+    o = O.causal_attention(q, k, v, pos, H, s)
+    got = O.attention_backward_stored(q, k, v, o, pos, dout, H, s, storage=None)
+    ref = O.causal_attention_backward(q, k, v, pos, dout, H, s)
+    for g, r in zip(got, ref):
+        np.testing.assert_allclose(g, r, rtol=1e-11, atol=1e-13)
+
+
+def _torch_stored_backward(q, k, v, o, pos, dout, H, s):
+    """The stored-value backward written independently with torch ops: the
+    probabilities from torch.softmax, 16-bit rounding by a cast to float16."""
+    f16 = lambda t: t.to(torch.float16).to(torch.float64)
+    q, k, v, o, dout = (torch.tensor(a) for a in (q, k, v, o, dout))
+    n, hd = q.shape
+    d = hd // H
+    T = k.shape[0]
+    mask = torch.tensor(np.arange(T)[None, :] > np.asarray(pos)[:, None])
+    do = f16(dout)
+    dq, dk, dv = torch.zeros(n, hd, dtype=torch.float64), torch.zeros(T, hd, dtype=torch.float64), \
+        torch.zeros(T, hd, dtype=torch.float64)
+    for j in range(H):
+        c = slice(j * d, (j + 1) * d)
+        p = torch.softmax((s * q[:, c] @ k[:, c].T).masked_fill(mask, -float("inf")), dim=1)
+        delta = (do[:, c] * o[:, c]).sum(dim=1, keepdim=True)
+        ds = f16(s * p * (do[:, c] @ v[:, c].T - delta))
+        dv[:, c] = f16(p).T @ do[:, c]
+        dq[:, c] = ds @ k[:, c]
+        dk[:, c] = ds.T @ q[:, c]
+    return dq.numpy(), dk.numpy(), dv.numpy()
+
+
+def test_stored_backward_matches_torch_composition():
+    H, d, T = 2, 16, 48
+    q, k, v, pos, dout = _inputs(7, 14, T, H, d)
+    q, k, v = (O.round_fp16(a) for a in (q, k, v))
+    s = 1.0 / np.sqrt(d)
+    o = O.round_fp16(O.causal_attention(q, k, v, pos, H, s))
+    got = O.attention_backward_stored(q, k, v, o, pos, dout, H, s)
+    ref = _torch_stored_backward(q, k, v, o, pos, dout, H, s)
+    for g, r in zip(got, ref):
+        np.testing.assert_allclose(g, r, rtol=1e-12, atol=1e-14)
+    # and it stays within fp16 rounding of the plain backward
+    plain = O.causal_attention_backward(q, k, v, pos, dout, H, s)
+    for g, r in zip(got, plain):
+        assert np.linalg.norm(g - r) <= 5e-3 * np.linalg.norm(r)
