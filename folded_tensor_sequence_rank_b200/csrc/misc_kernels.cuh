@@ -32,6 +32,18 @@ __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* src, f
 }
 
 template <>
+__device__ __forceinline__ void load8<__half>(const __half* src, float (&v)[8]) {
+  const uint4 q = __ldg(reinterpret_cast<const uint4*>(src));
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[j]));
+    v[2 * j] = f.x;
+    v[2 * j + 1] = f.y;
+  }
+}
+
+template <>
 __device__ __forceinline__ void load8<float>(const float* src, float (&v)[8]) {
   const float4 a = __ldg(reinterpret_cast<const float4*>(src));
   const float4 b = __ldg(reinterpret_cast<const float4*>(src) + 1);
@@ -168,7 +180,7 @@ __global__ void __launch_bounds__(256) transpose_bf16_kernel(const Tin* __restri
     const int rr = q >> 3, cc = (q & 7) * 8;
     if (r0 + rr < rows && c0 + cc < cols) {
       float f[8];
-      unpack8<Tin>(*reinterpret_cast<const uint4*>(in + (r0 + rr) * cols + c0 + cc), f);
+      load8<Tin>(in + (r0 + rr) * cols + c0 + cc, f);
 #pragma unroll
       for (int j = 0; j < 8; ++j) tile[rr][cc + j] = f[j];
     }
@@ -281,15 +293,33 @@ __global__ void __launch_bounds__(256) layernorm_block_kernel(const Tin* __restr
 //   dy1 = dy + rstd * (g - mean(g) - xhat * mean(g * xhat)),
 //   xhat = (y1 - mean(y1)) * rstd, rstd = 1 / sqrt(var(y1) + eps)
 // (biased variance, gamma = 1, beta = 0), statistics in fp32 from the row
-// held in registers (VPT values per thread, as float4 groups).
-template <int VPT>
-__global__ void __launch_bounds__(256) ln_backward_rows_kernel(const float* __restrict__ y1,
-                                                               const float* __restrict__ g,
-                                                               const __nv_bfloat16* __restrict__ dy,
-                                                               float* __restrict__ dy1, int h, float eps) {
+// held in registers (VPT values per thread, as groups of 4).  y1 (the
+// LayerNorm's input) is fp32 or bf16, dy (the residual's gradient) bf16 or
+// fp32; dy1 may be dy itself (each value is read before it is written).
+// dy1_bf16, when not null, receives a bf16 copy of dy1.
+template <typename Tx, typename Tr>
+__device__ __forceinline__ void load4f(const Tx* src, float* v);
+template <>
+__device__ __forceinline__ void load4f<float, float>(const float* src, float* v) {
+  const float4 a = *reinterpret_cast<const float4*>(src);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+}
+template <>
+__device__ __forceinline__ void load4f<__nv_bfloat16, __nv_bfloat16>(const __nv_bfloat16* src, float* v) {
+  const uint2 q = *reinterpret_cast<const uint2*>(src);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.y));
+  v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+}
+
+template <int VPT, typename Tx, typename Tr>
+__global__ void __launch_bounds__(256) ln_backward_rows_kernel(const Tx* __restrict__ y1,
+                                                               const float* __restrict__ g, const Tr* dy,
+                                                               float* dy1, __nv_bfloat16* __restrict__ dy1_bf16,
+                                                               int h, float eps) {
   __shared__ float red[16];
   const int64_t row = blockIdx.x;
-  const float* yr = y1 + row * h;
+  const Tx* yr = y1 + row * h;
   const float* gr = g + row * h;
   float yv[VPT], gv[VPT];
   float sum = 0.f, dummy = 0.f;
@@ -297,11 +327,10 @@ __global__ void __launch_bounds__(256) ln_backward_rows_kernel(const float* __re
   for (int i = 0; i < VPT / 4; ++i) {
     const int col = (i * 256 + threadIdx.x) * 4;
     if (col < h) {
-      const float4 a = *reinterpret_cast<const float4*>(yr + col);
+      load4f<Tx, Tx>(yr + col, &yv[4 * i]);
       const float4 b = *reinterpret_cast<const float4*>(gr + col);
-      yv[4 * i] = a.x; yv[4 * i + 1] = a.y; yv[4 * i + 2] = a.z; yv[4 * i + 3] = a.w;
       gv[4 * i] = b.x; gv[4 * i + 1] = b.y; gv[4 * i + 2] = b.z; gv[4 * i + 3] = b.w;
-      sum += (a.x + a.y) + (a.z + a.w);
+      sum += (yv[4 * i] + yv[4 * i + 1]) + (yv[4 * i + 2] + yv[4 * i + 3]);
     } else {
 #pragma unroll
       for (int j = 0; j < 4; ++j) yv[4 * i + j] = gv[4 * i + j] = 0.f;
@@ -339,23 +368,56 @@ __global__ void __launch_bounds__(256) ln_backward_rows_kernel(const float* __re
   }
   block_sum2(sg, sgx, red);
   const float mg = sg / h, mgx = sgx / h;
-  const __nv_bfloat16* dr = dy + row * h;
+  const Tr* dr = dy + row * h;
   float* outr = dy1 + row * h;
 #pragma unroll
   for (int i = 0; i < VPT / 4; ++i) {
     const int col = (i * 256 + threadIdx.x) * 4;
     if (col < h) {
-      const uint2 q = *reinterpret_cast<const uint2*>(dr + col);
-      const float2 d01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.x));
-      const float2 d23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.y));
+      float d[4];
+      load4f<Tr, Tr>(dr + col, d);
       float4 o;
-      o.x = d01.x + rstd * (gv[4 * i] - mg - yv[4 * i] * mgx);
-      o.y = d01.y + rstd * (gv[4 * i + 1] - mg - yv[4 * i + 1] * mgx);
-      o.z = d23.x + rstd * (gv[4 * i + 2] - mg - yv[4 * i + 2] * mgx);
-      o.w = d23.y + rstd * (gv[4 * i + 3] - mg - yv[4 * i + 3] * mgx);
+      o.x = d[0] + rstd * (gv[4 * i] - mg - yv[4 * i] * mgx);
+      o.y = d[1] + rstd * (gv[4 * i + 1] - mg - yv[4 * i + 1] * mgx);
+      o.z = d[2] + rstd * (gv[4 * i + 2] - mg - yv[4 * i + 2] * mgx);
+      o.w = d[3] + rstd * (gv[4 * i + 3] - mg - yv[4 * i + 3] * mgx);
       *reinterpret_cast<float4*>(outr + col) = o;
+      if (dy1_bf16)
+        *reinterpret_cast<uint2*>(dy1_bf16 + row * h + col) = make_uint2(pack_bf16x2(o.x, o.y), pack_bf16x2(o.z, o.w));
     }
   }
+}
+
+// out = bf16(in), n a multiple of 8 (row-major copies of fp32 gradients for
+// the bf16 tensor-core products).
+__global__ void __launch_bounds__(256) convert_bf16_kernel(const float* __restrict__ in, __nv_bfloat16* __restrict__ out,
+                                                           int64_t n) {
+  const int64_t i = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) * 8;
+  if (i >= n) return;
+  const float4 a = *reinterpret_cast<const float4*>(in + i);
+  const float4 b = *reinterpret_cast<const float4*>(in + i + 4);
+  *reinterpret_cast<uint4*>(out + i) =
+      make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+}
+
+// The key owner's rows of the summed dK, dV after the reduce-scatter: for
+// local row i at global position pos(i) (the zigzag map: r*c + i for i < c,
+// (2D-1-r)*c + (i-c) after), out[i] = [bf16(dk[pos(i)]) | bf16(dv[pos(i)])],
+// an [L, 2h] row-major bf16 matrix.  One thread per 8 columns.
+__global__ void __launch_bounds__(256) gather_kv_grad_kernel(const float* __restrict__ dk, const float* __restrict__ dv,
+                                                             __nv_bfloat16* __restrict__ out, int64_t L, int h,
+                                                             int64_t c, int64_t off0, int64_t off1) {
+  const int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  const int per_row = (2 * h) / 8;
+  const int64_t i = t / per_row;
+  if (i >= L) return;
+  const int col = static_cast<int>(t - i * per_row) * 8;
+  const int64_t pos = i < c ? off0 + i : off1 + i;
+  const float* src = (col < h ? dk + pos * h + col : dv + pos * h + (col - h));
+  const float4 a = *reinterpret_cast<const float4*>(src);
+  const float4 b = *reinterpret_cast<const float4*>(src + 4);
+  *reinterpret_cast<uint4*>(out + i * 2 * h + col) =
+      make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
 }
 
 // Self test of the bounded waits: one thread waits on a barrier that expects

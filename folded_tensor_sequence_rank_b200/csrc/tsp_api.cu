@@ -605,17 +605,170 @@ int launch_transpose(const Tin* in, int64_t rows, int cols, __nv_bfloat16* out, 
   return TSP_OK;
 }
 
-int launch_ln_backward(const float* y1, const float* g, const __nv_bfloat16* dy, float* dy1, int64_t rows, int h,
-                       float eps, cudaStream_t st) {
+template <typename Tx, typename Tr>
+int launch_ln_backward(const Tx* y1, const float* g, const Tr* dy, float* dy1, __nv_bfloat16* dy1_bf16, int64_t rows,
+                       int h, float eps, cudaStream_t st) {
   if (rows == 0) return TSP_OK;
-  const int groups = (h + 1023) / 1024;  // float4 groups per thread
+  const int groups = (h + 1023) / 1024;  // groups of 4 values per thread
   const dim3 grid(static_cast<unsigned>(rows));
-  if (groups <= 1) ln_backward_rows_kernel<4><<<grid, 256, 0, st>>>(y1, g, dy, dy1, h, eps);
-  else if (groups <= 2) ln_backward_rows_kernel<8><<<grid, 256, 0, st>>>(y1, g, dy, dy1, h, eps);
-  else if (groups <= 4) ln_backward_rows_kernel<16><<<grid, 256, 0, st>>>(y1, g, dy, dy1, h, eps);
-  else ln_backward_rows_kernel<32><<<grid, 256, 0, st>>>(y1, g, dy, dy1, h, eps);
+  if (groups <= 1) ln_backward_rows_kernel<4, Tx, Tr><<<grid, 256, 0, st>>>(y1, g, dy, dy1, dy1_bf16, h, eps);
+  else if (groups <= 2) ln_backward_rows_kernel<8, Tx, Tr><<<grid, 256, 0, st>>>(y1, g, dy, dy1, dy1_bf16, h, eps);
+  else if (groups <= 4) ln_backward_rows_kernel<16, Tx, Tr><<<grid, 256, 0, st>>>(y1, g, dy, dy1, dy1_bf16, h, eps);
+  else ln_backward_rows_kernel<32, Tx, Tr><<<grid, 256, 0, st>>>(y1, g, dy, dy1, dy1_bf16, h, eps);
   TSP_CUDA(cudaGetLastError());
   return TSP_OK;
+}
+
+int launch_convert_bf16(const float* in, __nv_bfloat16* out, int64_t n, cudaStream_t st) {
+  if (n == 0) return TSP_OK;
+  const int64_t threads = n / 8;
+  convert_bf16_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(in, out, n);
+  TSP_CUDA(cudaGetLastError());
+  return TSP_OK;
+}
+
+// Shapes the backward implements: whole 256-column tiles, and whole 128-row
+// tiles of tokens (the transposed epilogue stores need every lane of a warp).
+int check_backward_shape(const Sizes& s) {
+  if (s.h % 256 || s.F % 256 || s.L % 128) return TSP_ERR_UNSUPPORTED;
+  return TSP_OK;
+}
+
+// The MLP half of the backward (tsp_mlp_backward's steps): dY1 = dL/dY1 (fp32,
+// and a bf16 copy when dy1b is not null), dW1, dW2.
+int mlp_backward_core(const Sizes& s, const tsp_dims* dims, const tsp_weights* w, const void* w1_full,
+                      const void* w2_full, const float* y1, const __nv_bfloat16* dy, float* dy1, __nv_bfloat16* dy1b,
+                      float* dw1, float* dw2, uint8_t* base, const BwdLayout& b, cudaStream_t stream,
+                      cudaEvent_t* ev) {
+  int rc;
+  int* status = reinterpret_cast<int*>(base + b.status);
+  if ((rc = record(ev, 0, stream))) return rc;
+  if (s.L == 0) {  // no tokens: zero weight gradients
+    TSP_CUDA(cudaMemsetAsync(dw1, 0, static_cast<size_t>(s.h) * s.F * 4, stream));
+    TSP_CUDA(cudaMemsetAsync(dw2, 0, static_cast<size_t>(s.F) * s.h * 4, stream));
+    for (int i = 1; i < TSP_N_STEP_EVENTS; ++i)
+      if ((rc = record(ev, i, stream))) return rc;
+    return TSP_OK;
+  }
+  __half* xn2 = reinterpret_cast<__half*>(base + b.xn2);
+  __half* u = reinterpret_cast<__half*>(base + b.u);
+  __nv_bfloat16* du = reinterpret_cast<__nv_bfloat16*>(base + b.du);
+  float* dxn2 = reinterpret_cast<float*>(base + b.dxn2);
+  __nv_bfloat16* xn2t = reinterpret_cast<__nv_bfloat16*>(base + b.xn2t);
+  __nv_bfloat16* dut = reinterpret_cast<__nv_bfloat16*>(base + b.dut);
+  __nv_bfloat16* ht = reinterpret_cast<__nv_bfloat16*>(base + b.ht);
+  __nv_bfloat16* dyt = reinterpret_cast<__nv_bfloat16*>(base + b.dyt);
+  const int L = static_cast<int>(s.L);
+  // Xn2 = LN2(Y1), U = Xn2 W1 (fp16 shards, as in the forward); the same
+  // epilogue writes GELU(U)^T (bf16 [F, L]) for dW2
+  rc = launch_layernorm<float>(y1, xn2, s.L, s.h, dims->ln_eps, stream);
+  if (rc) return rc;
+  const void* const* w1fam[3] = {reinterpret_cast<const void* const*>(w->w1), nullptr, nullptr};
+  void* uout[3] = {u, nullptr, nullptr};
+  const int noremap[3] = {0, 0, 0};
+  rc = launch_proj(s, 0, xn2, w1fam, uout, noremap, 1, kEpiStoreBf16, s.F, status, stream, ht);
+  if (rc) return rc;
+  if ((rc = record(ev, 1, stream))) return rc;
+  // dU = (dY W2^T) * GELU'(U): B = W2 [F, h] is K-major over h; the
+  // epilogue also writes dU^T (bf16 [F, L]) for dW1
+  rc = launch_plain(dy, L, s.h, s.h, w2_full, s.F, s.h, true, kEpiGeluBwd, du, s.F, u, status, stream, dut, s.L);
+  if (rc) return rc;
+  if ((rc = record(ev, 2, stream))) return rc;
+  // dXn2 = dU W1^T: B = W1 [h, F] is K-major over F
+  rc = launch_plain(du, L, s.F, s.F, w1_full, s.h, s.F, true, kEpiStoreF32, dxn2, s.h, nullptr, status, stream);
+  if (rc) return rc;
+  if ((rc = record(ev, 3, stream))) return rc;
+  // dY1 = dY + LN2'(Y1)^T dXn2
+  rc = launch_ln_backward<float, __nv_bfloat16>(y1, dxn2, dy, dy1, dy1b, s.L, s.h, dims->ln_eps, stream);
+  if (rc) return rc;
+  if ((rc = record(ev, 4, stream))) return rc;
+  // token-major operands of the weight gradients (reduction over the tokens)
+  if ((rc = launch_transpose<__half>(xn2, s.L, s.h, xn2t, stream))) return rc;
+  if ((rc = launch_transpose<__nv_bfloat16>(dy, s.L, s.h, dyt, stream))) return rc;
+  if ((rc = record(ev, 5, stream))) return rc;
+  // dW1 [h, F] = Xn2^T dU ; dW2 [F, h] = GELU(U)^T dY
+  rc = launch_plain(xn2t, s.h, L, L, dut, s.F, L, true, kEpiStoreF32, dw1, s.F, nullptr, status, stream);
+  if (rc) return rc;
+  if ((rc = record(ev, 6, stream))) return rc;
+  rc = launch_plain(ht, s.F, L, L, dyt, s.h, L, true, kEpiStoreF32, dw2, s.h, nullptr, status, stream);
+  if (rc) return rc;
+  return record(ev, 7, stream);
+}
+
+// Workspace of tsp_layer_backward: the MLP half's (its status section first),
+// then the attention half's operands.
+struct LayerBwdLayout {
+  BwdLayout mlp;
+  size_t dy1, dy1b, dy1t, at, d_o, dq, dqb, dqt, xn1, xn1t, dxn1, counters, delta, total;
+};
+
+LayerBwdLayout lbwd_layout(const Sizes& s) {
+  LayerBwdLayout l;
+  l.mlp = bwd_layout(s);
+  const size_t Lh = static_cast<size_t>(s.L) * s.h;
+  size_t o = l.mlp.total;
+  l.dy1 = o; o += align_up(Lh * 4);
+  l.dy1b = o; o += align_up(Lh * 2);
+  l.dy1t = o; o += align_up(Lh * 2);
+  l.at = o; o += align_up(Lh * 2);
+  l.d_o = o; o += align_up(Lh * 2);
+  l.dq = o; o += align_up(Lh * 4);
+  l.dqb = o; o += align_up(Lh * 2);
+  l.dqt = o; o += align_up(Lh * 2);
+  l.xn1 = o; o += align_up(Lh * 2);
+  l.xn1t = o; o += align_up(Lh * 2);
+  l.dxn1 = o; o += align_up(Lh * 4);
+  l.counters = o; o += align_up(256);
+  l.delta = o; o += align_up(stash_bytes(s));
+  l.total = o;
+  return l;
+}
+
+// Workspace of tsp_kv_backward.
+struct KvBwdLayout {
+  size_t status, xn1, xn1t, kv, kvt, dxn, total;
+};
+
+KvBwdLayout kvbwd_layout(const Sizes& s) {
+  KvBwdLayout k;
+  const size_t Lh = static_cast<size_t>(s.L) * s.h;
+  size_t o = 0;
+  k.status = o; o += align_up(256);
+  k.xn1 = o; o += align_up(Lh * 2);
+  k.xn1t = o; o += align_up(Lh * 2);
+  k.kv = o; o += align_up(Lh * 4);
+  k.kvt = o; o += align_up(Lh * 4);
+  k.dxn = o; o += align_up(Lh * 4);
+  k.total = o;
+  return k;
+}
+
+// dXn [L, h] = [dK | dV] [Wk ; Wv]^T: A = [dK | dV] bf16 [L, 2h]; the K loop
+// walks Wk (row-major [h_in, h_out]: K-major over h_out) for its first h
+// columns and Wv for the next h; fp32 out.
+int launch_kv_grad_input(const __nv_bfloat16* kv, int L, int h, const void* wk, const void* wv, float* out,
+                         int* status, cudaStream_t st) {
+  static thread_local GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  const int bn = pick_bn(h);
+  int rc = make_map(&p.map_a, kv, L, 2 * h, 2 * h, kGemmBM, true);
+  if (rc) return rc;
+  if ((rc = make_map(&p.map_b[0], wk, h, h, h, b_box_rows(bn), true))) return rc;
+  if ((rc = make_map(&p.map_b[1], wv, h, h, h, b_box_rows(bn), true))) return rc;
+  p.M = L;
+  p.N = h;
+  p.K = 2 * h;
+  p.ksplit = 1;
+  p.shard_n = h;
+  p.shard_k = h;
+  p.seg_n = h;
+  p.epi = kEpiStoreF32;
+  p.fmt_bf16 = 1;
+  p.out[0] = out;
+  p.ldo = h;
+  p.status = status;
+  p.timeout_ns = kDefaultTimeoutNs;
+  return launch_gemm(p, bn, st);
 }
 
 // ---------------------------------------------------------------- allocation-free K/V projection
@@ -993,66 +1146,175 @@ int tsp_mlp_backward(const tsp_dims* dims, const tsp_weights* w, const void* w1_
   for (int i = 0; i < (s.L == 0 ? 4 : 7); ++i)
     if (!ptrs[i] || !aligned16(ptrs[i])) return TSP_ERR_INVALID_ARG;
   if (!bws || (reinterpret_cast<uintptr_t>(bws) & 255)) return TSP_ERR_INVALID_ARG;
-  // whole 256-column tiles, and whole 128-row tiles of tokens (the
-  // transposed epilogue stores need every lane of a warp)
-  if (s.h % 256 || s.F % 256 || s.L % 128) return TSP_ERR_UNSUPPORTED;
+  if ((rc = check_backward_shape(s))) return rc;
   const BwdLayout b = bwd_layout(s);
   if (bws_bytes < b.total) return TSP_ERR_WORKSPACE;
-  uint8_t* base = static_cast<uint8_t*>(bws);
-  int* status = reinterpret_cast<int*>(base + b.status);
+  return mlp_backward_core(s, dims, w, w1_full, w2_full, static_cast<const float*>(y1),
+                           static_cast<const __nv_bfloat16*>(dy), static_cast<float*>(dy1), nullptr,
+                           static_cast<float*>(dw1), static_cast<float*>(dw2), static_cast<uint8_t*>(bws), b, stream,
+                           ev);
+}
+
+size_t tsp_layer_backward_workspace_bytes(const tsp_dims* dims, int D) {
+  if (check_dims(dims, D) != TSP_OK) return 0;
+  return lbwd_layout(sizes_of(dims, D)).total;
+}
+
+size_t tsp_kv_backward_workspace_bytes(const tsp_dims* dims, int D) {
+  if (check_dims(dims, D) != TSP_OK) return 0;
+  return kvbwd_layout(sizes_of(dims, D)).total;
+}
+
+int tsp_layer_backward(const tsp_dims* dims, const tsp_weights* w, const void* const w_full[6], int rank,
+                       const void* x_local, const void* fwd_ws, size_t fwd_ws_bytes, const void* k_full,
+                       const void* v_full, const void* dy, void* dx, void* dwq, void* dwo, void* dw1, void* dw2,
+                       void* dk_full, void* dv_full, void* bws, size_t bws_bytes, cudaStream_t stream,
+                       cudaEvent_t* ev) {
+  const int D = w ? w->D : 0;
+  int rc = check_dims(dims, D);
+  if (rc) return rc;
+  if ((rc = check_weights(w, D))) return rc;
+  if (rank < 0 || rank >= D || !w_full) return TSP_ERR_INVALID_ARG;
+  const Sizes s = sizes_of(dims, D);
+  for (int i = 0; i < 6; ++i)
+    if (!w_full[i] || !aligned16(w_full[i])) return TSP_ERR_INVALID_ARG;
+  const void* ptrs[11] = {dwq, dwo, dw1, dw2, x_local, fwd_ws, k_full, v_full, dy, dx, dk_full};
+  for (int i = 0; i < (s.L == 0 ? 4 : 11); ++i)
+    if (!ptrs[i] || !aligned16(ptrs[i])) return TSP_ERR_INVALID_ARG;
+  if (s.L > 0 && (!dv_full || !aligned16(dv_full))) return TSP_ERR_INVALID_ARG;
+  if (!bws || (reinterpret_cast<uintptr_t>(bws) & 255)) return TSP_ERR_INVALID_ARG;
+  if ((rc = check_backward_shape(s))) return rc;
+  const LayerBwdLayout lb = lbwd_layout(s);
+  if (bws_bytes < lb.total) return TSP_ERR_WORKSPACE;
+  const WsLayout fl = ws_layout(s);
+  if (s.L > 0 && fwd_ws_bytes < fl.total) return TSP_ERR_WORKSPACE;
+  const size_t hh = static_cast<size_t>(s.h) * s.h * 4;
   if ((rc = record(ev, 0, stream))) return rc;
   if (s.L == 0) {  // no tokens: zero weight gradients
+    TSP_CUDA(cudaMemsetAsync(dwq, 0, hh, stream));
+    TSP_CUDA(cudaMemsetAsync(dwo, 0, hh, stream));
     TSP_CUDA(cudaMemsetAsync(dw1, 0, static_cast<size_t>(s.h) * s.F * 4, stream));
     TSP_CUDA(cudaMemsetAsync(dw2, 0, static_cast<size_t>(s.F) * s.h * 4, stream));
     for (int i = 1; i < TSP_N_STEP_EVENTS; ++i)
       if ((rc = record(ev, i, stream))) return rc;
     return TSP_OK;
   }
-  __half* xn2 = reinterpret_cast<__half*>(base + b.xn2);
-  __half* u = reinterpret_cast<__half*>(base + b.u);
-  __nv_bfloat16* du = reinterpret_cast<__nv_bfloat16*>(base + b.du);
-  float* dxn2 = reinterpret_cast<float*>(base + b.dxn2);
-  __nv_bfloat16* xn2t = reinterpret_cast<__nv_bfloat16*>(base + b.xn2t);
-  __nv_bfloat16* dut = reinterpret_cast<__nv_bfloat16*>(base + b.dut);
-  __nv_bfloat16* ht = reinterpret_cast<__nv_bfloat16*>(base + b.ht);
-  __nv_bfloat16* dyt = reinterpret_cast<__nv_bfloat16*>(base + b.dyt);
+  uint8_t* base = static_cast<uint8_t*>(bws);
+  int* status = reinterpret_cast<int*>(base + lb.mlp.status);
+  const uint8_t* fws = static_cast<const uint8_t*>(fwd_ws);
+  const __half* q = reinterpret_cast<const __half*>(fws + fl.q);
+  const __half* a = reinterpret_cast<const __half*>(fws + fl.a);
+  const float* y1 = reinterpret_cast<const float*>(fws + fl.y1);
+  const float* lse = reinterpret_cast<const float*>(fws + fl.lse);
+  float* dy1 = reinterpret_cast<float*>(base + lb.dy1);
+  __nv_bfloat16* dy1b = reinterpret_cast<__nv_bfloat16*>(base + lb.dy1b);
+  __nv_bfloat16* dy1t = reinterpret_cast<__nv_bfloat16*>(base + lb.dy1t);
+  __nv_bfloat16* at = reinterpret_cast<__nv_bfloat16*>(base + lb.at);
+  __half* d_o = reinterpret_cast<__half*>(base + lb.d_o);
+  float* dq = reinterpret_cast<float*>(base + lb.dq);
+  __nv_bfloat16* dqb = reinterpret_cast<__nv_bfloat16*>(base + lb.dqb);
+  __nv_bfloat16* dqt = reinterpret_cast<__nv_bfloat16*>(base + lb.dqt);
+  __half* xn1 = reinterpret_cast<__half*>(base + lb.xn1);
+  __nv_bfloat16* xn1t = reinterpret_cast<__nv_bfloat16*>(base + lb.xn1t);
+  float* dxn1 = reinterpret_cast<float*>(base + lb.dxn1);
   const int L = static_cast<int>(s.L);
-  // Xn2 = LN2(Y1), U = Xn2 W1 (fp16 shards, as in the forward); the same
-  // epilogue writes GELU(U)^T (bf16 [F, L]) for dW2
-  rc = launch_layernorm<float>(static_cast<const float*>(y1), xn2, s.L, s.h, dims->ln_eps, stream);
-  if (rc) return rc;
-  const void* const* w1fam[3] = {reinterpret_cast<const void* const*>(w->w1), nullptr, nullptr};
-  void* uout[3] = {u, nullptr, nullptr};
-  const int noremap[3] = {0, 0, 0};
-  rc = launch_proj(s, 0, xn2, w1fam, uout, noremap, 1, kEpiStoreBf16, s.F, status, stream, ht);
+  // MLP half: dY1 (and its bf16 copy), dW1, dW2
+  rc = mlp_backward_core(s, dims, w, w_full[4], w_full[5], y1, static_cast<const __nv_bfloat16*>(dy), dy1, dy1b,
+                         static_cast<float*>(dw1), static_cast<float*>(dw2), base, lb.mlp, stream, nullptr);
   if (rc) return rc;
   if ((rc = record(ev, 1, stream))) return rc;
-  // dU = (dY W2^T) * GELU'(U): B = W2 [F, h] is K-major over h; the
-  // epilogue also writes dU^T (bf16 [F, L]) for dW1
-  rc = launch_plain(dy, L, s.h, s.h, w2_full, s.F, s.h, true, kEpiGeluBwd, du, s.F, u, status, stream, dut, s.L);
+  // dA = dY1 Wo^T (Wo [h_in, h_out] row-major is K-major over h_out), fp16 for
+  // the attention backward's tensor cores
+  rc = launch_plain(dy1b, L, s.h, s.h, w_full[3], s.h, s.h, true, kEpiStoreBf16, d_o, s.h, nullptr, status, stream);
   if (rc) return rc;
   if ((rc = record(ev, 2, stream))) return rc;
-  // dXn2 = dU W1^T: B = W1 [h, F] is K-major over F
-  rc = launch_plain(du, L, s.F, s.F, w1_full, s.h, s.F, true, kEpiStoreF32, dxn2, s.h, nullptr, status, stream);
+  // dWo = A^T dY1: both operands token-major
+  if ((rc = launch_transpose<__half>(a, s.L, s.h, at, stream))) return rc;
+  if ((rc = launch_transpose<float>(dy1, s.L, s.h, dy1t, stream))) return rc;
+  rc = launch_plain(at, s.h, L, L, dy1t, s.h, L, true, kEpiStoreF32, dwo, s.h, nullptr, status, stream);
   if (rc) return rc;
   if ((rc = record(ev, 3, stream))) return rc;
-  // dY1 = dY + LN2'(Y1)^T dXn2
-  rc = launch_ln_backward(static_cast<const float*>(y1), dxn2, static_cast<const __nv_bfloat16*>(dy),
-                          static_cast<float*>(dy1), s.L, s.h, dims->ln_eps, stream);
+  // the attention: dQ, and this rank's dK, dV for all keys
+  rc = launch_attn_backward(s, rank, dims, q, k_full, v_full, a, lse, d_o, dq, static_cast<float*>(dk_full),
+                            static_cast<float*>(dv_full), reinterpret_cast<float*>(base + lb.delta),
+                            reinterpret_cast<int*>(base + lb.counters), status, stream);
   if (rc) return rc;
   if ((rc = record(ev, 4, stream))) return rc;
-  // token-major operands of the weight gradients (reduction over the tokens)
-  if ((rc = launch_transpose<__half>(xn2, s.L, s.h, xn2t, stream))) return rc;
-  if ((rc = launch_transpose<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(dy), s.L, s.h, dyt, stream)))
-    return rc;
+  // bf16 copies of dQ (row-major and token-major), LN1(x) recomputed
+  if ((rc = launch_convert_bf16(dq, dqb, static_cast<int64_t>(s.L) * s.h, stream))) return rc;
+  if ((rc = launch_transpose<float>(dq, s.L, s.h, dqt, stream))) return rc;
+  rc = launch_layernorm<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x_local), xn1, s.L, s.h, dims->ln_eps, stream);
+  if (rc) return rc;
+  if ((rc = launch_transpose<__half>(xn1, s.L, s.h, xn1t, stream))) return rc;
   if ((rc = record(ev, 5, stream))) return rc;
-  // dW1 [h, F] = Xn2^T dU ; dW2 [F, h] = GELU(U)^T dY
-  rc = launch_plain(xn2t, s.h, L, L, dut, s.F, L, true, kEpiStoreF32, dw1, s.F, nullptr, status, stream);
+  // dWq = LN1(X)^T dQ
+  rc = launch_plain(xn1t, s.h, L, L, dqt, s.h, L, true, kEpiStoreF32, dwq, s.h, nullptr, status, stream);
   if (rc) return rc;
   if ((rc = record(ev, 6, stream))) return rc;
-  rc = launch_plain(ht, s.F, L, L, dyt, s.h, L, true, kEpiStoreF32, dw2, s.h, nullptr, status, stream);
+  // dX = dY1 + LN1'(X)^T (dQ Wq^T)   (Wq [h_in, h_out] is K-major over h_out)
+  rc = launch_plain(dqb, L, s.h, s.h, w_full[0], s.h, s.h, true, kEpiStoreF32, dxn1, s.h, nullptr, status, stream);
+  if (rc) return rc;
+  rc = launch_ln_backward<__nv_bfloat16, float>(static_cast<const __nv_bfloat16*>(x_local), dxn1, dy1,
+                                                static_cast<float*>(dx), nullptr, s.L, s.h, dims->ln_eps, stream);
   if (rc) return rc;
   return record(ev, 7, stream);
+}
+
+int tsp_kv_backward(const tsp_dims* dims, int D, const void* const w_full[6], int rank, const void* x_local,
+                    const void* dk_full, const void* dv_full, void* dx, void* dwk, void* dwv, void* kws,
+                    size_t kws_bytes, cudaStream_t stream) {
+  int rc = check_dims(dims, D);
+  if (rc) return rc;
+  if (rank < 0 || rank >= D || !w_full) return TSP_ERR_INVALID_ARG;
+  const Sizes s = sizes_of(dims, D);
+  if (!w_full[1] || !w_full[2] || !aligned16(w_full[1]) || !aligned16(w_full[2])) return TSP_ERR_INVALID_ARG;
+  const void* ptrs[7] = {dwk, dwv, x_local, dk_full, dv_full, dx, nullptr};
+  for (int i = 0; i < (s.L == 0 ? 2 : 6); ++i)
+    if (!ptrs[i] || !aligned16(ptrs[i])) return TSP_ERR_INVALID_ARG;
+  if (!kws || (reinterpret_cast<uintptr_t>(kws) & 255)) return TSP_ERR_INVALID_ARG;
+  if ((rc = check_backward_shape(s))) return rc;
+  const KvBwdLayout kb = kvbwd_layout(s);
+  if (kws_bytes < kb.total) return TSP_ERR_WORKSPACE;
+  const size_t hh = static_cast<size_t>(s.h) * s.h * 4;
+  if (s.L == 0) {
+    TSP_CUDA(cudaMemsetAsync(dwk, 0, hh, stream));
+    TSP_CUDA(cudaMemsetAsync(dwv, 0, hh, stream));
+    return TSP_OK;
+  }
+  uint8_t* base = static_cast<uint8_t*>(kws);
+  int* status = reinterpret_cast<int*>(base + kb.status);
+  __half* xn1 = reinterpret_cast<__half*>(base + kb.xn1);
+  __nv_bfloat16* xn1t = reinterpret_cast<__nv_bfloat16*>(base + kb.xn1t);
+  __nv_bfloat16* kv = reinterpret_cast<__nv_bfloat16*>(base + kb.kv);
+  __nv_bfloat16* kvt = reinterpret_cast<__nv_bfloat16*>(base + kb.kvt);
+  float* dxn = reinterpret_cast<float*>(base + kb.dxn);
+  const int L = static_cast<int>(s.L);
+  // the rank's rows of the summed dK, dV: [dK | dV] bf16 [L, 2h], and
+  // token-major [2h, L]
+  {
+    const int64_t threads = s.L * (2 * s.h / 8);
+    gather_kv_grad_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
+        static_cast<const float*>(dk_full), static_cast<const float*>(dv_full), kv, s.L, s.h, s.c,
+        static_cast<int64_t>(rank) * s.c, static_cast<int64_t>(2 * s.D - 1 - rank) * s.c - s.c);
+    TSP_CUDA(cudaGetLastError());
+  }
+  if ((rc = launch_transpose<__nv_bfloat16>(kv, s.L, 2 * s.h, kvt, stream))) return rc;
+  rc = launch_layernorm<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x_local), xn1, s.L, s.h, dims->ln_eps, stream);
+  if (rc) return rc;
+  if ((rc = launch_transpose<__half>(xn1, s.L, s.h, xn1t, stream))) return rc;
+  // dWk = LN1(X)^T dK, dWv = LN1(X)^T dV
+  rc = launch_plain(xn1t, s.h, L, L, kvt, s.h, L, true, kEpiStoreF32, dwk, s.h, nullptr, status, stream);
+  if (rc) return rc;
+  rc = launch_plain(xn1t, s.h, L, L, kvt + static_cast<size_t>(s.h) * s.L, s.h, L, true, kEpiStoreF32, dwv, s.h,
+                    nullptr, status, stream);
+  if (rc) return rc;
+  // dXn = dK Wk^T + dV Wv^T: one K-split product over [dK | dV] with the two
+  // weights as its two K blocks; then dX += LN1'(X)^T dXn
+  rc = launch_kv_grad_input(kv, L, s.h, w_full[1], w_full[2], dxn, status, stream);
+  if (rc) return rc;
+  return launch_ln_backward<__nv_bfloat16, float>(static_cast<const __nv_bfloat16*>(x_local), dxn,
+                                                  static_cast<const float*>(dx), static_cast<float*>(dx), nullptr,
+                                                  s.L, s.h, dims->ln_eps, stream);
 }
 
 int tsp_selftest_wait_timeout(void* ws, uint64_t timeout_ns, cudaStream_t stream) {

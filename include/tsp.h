@@ -328,6 +328,63 @@ int tsp_mlp_backward(const tsp_dims* dims, const tsp_weights* w,
                      void* bws, size_t bws_bytes, cudaStream_t stream,
                      cudaEvent_t* step_events);
 
+/* Workspace bytes of tsp_layer_backward at this D (the MLP half's sections,
+ * its status section first, then the attention half's); 0 on a bad
+ * argument. */
+size_t tsp_layer_backward_workspace_bytes(const tsp_dims* dims, int D);
+
+/* One rank's share of the whole layer's backward [zubnet.ai TSP item,
+ * paragraph 1: the validated workload is training; paragraph 2: the
+ * attention shards are applied to the rank's own tokens against the
+ * all-gathered K/V, and the MLP shards' contributions are summed locally].
+ * The chain rule through the forward (the pages give none), for the rank's
+ * rows and the loss gradient dY of its output:
+ *   the MLP half as tsp_mlp_backward: dY1, dW1, dW2;
+ *   dA = dY1 Wo^T (fp16),  dWo = A^T dY1;
+ *   the attention as tsp_attn_backward: dQ, and dK, dV for every key;
+ *   dWq = LN1(X)^T dQ,  dX = dY1 + LN1'(X)^T (dQ Wq^T).
+ * What the key owners add after the dK/dV reduce-scatter (LN1'^T (dK Wk^T +
+ * dV Wv^T), dWk, dWv) is tsp_kv_backward.  Inputs: w (fp16 shards, for the
+ * recomputed U) and w_full = {Wq, Wk, Wv, Wo, W1, W2} bf16 in the math
+ * orientation [in, out] (operands of the gradient products, bf16 as in
+ * tsp_mlp_backward); x_local bf16 [T/D, h]; fwd_ws: the workspace of this
+ * rank's tsp_layer_forward or tsp_rank_step (same dims, D and rank; read:
+ * Q, A, Y1 and the log-sum-exp stash); k_full, v_full fp16 [T, h] as in that
+ * forward; dy bf16 [T/D, h].  Outputs: dx fp32 [T/D, h] (overwritten);
+ * dwq, dwo fp32 [h, h], dw1 fp32 [h, F], dw2 fp32 [F, h]: this rank's
+ * contributions summed over its tokens (overwritten); dk_full, dv_full fp32
+ * [T, h] natural order, ADDED to (see tsp_attn_backward).  Same shape limits
+ * as tsp_mlp_backward.  bws: tsp_layer_backward_workspace_bytes bytes,
+ * 256-byte aligned; its status section (read by tsp_get_device_status) is at
+ * its start.  step_events: NULL, or TSP_N_STEP_EVENTS events recorded before
+ * the first launch and after the MLP half, dA, dWo, the attention, the dQ
+ * and LN1 preparations, dWq, and dX. */
+int tsp_layer_backward(const tsp_dims* dims, const tsp_weights* w, const void* const w_full[6], int rank,
+                       const void* x_local, const void* fwd_ws, size_t fwd_ws_bytes, const void* k_full,
+                       const void* v_full, const void* dy, void* dx, void* dwq, void* dwo, void* dw1, void* dw2,
+                       void* dk_full, void* dv_full, void* bws, size_t bws_bytes, cudaStream_t stream,
+                       cudaEvent_t* step_events);
+
+/* Workspace bytes of tsp_kv_backward at this D; 0 on a bad argument. */
+size_t tsp_kv_backward_workspace_bytes(const tsp_dims* dims, int D);
+
+/* The key owner's part of the layer's backward, once dK and dV of the whole
+ * sequence have been summed over the ranks [zubnet.ai TSP item, paragraph 2:
+ * K/V were all-gathered with the zigzag partition, so their gradients are
+ * reduce-scattered back to the ranks that own those tokens]: for rank
+ * `rank`'s own tokens at global positions pos(i),
+ *   dX[i] += LN1'(X_i)^T (dK[pos(i)] Wk^T + dV[pos(i)] Wv^T),
+ *   dWk = LN1(X)^T dK[pos],  dWv = LN1(X)^T dV[pos]  (this rank's tokens).
+ * w_full as in tsp_layer_backward (Wk, Wv read); x_local bf16 [T/D, h];
+ * dk_full, dv_full fp32 [T, h] (read; each rank reads only its own rows);
+ * dx fp32 [T/D, h] added to (tsp_layer_backward's output); dwk, dwv fp32
+ * [h, h] overwritten.  dK and dV enter their products as bf16.  kws:
+ * tsp_kv_backward_workspace_bytes bytes, 256-byte aligned, status section
+ * first. */
+int tsp_kv_backward(const tsp_dims* dims, int D, const void* const w_full[6], int rank, const void* x_local,
+                    const void* dk_full, const void* dv_full, void* dx, void* dwk, void* dwv, void* kws,
+                    size_t kws_bytes, cudaStream_t stream);
+
 /* Fault-detection self test: launches one block that waits on a barrier
  * nothing will ever complete, with a limit of `timeout_ns` nanoseconds
  * (at most 2e9).  The wait gives up, the kernel records TSP_ERR_TIMEOUT in
