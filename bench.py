@@ -605,6 +605,91 @@ def run_sweep_mlp_bwd(args):
     print(json.dumps(line), flush=True)
 
 
+LBWD_NAMES = ["mlp_half", "d_a", "d_wo", "attention", "prep_dq_ln1", "d_wq", "d_x"]
+
+
+def run_sweep_layer_bwd(args):
+    """The whole layer's backward for rank 0 (T and D from --workload; 128K,
+    D = 8 by default): the rank's forward (tsp_rank_step, which stashes Q, A,
+    Y1 and the attention's log-sum-exp), then tsp_layer_backward (MLP half,
+    dA, dWo, the attention backward, dWq, dX) and tsp_kv_backward (the key
+    owner's dWk, dWv and dX terms).  Only the backward is timed.  The
+    attention backward's algorithmic work is five products per causal
+    (query, key) pair and head dim (S, dP, dV, dK, dQ): 10 h pairs FLOPs."""
+    import torch
+    from folded_tensor_sequence_rank_b200 import tsp
+    wl = WORKLOADS[args.workload]
+    T, h, H, F, D = wl["T"], wl["h"], wl["H"], wl["F"], wl["D"]
+    L = T // D
+    torch.cuda.set_device(0)
+    dims = tsp.make_dims(T, h, H, F)
+    rnd, w_full = _synthetic(T, h, F, 6)
+    sw = tsp.pack_shards(dims, D, w_full)
+    kv_std = 0.02 * math.sqrt(h)
+    x = rnd(L, h)
+    K = rnd(T, h, std=kv_std, dtype=torch.float16)
+    V = rnd(T, h, std=kv_std, dtype=torch.float16)
+    y = torch.empty(L, h, dtype=torch.bfloat16, device="cuda")
+    ws = tsp.alloc_workspace(dims, D)
+    tsp.rank_step(dims, sw, 0, x, K, V, y, ws)
+    dy = rnd(L, h)
+    dx = torch.empty(L, h, dtype=torch.float32, device="cuda")
+    g = {"wq": torch.empty(h, h, device="cuda"), "wo": torch.empty(h, h, device="cuda"),
+         "w1": torch.empty(h, F, device="cuda"), "w2": torch.empty(F, h, device="cuda")}
+    dwk = torch.empty(h, h, device="cuda")
+    dwv = torch.empty(h, h, device="cuda")
+    dK = torch.zeros(T, h, dtype=torch.float32, device="cuda")
+    dV = torch.zeros_like(dK)
+    bws = tsp.alloc_layer_backward_workspace(dims, D)
+    kws = tsp.alloc_kv_backward_workspace(dims, D)
+
+    def step(events=None, kv_ev=None):
+        tsp.layer_backward(dims, sw, w_full, 0, x, ws, K, V, dy, dx, g, dK, dV, bws, events=events)
+        tsp.kv_backward(dims, D, w_full, 0, x, dK, dV, dx, dwk, dwv, kws)
+        if kv_ev is not None:
+            kv_ev.record()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert tsp.get_device_status(bws) == tsp.TSP_OK, "device wait timed out during warm-up"
+    steps = max(1, min(args.steps, 10))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(tsp.N_STEP_EVENTS)] for _ in range(steps)]
+    kvs = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    clocks = ClockSampler(0)
+    time.sleep(0.3)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(steps):
+        step(evs[i], kvs[i])
+    t1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    assert tsp.get_device_status(bws) == tsp.TSP_OK and tsp.get_device_status(kws) == tsp.TSP_OK
+    ms = t0.elapsed_time(t1) / steps
+    part = {n: statistics.median(e[j].elapsed_time(e[j + 1]) for e in evs) for j, n in enumerate(LBWD_NAMES)}
+    part["kv_backward"] = statistics.median(evs[i][7].elapsed_time(kvs[i]) for i in range(steps))
+    fl = rank_flops(T, h, F, D, 0)
+    attn_bwd_fl = 2.5 * fl["attention"]
+    gemm_fl = 5 * 2.0 * L * h * F + 4 * 2.0 * L * h * h + 4 * 2.0 * L * h * h  # MLP; dA, dWo, dWq, dXn1; kv: dWk, dWv, dXn (2h)
+    pk, src = peaks()
+    attn_tf = attn_bwd_fl / (part["attention"] * 1e-3) / 1e12
+    line = {"metric": f"TSP layer backward tokens/s on 1 B200 (7B layer, T={T}, D={D}, rank 0)",
+            "value": L / (ms * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "dtype": "fp16/bf16", "data": "synthetic",
+            "config": {"workload": f"backward of one TSP rank of the 7B layer, T={T}, D={D}, rank 0: {L} tokens; "
+                                   f"layer backward + key-owner K/V backward (seed 6)",
+                       "l2": "inputs larger than L2; no flush"},
+            "tflop_per_step": (attn_bwd_fl + gemm_fl) / 1e12,
+            "tflops": (attn_bwd_fl + gemm_fl) / (ms * 1e-3) / 1e12,
+            "roofline": {"bound": "tensor", "kernel": "attn_bwd_tcgen05<128>", "achieved": attn_tf,
+                         "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                         "frac": attn_tf / pk["bf16_tflops_sustained"],
+                         "peak_source": f"{src} bf16_tflops_sustained",
+                         "algorithmic_per_launch": f"{attn_bwd_fl:.4e} FLOP = 10 h x causal pairs"},
+            "part_ms": {k: round(v, 4) for k, v in part.items()}, "clocks": clk}
+    print(json.dumps(line), flush=True)
+
+
 def run_sweep_stack(args):
     """A 32-layer stack of the 7B layer at T = 131072 on one GPU, all D = 8
     ranks in turn per layer (K/V projections, then layer forwards), random
@@ -665,10 +750,11 @@ def main():
     ap.add_argument("--impl", default="tsp", choices=["tsp", "reference"])
     ap.add_argument("--workload", default="7b-128k-d8", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--sweep", choices=["ranks", "shards", "stack", "mlp_bwd"], default=None,
+    ap.add_argument("--sweep", choices=["ranks", "shards", "stack", "mlp_bwd", "layer_bwd"], default=None,
                     help="ranks: all 8 ranks of the 128K layer in turn (per-rank spread, whole-layer tokens/s); "
                          "shards: rank 0 at T=32768 for D=1..16; stack: a 32-layer forward at 128K; "
-                         "mlp_bwd: the MLP-half backward of rank 0 at 128K")
+                         "mlp_bwd: the MLP-half backward of rank 0 at 128K; "
+                         "layer_bwd: the whole layer's backward of rank 0 at 128K")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -679,6 +765,8 @@ def main():
         run_sweep_shards(args)
     elif args.sweep == "mlp_bwd":
         run_sweep_mlp_bwd(args)
+    elif args.sweep == "layer_bwd":
+        run_sweep_layer_bwd(args)
     elif args.sweep == "stack":
         run_sweep_stack(args)
     elif args.impl == "reference":

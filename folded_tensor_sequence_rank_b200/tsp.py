@@ -81,6 +81,11 @@ def lib() -> ctypes.CDLL:
         "tsp_selftest_wait_timeout": (i32, [vp, ctypes.c_uint64, vp]),
         "tsp_attn_backward_workspace_bytes": (sz, [pd, i32]),
         "tsp_attn_backward": (i32, [pd, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "tsp_layer_backward_workspace_bytes": (sz, [pd, i32]),
+        "tsp_layer_backward": (i32, [pd, pw, ctypes.POINTER(vp), i32, vp, vp, sz, vp, vp, vp, vp, vp, vp, vp, vp,
+                                     vp, vp, vp, sz, vp, ctypes.POINTER(vp)]),
+        "tsp_kv_backward_workspace_bytes": (sz, [pd, i32]),
+        "tsp_kv_backward": (i32, [pd, i32, ctypes.POINTER(vp), i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "tsp_mlp_backward_workspace_bytes": (sz, [pd, i32]),
         "tsp_mlp_backward": (i32, [pd, pw, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, ctypes.POINTER(vp)]),
     }
@@ -318,6 +323,57 @@ def attn_backward(dims: Dims, D: int, rank: int, q, k_full, v_full, o, lse, d_o,
             _ptr(dk_full, "dk_full", torch.float32, (T, h)), _ptr(dv_full, "dv_full", torch.float32, (T, h))]
     _check(lib().tsp_attn_backward(ctypes.byref(dims), D, rank, *args, _ptr(aws, "aws", torch.uint8), aws.numel(),
                                    _stream(stream)), "tsp_attn_backward")
+
+
+def _alloc_ws(fn_name: str, dims: Dims, D: int, device="cuda") -> torch.Tensor:
+    n = getattr(lib(), fn_name)(ctypes.byref(dims), D)
+    if n == 0:
+        _check(check_dims(dims, D) or TSP_ERR_INVALID_ARG, fn_name)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def alloc_layer_backward_workspace(dims: Dims, D: int, device="cuda") -> torch.Tensor:
+    return _alloc_ws("tsp_layer_backward_workspace_bytes", dims, D, device)
+
+
+def alloc_kv_backward_workspace(dims: Dims, D: int, device="cuda") -> torch.Tensor:
+    return _alloc_ws("tsp_kv_backward_workspace_bytes", dims, D, device)
+
+
+def _w_full_ptrs(dims: Dims, w_full: dict):
+    h, F = dims.h, dims.ffn
+    shapes = {"wq": (h, h), "wk": (h, h), "wv": (h, h), "wo": (h, h), "w1": (h, F), "w2": (F, h)}
+    return (ctypes.c_void_p * 6)(*[_ptr(w_full[n], n, torch.bfloat16, shapes[n]) for n in WEIGHT_NAMES])
+
+
+def layer_backward(dims: Dims, w: ShardedWeights, w_full: dict, rank: int, x_local, fwd_ws, k_full, v_full, dy,
+                   dx, grads: dict, dk_full, dv_full, bws, stream=None, events=None):
+    """One rank's share of the layer's backward (see tsp_layer_backward):
+    dx [T/D, h] fp32, grads["wq"|"wo"|"w1"|"w2"] fp32 in the math orientation
+    (overwritten); dk_full, dv_full [T, h] fp32 added to.  fwd_ws is this
+    rank's forward workspace; w_full the bf16 model weights [in, out]."""
+    L, h, F, T = dims.T // w.D, dims.h, dims.ffn, dims.T
+    args = [_ptr(x_local, "x_local", torch.bfloat16, (L, h)), _ptr(fwd_ws, "fwd_ws", torch.uint8), fwd_ws.numel(),
+            _ptr(k_full, "k_full", torch.float16, (T, h)), _ptr(v_full, "v_full", torch.float16, (T, h)),
+            _ptr(dy, "dy", torch.bfloat16, (L, h)), _ptr(dx, "dx", torch.float32, (L, h)),
+            _ptr(grads["wq"], "dwq", torch.float32, (h, h)), _ptr(grads["wo"], "dwo", torch.float32, (h, h)),
+            _ptr(grads["w1"], "dw1", torch.float32, (h, F)), _ptr(grads["w2"], "dw2", torch.float32, (F, h)),
+            _ptr(dk_full, "dk_full", torch.float32, (T, h)), _ptr(dv_full, "dv_full", torch.float32, (T, h))]
+    _check(lib().tsp_layer_backward(ctypes.byref(dims), ctypes.byref(w.struct), _w_full_ptrs(dims, w_full), rank,
+                                    *args, _ptr(bws, "bws", torch.uint8), bws.numel(), _stream(stream),
+                                    _events(events)), "tsp_layer_backward")
+
+
+def kv_backward(dims: Dims, D: int, w_full: dict, rank: int, x_local, dk_full, dv_full, dx, dwk, dwv, kws,
+                stream=None):
+    """The key owner's step after the dK/dV sum (see tsp_kv_backward): dx added
+    to, dwk, dwv [h, h] fp32 overwritten."""
+    L, h, T = dims.T // D, dims.h, dims.T
+    args = [_ptr(x_local, "x_local", torch.bfloat16, (L, h)), _ptr(dk_full, "dk_full", torch.float32, (T, h)),
+            _ptr(dv_full, "dv_full", torch.float32, (T, h)), _ptr(dx, "dx", torch.float32, (L, h)),
+            _ptr(dwk, "dwk", torch.float32, (h, h)), _ptr(dwv, "dwv", torch.float32, (h, h))]
+    _check(lib().tsp_kv_backward(ctypes.byref(dims), D, _w_full_ptrs(dims, w_full), rank, *args,
+                                 _ptr(kws, "kws", torch.uint8), kws.numel(), _stream(stream)), "tsp_kv_backward")
 
 
 def mlp_backward_workspace_bytes(dims: Dims, D: int) -> int:

@@ -520,52 +520,75 @@ def attention_backward_stored(q, k, v, o, q_pos, dout, n_heads: int, scale: floa
 
 
 def rank_layer_backward(rank: int, D: int, x_full, w: dict, dy_local, n_heads: int,
-                        eps: float = LN_EPS, scale: float | None = None) -> dict:
-    """One TSP rank's share of the whole layer's backward, in plain fp64 (no
-    16-bit storage), for the loss gradient dy_local [L, h] of its own output
-    rows (rank-local order).  x_full [T, h] is the sequence in natural order.
+                        eps: float = LN_EPS, scale: float | None = None,
+                        storage=None, grad_storage=None) -> dict:
+    """One TSP rank's share of the whole layer's backward for the loss
+    gradient dy_local [L, h] of its own output rows (rank-local order).
+    x_full [T, h] is the sequence in natural order.
 
     The rank computes, from its own rows and the all-gathered K/V:
       the MLP half (mlp_backward): dY1, and its dW1, dW2 contributions;
-      the attention half: dA = dY1 Wo^T, dWo = A^T dY1, then
-      causal_attention_backward gives dQ for its rows and dK, dV for all T
-      keys; dWq = Xn1^T dQ; dXn1 = dQ Wq^T.
+      the attention half: dA = dY1 Wo^T, dWo = A^T dY1, then the attention
+      backward gives dQ for its rows and dK, dV for all T keys;
+      dWq = Xn1^T dQ; dXn1 = dQ Wq^T; dX = dY1 + LN1'^T dXn1.
     What crosses ranks: "dk_full", "dv_full" (every rank's contributions,
     summed by a reduce-scatter back to the key owners).  After that sum, each
     owner adds LN1'^T (dK Wk^T + dV Wv^T) to its rows' dX and forms dWk, dWv
     (kv_backward_rows).  Weight-gradient entries are this rank's
-    contributions over its tokens; summed over ranks they give the layer's."""
+    contributions over its tokens; summed over ranks they give the layer's.
+
+    Precision: storage=None and grad_storage=None (the defaults) give the
+    plain fp64 chain rule.  Otherwise the forward values are stored as in
+    rank_rows_forward(storage) (the weights, LN outputs, Q, K, V, A, H), the
+    MLP half follows mlp_backward(storage, grad_storage), the attention
+    backward follows attention_backward_stored(storage) with dA stored in
+    `storage`, and the gradient products take their operands rounded to
+    `grad_storage`: dY1 (for dA and dWo), A (for dWo), dQ and LN1(X) (for
+    dWq, dXn1); the bf16 model weights enter those products as given."""
     x_full = np.asarray(x_full, dtype=np.float64)
     T, h = x_full.shape
     if scale is None:
         scale = 1.0 / np.sqrt(h // n_heads)
-    w = {n: np.asarray(a, dtype=np.float64) for n, a in w.items()}
+    rnd, grnd = _rounder(storage), _rounder(grad_storage)
+    w_raw = {n: np.asarray(a, dtype=np.float64) for n, a in w.items()}
+    w16 = _weights(w_raw, rnd, storage)
     pos = zigzag_index(T, D, rank)
     x = x_full[pos]
-    xn_full = layer_norm(x_full, eps)
-    k_full, v_full = xn_full @ w["wk"], xn_full @ w["wv"]
+    xn_full = rnd(layer_norm(x_full, eps))
+    k_full, v_full = rnd(xn_full @ w16["wk"]), rnd(xn_full @ w16["wv"])
     xn1 = xn_full[pos]
-    q = xn1 @ w["wq"]
-    a = causal_attention(q, k_full, v_full, pos, n_heads, scale)
-    y1 = x + a @ w["wo"]
-    mlp = mlp_backward(y1, dy_local, w, eps, storage=None, grad_storage=None)
+    q = rnd(xn1 @ w16["wq"])
+    a = rnd(causal_attention(q, k_full, v_full, pos, n_heads, scale))
+    y1 = x + a @ w16["wo"]
+    mlp = mlp_backward(y1, dy_local, w_raw, eps, storage=storage, grad_storage=grad_storage)
     dy1 = mlp["dy1"]
-    da = dy1 @ w["wo"].T
-    dwo = a.T @ dy1
-    dq, dk_full, dv_full = causal_attention_backward(q, k_full, v_full, pos, da, n_heads, scale)
-    dwq = xn1.T @ dq
-    dx = dy1 + layer_norm_backward(x, dq @ w["wq"].T, eps)
+    dy1_g = grnd(dy1)
+    da = rnd(dy1_g @ w_raw["wo"].T)
+    dwo = grnd(a).T @ dy1_g
+    if storage is None:
+        dq, dk_full, dv_full = causal_attention_backward(q, k_full, v_full, pos, da, n_heads, scale)
+    else:
+        dq, dk_full, dv_full = attention_backward_stored(q, k_full, v_full, a, pos, da, n_heads, scale, storage)
+    dq_g = grnd(dq)
+    dwq = grnd(xn1).T @ dq_g
+    dx = dy1 + layer_norm_backward(x, dq_g @ w_raw["wq"].T, eps)
     return {"dx_partial": dx, "dwq": dwq, "dwo": dwo, "dw1": mlp["dw1"], "dw2": mlp["dw2"],
             "dk_full": dk_full, "dv_full": dv_full}
 
 
-def kv_backward_rows(x_rows, dk_rows, dv_rows, w: dict, eps: float = LN_EPS) -> dict:
+def kv_backward_rows(x_rows, dk_rows, dv_rows, w: dict, eps: float = LN_EPS,
+                     storage=None, grad_storage=None) -> dict:
     """For rows whose keys/values are K = LN1(x) Wk, V = LN1(x) Wv and whose
     summed gradients are dK, dV: the rows' extra input gradient
-    LN1'^T (dK Wk^T + dV Wv^T) and their dWk = LN1(x)^T dK, dWv = LN1(x)^T dV."""
+    LN1'^T (dK Wk^T + dV Wv^T) and their dWk = LN1(x)^T dK, dWv = LN1(x)^T dV.
+    With grad_storage, dK, dV and LN1(x) (itself stored in `storage`) enter
+    the products rounded to grad_storage; the weights as given."""
+    rnd, grnd = _rounder(storage), _rounder(grad_storage)
     x_rows = np.asarray(x_rows, dtype=np.float64)
-    xn = layer_norm(x_rows, eps)
+    xn = grnd(rnd(layer_norm(x_rows, eps)))
+    dk = grnd(np.asarray(dk_rows, dtype=np.float64))
+    dv = grnd(np.asarray(dv_rows, dtype=np.float64))
     wk = np.asarray(w["wk"], dtype=np.float64)
     wv = np.asarray(w["wv"], dtype=np.float64)
-    return {"dx": layer_norm_backward(x_rows, dk_rows @ wk.T + dv_rows @ wv.T, eps),
-            "dwk": xn.T @ dk_rows, "dwv": xn.T @ dv_rows}
+    return {"dx": layer_norm_backward(x_rows, dk @ wk.T + dv @ wv.T, eps),
+            "dwk": xn.T @ dk, "dwv": xn.T @ dv}

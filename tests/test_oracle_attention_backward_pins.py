@@ -123,25 +123,18 @@ def test_planted_softmax_backward_mistake_is_caught(monkeypatch):
         test_attention_backward_matches_torch_autograd()
 
 
-@pytest.mark.parametrize("T,D", [(8, 2), (12, 3)])
-def test_rank_backwards_sum_to_the_whole_layer_gradient(T, D):
-    """The D ranks' shares, with dK, dV summed over ranks (the reduce-scatter)
-    and each owner's K/V backward added, equal torch autograd of the whole
-    unsharded layer (fp64) for every input row and all six weights."""
-    h, H, F = 8, 2, 16
-    rng = np.random.default_rng(11)
-    x = rng.normal(size=(T, h))
-    w = {n: rng.normal(size=s) * 0.3 for n, s in (("wq", (h, h)), ("wk", (h, h)), ("wv", (h, h)), ("wo", (h, h)),
-                                                    ("w1", (h, F)), ("w2", (F, h)))}
-    dy = rng.normal(size=(T, h))
-    s = 1.0 / np.sqrt(h // H)
+def _rank_sum(T, D, x, w, dy, H, s, **prec):
+    """dX and the six weight gradients summed over the D ranks' shares, with
+    dK, dV summed over ranks (the reduce-scatter) and each owner's K/V
+    backward added."""
+    h = x.shape[1]
     dx = np.zeros((T, h))
     grads = {n: np.zeros_like(w[n]) for n in w}
     dk = np.zeros((T, h))
     dv = np.zeros((T, h))
     for r in range(D):
         idx = O.zigzag_index(T, D, r)
-        g = O.rank_layer_backward(r, D, x, w, dy[idx], H, scale=s)
+        g = O.rank_layer_backward(r, D, x, w, dy[idx], H, scale=s, **prec)
         dx[idx] += g["dx_partial"]
         for n in ("wq", "wo", "w1", "w2"):
             grads[n] += g["d" + n]
@@ -149,10 +142,31 @@ def test_rank_backwards_sum_to_the_whole_layer_gradient(T, D):
         dv += g["dv_full"]
     for r in range(D):   # each owner's K/V backward for its own rows
         idx = O.zigzag_index(T, D, r)
-        kv = O.kv_backward_rows(x[idx], dk[idx], dv[idx], w)
+        kv = O.kv_backward_rows(x[idx], dk[idx], dv[idx], w, **prec)
         dx[idx] += kv["dx"]
         grads["wk"] += kv["dwk"]
         grads["wv"] += kv["dwv"]
+    return dx, grads
+
+
+def _small_layer(T, seed=11):
+    h, H, F = 8, 2, 16
+    rng = np.random.default_rng(seed)
+    x = rng.normal(size=(T, h))
+    w = {n: rng.normal(size=s) * 0.3 for n, s in (("wq", (h, h)), ("wk", (h, h)), ("wv", (h, h)), ("wo", (h, h)),
+                                                    ("w1", (h, F)), ("w2", (F, h)))}
+    dy = rng.normal(size=(T, h))
+    return x, w, dy, h, H, F
+
+
+@pytest.mark.parametrize("T,D", [(8, 2), (12, 3)])
+def test_rank_backwards_sum_to_the_whole_layer_gradient(T, D):
+    """The D ranks' shares, with dK, dV summed over ranks (the reduce-scatter)
+    and each owner's K/V backward added, equal torch autograd of the whole
+    unsharded layer (fp64) for every input row and all six weights."""
+    x, w, dy, h, H, F = _small_layer(T)
+    s = 1.0 / np.sqrt(h // H)
+    dx, grads = _rank_sum(T, D, x, w, dy, H, s)
     xt = torch.tensor(x, requires_grad=True)
     wt = {n: torch.tensor(a, requires_grad=True) for n, a in w.items()}
     xn = Fn.layer_norm(xt, (h,), eps=O.LN_EPS)
@@ -165,6 +179,24 @@ def test_rank_backwards_sum_to_the_whole_layer_gradient(T, D):
     np.testing.assert_allclose(dx, xt.grad.numpy(), rtol=1e-9, atol=1e-11)
     for n in w:
         np.testing.assert_allclose(grads[n], wt[n].grad.numpy(), rtol=1e-9, atol=1e-11, err_msg=n)
+
+
+def test_stored_layer_backward_is_the_plain_one_up_to_16_bit_rounding():
+    """With the kernels' precision model (fp16 forward storage and dA, bf16
+    gradient operands) the rank-summed gradients stay within 16-bit rounding
+    of the plain ones (pinned to autograd above), and the rounding really
+    happens.  A transposed operand, a dropped term or a wrong index in the
+    stored branch would move them by O(1)."""
+    T, D = 64, 2
+    x, w, dy, h, H, F = _small_layer(T, seed=12)
+    w = {n: O.round_bf16(a) for n, a in w.items()}   # bf16 model weights
+    s = 1.0 / np.sqrt(h // H)
+    dx0, g0 = _rank_sum(T, D, x, w, dy, H, s)
+    dx1, g1 = _rank_sum(T, D, x, w, dy, H, s, storage="fp16", grad_storage="bf16")
+    rel = lambda a, b: np.linalg.norm(a - b) / np.linalg.norm(b)
+    assert 1e-6 < rel(dx1, dx0) < 2e-2, rel(dx1, dx0)
+    for n in w:
+        assert 1e-6 < rel(g1[n], g0[n]) < 2e-2, (n, rel(g1[n], g0[n]))
 
 
 # --------------------------------------------------------------------------
