@@ -690,6 +690,88 @@ def run_sweep_layer_bwd(args):
     print(json.dumps(line), flush=True)
 
 
+def run_sweep_tp(args):
+    """The tensor-parallel baseline beside TSP at the 7B layer, T = 131072,
+    D = 8 (seed 7), on one GPU.  Measured: one TP rank's compute (its
+    attention and MLP partials over all T tokens with 1/D of the weights), the
+    two all-reduces as sums of the D partials in device memory (the whole
+    job's reduction arithmetic and HBM traffic, not NVLink), and one TSP rank
+    step (the bench's own step) on the same shards.  The all-reduce's
+    communication on 8 GPUs is estimated, not measured: a ring all-reduce
+    moves 2 (D-1)/D of the [T, h] bf16 tensor per rank, at the 725 GB/s bus
+    bandwidth measured on this machine for an 8-rank all-reduce of 1 GiB."""
+    import torch
+    from folded_tensor_sequence_rank_b200 import stack, tp, tsp
+    T, h, H, F, D = 131072, 4096, 32, 16384, 8
+    L = T // D
+    torch.cuda.set_device(0)
+    dims = tsp.make_dims(T, h, H, F)
+    rnd, w_full = _synthetic(T, h, F, 7)
+    sw = tsp.pack_shards(dims, D, w_full)
+    del w_full
+    x = rnd(T, h)
+    tws = tsp.alloc_tp_workspace(dims, D)
+    parts = [torch.empty(T, h, dtype=torch.float32, device="cuda") for _ in range(D)]
+    y1 = torch.empty(T, h, dtype=torch.float32, device="cuda")
+    y = torch.empty(T, h, dtype=torch.bfloat16, device="cuda")
+    # the TSP rank step on the same shards
+    kv_std = 0.02 * math.sqrt(h)
+    K = rnd(T, h, std=kv_std, dtype=torch.float16)
+    V = rnd(T, h, std=kv_std, dtype=torch.float16)
+    xl = rnd(L, h)
+    yl = torch.empty(L, h, dtype=torch.bfloat16, device="cuda")
+    ws = tsp.alloc_workspace(dims, D)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def tp_rank(k):
+        tsp.tp_attention_partial(dims, sw, k, x, parts[k], tws)
+        tsp.tp_mlp_partial(dims, sw, k, y1, parts[k], tws)
+    for _ in range(args.warmup):
+        tp_rank(0)
+        tsp.tp_all_reduce(dims, parts, x, y1)
+        tsp.tp_all_reduce(dims, parts, y1, y)
+        tsp.rank_step(dims, sw, 0, xl, K, V, yl, ws)
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 10))
+    clocks = ClockSampler(0)
+    time.sleep(0.3)
+    rec = {"tp_rank": [], "all_reduce_x2": [], "tsp_rank": []}
+    for _ in range(steps):
+        e = [ev() for _ in range(4)]
+        e[0].record()
+        tp_rank(0)
+        e[1].record()
+        tsp.tp_all_reduce(dims, parts, x, y1)
+        tsp.tp_all_reduce(dims, parts, y1, y)
+        e[2].record()
+        tsp.rank_step(dims, sw, 0, xl, K, V, yl, ws)
+        e[3].record()
+        torch.cuda.synchronize()
+        rec["tp_rank"].append(e[0].elapsed_time(e[1]))
+        rec["all_reduce_x2"].append(e[1].elapsed_time(e[2]))
+        rec["tsp_rank"].append(e[2].elapsed_time(e[3]))
+    clk = clocks.stop()
+    assert tsp.get_device_status(tws) == tsp.TSP_OK and tsp.get_device_status(ws) == tsp.TSP_OK
+    ms = {k: statistics.median(v) for k, v in rec.items()}
+    comm_ms = 2 * (2 * (D - 1) / D * T * h * 2) / 725e9 * 1e3   # two ring all-reduces of bf16 [T, h]
+    tsp_acc = stack.memory_account(dims, D, 1)
+    tp_acc = tp.memory_account(dims, D)
+    line = {"metric": "TP baseline vs TSP, one layer's forward, per GPU (7B layer, 128K, D=8)",
+            "value": ms["tp_rank"] / ms["tsp_rank"], "unit": "TP rank compute time / TSP rank step time",
+            "n_gpus": 1, "steps": steps, "warmup": args.warmup, "higher_is_better": False, "dtype": "fp16",
+            "data": "synthetic",
+            "config": {"workload": "7B dense layer, T=131072, D=8, rank 0 of each scheme, the same shards (seed 7)"},
+            "ms": {k: round(v, 4) for k, v in ms.items()},
+            "tp_all_reduce_comm_ms_estimated": round(comm_ms, 3),
+            "tp_step_ms_with_estimated_comm": round(ms["tp_rank"] + comm_ms, 3),
+            "tokens_per_s_whole_layer": {"tsp": T / (ms["tsp_rank"] * 1e-3),
+                                         "tp_compute_only": T / (ms["tp_rank"] * 1e-3),
+                                         "tp_with_estimated_comm": T / ((ms["tp_rank"] + comm_ms) * 1e-3)},
+            "memory_per_gpu_bytes": {"tsp_one_layer": tsp_acc, "tp_one_layer": tp_acc},
+            "clocks": clk}
+    print(json.dumps(line), flush=True)
+
+
 def run_sweep_stack(args):
     """A 32-layer stack of the 7B layer at T = 131072 on one GPU, all D = 8
     ranks in turn per layer (K/V projections, then layer forwards), random
@@ -750,11 +832,12 @@ def main():
     ap.add_argument("--impl", default="tsp", choices=["tsp", "reference"])
     ap.add_argument("--workload", default="7b-128k-d8", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--sweep", choices=["ranks", "shards", "stack", "mlp_bwd", "layer_bwd"], default=None,
+    ap.add_argument("--sweep", choices=["ranks", "shards", "stack", "mlp_bwd", "layer_bwd", "tp"], default=None,
                     help="ranks: all 8 ranks of the 128K layer in turn (per-rank spread, whole-layer tokens/s); "
                          "shards: rank 0 at T=32768 for D=1..16; stack: a 32-layer forward at 128K; "
                          "mlp_bwd: the MLP-half backward of rank 0 at 128K; "
-                         "layer_bwd: the whole layer's backward of rank 0 at 128K")
+                         "layer_bwd: the whole layer's backward of rank 0 at 128K; "
+                         "tp: the tensor-parallel baseline layer beside a TSP rank step at 128K")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -767,6 +850,8 @@ def main():
         run_sweep_mlp_bwd(args)
     elif args.sweep == "layer_bwd":
         run_sweep_layer_bwd(args)
+    elif args.sweep == "tp":
+        run_sweep_tp(args)
     elif args.sweep == "stack":
         run_sweep_stack(args)
     elif args.impl == "reference":

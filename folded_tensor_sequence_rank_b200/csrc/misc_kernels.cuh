@@ -420,6 +420,32 @@ __global__ void __launch_bounds__(256) gather_kv_grad_kernel(const float* __rest
       make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
 }
 
+// The all-reduce of a tensor-parallel layer, on one GPU: out = resid +
+// sum_k part[k] over the n_parts fp32 partial products [n] (each rank's
+// row-parallel product), with the residual bf16 or fp32 and the output fp32
+// or bf16.  Four values per thread; n a multiple of 4.
+struct PartList {
+  const float* p[16];
+};
+
+template <typename Tr, bool kOutF32>
+__global__ void __launch_bounds__(256) sum_partials_kernel(PartList parts, int n_parts, const Tr* __restrict__ resid,
+                                                           void* __restrict__ out, int64_t n) {
+  const int64_t i = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) * 4;
+  if (i >= n) return;
+  float v[4];
+  load4f<Tr, Tr>(resid + i, v);
+  for (int k = 0; k < n_parts; ++k) {
+    const float4 a = *reinterpret_cast<const float4*>(parts.p[k] + i);
+    v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+  }
+  if (kOutF32)
+    *reinterpret_cast<float4*>(static_cast<float*>(out) + i) = make_float4(v[0], v[1], v[2], v[3]);
+  else
+    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out) + i) =
+        make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+}
+
 // Self test of the bounded waits: one thread waits on a barrier that expects
 // an arrival nobody makes.  The wait gives up after timeout_ns, records the
 // timeout in the status word and the kernel returns normally.

@@ -771,6 +771,43 @@ int launch_kv_grad_input(const __nv_bfloat16* kv, int L, int h, const void* wk, 
   return launch_gemm(p, bn, st);
 }
 
+// ---------------------------------------------------------------- tensor-parallel baseline layer
+// One tensor-parallel rank k of D holds head group k (Wq, Wk, Wv columns, Wo
+// rows) and FFN block k (W1 columns, W2 rows) - the same shards as TSP - but
+// ALL T tokens.  Its workspace: status section, scheduler counters, LN output
+// [T, h] fp16, Q_k, K_k, V_k and A_k [T, h/D] fp16, H_k [T, F/D] fp16.
+struct TpLayout {
+  size_t status, counters, xn, q, k, v, a, hbuf, total;
+};
+
+TpLayout tp_layout(const Sizes& s) {
+  TpLayout t;
+  const size_t Th = static_cast<size_t>(s.T) * s.h, Ths = static_cast<size_t>(s.T) * s.hs;
+  size_t o = 0;
+  t.status = o; o += align_up(256);
+  t.counters = o; o += align_up(256);
+  t.xn = o; o += align_up(Th * 2);
+  t.q = o; o += align_up(Ths * 2);
+  t.k = o; o += align_up(Ths * 2);
+  t.v = o; o += align_up(Ths * 2);
+  t.a = o; o += align_up(Ths * 2);
+  t.hbuf = o; o += align_up(static_cast<size_t>(s.T) * s.Fs * 2);
+  t.total = o;
+  return t;
+}
+
+// The whole sequence as one "rank" (D = 1: chunks 0 and 1 in natural order).
+Sizes whole_sequence(const Sizes& s) {
+  Sizes w = s;
+  w.D = 1;
+  w.c = s.T / 2;
+  w.c_pad = (w.c + 127) / 128 * 128;
+  w.L = s.T;
+  w.hs = s.h;
+  w.Fs = s.F;
+  return w;
+}
+
 // ---------------------------------------------------------------- allocation-free K/V projection
 // Scratch for tsp_kv_project_noalloc: a file-scope device array, so the call
 // needs no device allocation.  Layout: status word (256 B), 768 B spare, then
@@ -1315,6 +1352,115 @@ int tsp_kv_backward(const tsp_dims* dims, int D, const void* const w_full[6], in
   return launch_ln_backward<__nv_bfloat16, float>(static_cast<const __nv_bfloat16*>(x_local), dxn,
                                                   static_cast<const float*>(dx), static_cast<float*>(dx), nullptr,
                                                   s.L, s.h, dims->ln_eps, stream);
+}
+
+size_t tsp_tp_workspace_bytes(const tsp_dims* dims, int D) {
+  if (check_dims(dims, D) != TSP_OK) return 0;
+  return tp_layout(sizes_of(dims, D)).total;
+}
+
+int tsp_tp_attention_partial(const tsp_dims* dims, const tsp_weights* w, int k, const void* x, void* part, void* ws,
+                             size_t ws_bytes, cudaStream_t stream) {
+  const int D = w ? w->D : 0;
+  int rc = check_dims(dims, D);
+  if (rc) return rc;
+  if ((rc = check_weights(w, D))) return rc;
+  if (k < 0 || k >= D) return TSP_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return TSP_ERR_INVALID_ARG;
+  const Sizes s = sizes_of(dims, D);
+  const TpLayout t = tp_layout(s);
+  if (ws_bytes < t.total) return TSP_ERR_WORKSPACE;
+  if (s.T == 0) return TSP_OK;
+  if (!x || !part || !aligned16(x) || !aligned16(part)) return TSP_ERR_INVALID_ARG;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int* status = reinterpret_cast<int*>(base + t.status);
+  __half* xn = reinterpret_cast<__half*>(base + t.xn);
+  __half* q = reinterpret_cast<__half*>(base + t.q);
+  __half* kk = reinterpret_cast<__half*>(base + t.k);
+  __half* v = reinterpret_cast<__half*>(base + t.v);
+  __half* a = reinterpret_cast<__half*>(base + t.a);
+  const Sizes full = whole_sequence(s);
+  // LN1 of every token (each tensor-parallel rank computes it)
+  rc = launch_layernorm<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x), xn, s.T, s.h, dims->ln_eps, stream);
+  if (rc) return rc;
+  // Q_k, K_k, V_k = LN1(X) [Wq_k | Wk_k | Wv_k]: the column-parallel product
+  const void* const* fam[3] = {reinterpret_cast<const void* const*>(&w->wq[k]),
+                               reinterpret_cast<const void* const*>(&w->wk[k]),
+                               reinterpret_cast<const void* const*>(&w->wv[k])};
+  void* out[3] = {q, kk, v};
+  const int noremap[3] = {0, 0, 0};
+  rc = launch_proj(full, 0, xn, fam, out, noremap, 3, kEpiStoreBf16, s.hs, status, stream);
+  if (rc) return rc;
+  // causal attention of head group k over the whole sequence
+  tsp_dims dk = *dims;
+  dk.h = s.hs;
+  dk.n_heads = s.H / D;
+  Sizes sa = full;
+  sa.h = s.hs;
+  sa.H = s.H / D;
+  rc = launch_attention(sa, 0, &dk, q, kk, v, a, nullptr, reinterpret_cast<int*>(base + t.counters), status, stream);
+  if (rc) return rc;
+  // the row-parallel product A_k Wo_k^T: this rank's partial of the sum the
+  // all-reduce forms
+  return launch_plain(a, static_cast<int>(s.T), s.hs, s.hs, w->wo[k], s.h, s.hs, false, kEpiStoreF32, part, s.h,
+                      nullptr, status, stream);
+}
+
+int tsp_tp_mlp_partial(const tsp_dims* dims, const tsp_weights* w, int k, const void* y1, void* part, void* ws,
+                       size_t ws_bytes, cudaStream_t stream) {
+  const int D = w ? w->D : 0;
+  int rc = check_dims(dims, D);
+  if (rc) return rc;
+  if ((rc = check_weights(w, D))) return rc;
+  if (k < 0 || k >= D) return TSP_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return TSP_ERR_INVALID_ARG;
+  const Sizes s = sizes_of(dims, D);
+  const TpLayout t = tp_layout(s);
+  if (ws_bytes < t.total) return TSP_ERR_WORKSPACE;
+  if (s.T == 0) return TSP_OK;
+  if (!y1 || !part || !aligned16(y1) || !aligned16(part)) return TSP_ERR_INVALID_ARG;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int* status = reinterpret_cast<int*>(base + t.status);
+  __half* xn = reinterpret_cast<__half*>(base + t.xn);
+  __half* hb = reinterpret_cast<__half*>(base + t.hbuf);
+  const Sizes full = whole_sequence(s);
+  rc = launch_layernorm<float>(static_cast<const float*>(y1), xn, s.T, s.h, dims->ln_eps, stream);
+  if (rc) return rc;
+  // H_k = GELU(LN2(Y1) W1_k) (column-parallel), then H_k W2_k^T (row-parallel)
+  const void* const* fam[3] = {reinterpret_cast<const void* const*>(&w->w1[k]), nullptr, nullptr};
+  void* out[3] = {hb, nullptr, nullptr};
+  const int noremap[3] = {0, 0, 0};
+  rc = launch_proj(full, 0, xn, fam, out, noremap, 1, kEpiGeluBf16, s.Fs, status, stream);
+  if (rc) return rc;
+  return launch_plain(hb, static_cast<int>(s.T), s.Fs, s.Fs, w->w2[k], s.h, s.Fs, false, kEpiStoreF32, part, s.h,
+                      nullptr, status, stream);
+}
+
+int tsp_tp_all_reduce(const tsp_dims* dims, int n_parts, const void* const parts[], const void* resid, int resid_f32,
+                      void* out, int out_dtype, cudaStream_t stream) {
+  if (!dims || n_parts < 1 || n_parts > TSP_MAX_D || !parts) return TSP_ERR_INVALID_ARG;
+  if (dims->T < 0 || dims->h <= 0 || dims->h % 4) return TSP_ERR_INVALID_ARG;
+  if (out_dtype != TSP_OUT_BF16 && out_dtype != TSP_OUT_F32) return TSP_ERR_INVALID_ARG;
+  const int64_t n = dims->T * dims->h;
+  if (n == 0) return TSP_OK;
+  PartList pl = {};
+  for (int i = 0; i < n_parts; ++i) {
+    if (!parts[i] || !aligned16(parts[i])) return TSP_ERR_INVALID_ARG;
+    pl.p[i] = static_cast<const float*>(parts[i]);
+  }
+  if (!resid || !out || !aligned16(resid) || !aligned16(out)) return TSP_ERR_INVALID_ARG;
+  const unsigned blocks = static_cast<unsigned>((n / 4 + 255) / 256);
+  const bool of = out_dtype == TSP_OUT_F32;
+  if (resid_f32) {
+    if (of) sum_partials_kernel<float, true><<<blocks, 256, 0, stream>>>(pl, n_parts, static_cast<const float*>(resid), out, n);
+    else sum_partials_kernel<float, false><<<blocks, 256, 0, stream>>>(pl, n_parts, static_cast<const float*>(resid), out, n);
+  } else {
+    const __nv_bfloat16* r = static_cast<const __nv_bfloat16*>(resid);
+    if (of) sum_partials_kernel<__nv_bfloat16, true><<<blocks, 256, 0, stream>>>(pl, n_parts, r, out, n);
+    else sum_partials_kernel<__nv_bfloat16, false><<<blocks, 256, 0, stream>>>(pl, n_parts, r, out, n);
+  }
+  TSP_CUDA(cudaGetLastError());
+  return TSP_OK;
 }
 
 int tsp_selftest_wait_timeout(void* ws, uint64_t timeout_ns, cudaStream_t stream) {

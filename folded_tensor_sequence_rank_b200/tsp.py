@@ -86,6 +86,10 @@ def lib() -> ctypes.CDLL:
                                      vp, vp, vp, sz, vp, ctypes.POINTER(vp)]),
         "tsp_kv_backward_workspace_bytes": (sz, [pd, i32]),
         "tsp_kv_backward": (i32, [pd, i32, ctypes.POINTER(vp), i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "tsp_tp_workspace_bytes": (sz, [pd, i32]),
+        "tsp_tp_attention_partial": (i32, [pd, pw, i32, vp, vp, vp, sz, vp]),
+        "tsp_tp_mlp_partial": (i32, [pd, pw, i32, vp, vp, vp, sz, vp]),
+        "tsp_tp_all_reduce": (i32, [pd, i32, ctypes.POINTER(vp), vp, i32, vp, i32, vp]),
         "tsp_mlp_backward_workspace_bytes": (sz, [pd, i32]),
         "tsp_mlp_backward": (i32, [pd, pw, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, ctypes.POINTER(vp)]),
     }
@@ -374,6 +378,40 @@ def kv_backward(dims: Dims, D: int, w_full: dict, rank: int, x_local, dk_full, d
             _ptr(dwk, "dwk", torch.float32, (h, h)), _ptr(dwv, "dwv", torch.float32, (h, h))]
     _check(lib().tsp_kv_backward(ctypes.byref(dims), D, _w_full_ptrs(dims, w_full), rank, *args,
                                  _ptr(kws, "kws", torch.uint8), kws.numel(), _stream(stream)), "tsp_kv_backward")
+
+
+def alloc_tp_workspace(dims: Dims, D: int, device="cuda") -> torch.Tensor:
+    return _alloc_ws("tsp_tp_workspace_bytes", dims, D, device)
+
+
+def tp_attention_partial(dims: Dims, w: ShardedWeights, k: int, x, part, ws, stream=None):
+    """Tensor-parallel rank k's attention partial A_k Wo_k^T over all T tokens
+    (x bf16 [T, h]; part fp32 [T, h])."""
+    T, h = dims.T, dims.h
+    _check(lib().tsp_tp_attention_partial(ctypes.byref(dims), ctypes.byref(w.struct), k,
+                                          _ptr(x, "x", torch.bfloat16, (T, h)), _ptr(part, "part", torch.float32, (T, h)),
+                                          _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream)),
+           "tsp_tp_attention_partial")
+
+
+def tp_mlp_partial(dims: Dims, w: ShardedWeights, k: int, y1, part, ws, stream=None):
+    """Tensor-parallel rank k's MLP partial GELU(LN2(Y1) W1_k^T) W2_k^T (y1, part fp32 [T, h])."""
+    T, h = dims.T, dims.h
+    _check(lib().tsp_tp_mlp_partial(ctypes.byref(dims), ctypes.byref(w.struct), k,
+                                    _ptr(y1, "y1", torch.float32, (T, h)), _ptr(part, "part", torch.float32, (T, h)),
+                                    _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream)), "tsp_tp_mlp_partial")
+
+
+def tp_all_reduce(dims: Dims, parts: list, resid, out, stream=None):
+    """out = resid + sum(parts): the tensor-parallel all-reduce, on one GPU."""
+    T, h = dims.T, dims.h
+    ptrs = (ctypes.c_void_p * len(parts))(*[_ptr(t, "part", torch.float32, (T, h)) for t in parts])
+    if resid.dtype not in (torch.float32, torch.bfloat16) or out.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("resid and out must be fp32 or bf16")
+    _check(lib().tsp_tp_all_reduce(ctypes.byref(dims), len(parts), ptrs, _ptr(resid, "resid", None, (T, h)),
+                                   int(resid.dtype == torch.float32), _ptr(out, "out", None, (T, h)),
+                                   OUT_F32 if out.dtype == torch.float32 else OUT_BF16, _stream(stream)),
+           "tsp_tp_all_reduce")
 
 
 def mlp_backward_workspace_bytes(dims: Dims, D: int) -> int:

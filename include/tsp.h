@@ -385,6 +385,41 @@ int tsp_kv_backward(const tsp_dims* dims, int D, const void* const w_full[6], in
                     const void* dk_full, const void* dv_full, void* dx, void* dwk, void* dwv, void* kws,
                     size_t kws_bytes, cudaStream_t stream);
 
+/* ---- Tensor-parallel baseline layer ------------------------------------
+ * The layer TSP is compared with [zubnet.ai TSP item, paragraphs 1-2: TSP
+ * against tensor parallelism (TP, and TP with sequence parallelism), whose
+ * MLP needs an all-reduce].  A TP rank k of D holds the same shards as TSP
+ * rank k - head group k of Wq, Wk, Wv (columns) and Wo (rows), FFN block k
+ * of W1 (columns) and W2 (rows) - but every one of the T tokens:
+ *   Y1 = X + sum_k Attn_k(LN1(X) Wq_k, LN1(X) Wk_k, LN1(X) Wv_k) Wo_k^T,
+ *   Y  = Y1 + sum_k GELU(LN2(Y1) W1_k^T) W2_k^T,
+ * and each sum over k is an all-reduce across the D ranks.  On one GPU the
+ * ranks run in turn and the all-reduce is tsp_tp_all_reduce, a sum over the
+ * ranks' partial products in device memory.  Operand formats as in the TSP
+ * layer (fp16 matmul operands, fp32 accumulation and residual stream). */
+
+/* Workspace bytes of one TP rank (tsp_tp_attention_partial and
+ * tsp_tp_mlp_partial share it; status section first); 0 on a bad argument. */
+size_t tsp_tp_workspace_bytes(const tsp_dims* dims, int D);
+
+/* TP rank k's partial of the attention half: LN1(X) over all T tokens, its
+ * head group's Q, K, V, causal attention over the whole sequence, and
+ * A_k Wo_k^T.  x: bf16 [T, h] natural order; part: fp32 [T, h] written; w:
+ * the packed shards (w->D = D, the TP degree). */
+int tsp_tp_attention_partial(const tsp_dims* dims, const tsp_weights* w, int k, const void* x, void* part,
+                             void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* TP rank k's partial of the MLP half: GELU(LN2(Y1) W1_k^T) W2_k^T over all T
+ * tokens.  y1: fp32 [T, h]; part: fp32 [T, h] written. */
+int tsp_tp_mlp_partial(const tsp_dims* dims, const tsp_weights* w, int k, const void* y1, void* part, void* ws,
+                       size_t ws_bytes, cudaStream_t stream);
+
+/* The all-reduce of the TP layer on one GPU: out = resid + sum of the
+ * n_parts fp32 [T, h] partials (1 <= n_parts <= TSP_MAX_D).  resid: fp32
+ * (resid_f32 = 1) or bf16 [T, h]; out: TSP_OUT_F32 or TSP_OUT_BF16 [T, h]. */
+int tsp_tp_all_reduce(const tsp_dims* dims, int n_parts, const void* const parts[], const void* resid,
+                      int resid_f32, void* out, int out_dtype, cudaStream_t stream);
+
 /* Fault-detection self test: launches one block that waits on a barrier
  * nothing will ever complete, with a limit of `timeout_ns` nanoseconds
  * (at most 2e9).  The wait gives up, the kernel records TSP_ERR_TIMEOUT in
