@@ -333,6 +333,39 @@ int launch_proj(const Sizes& s, int rank, const __half* xn, const void* const* f
   return launch_gemm(p, bn, st);
 }
 
+// launch_proj with the shard list of `shards` (its D) and the zigzag row
+// mapping of `zz` (rank, D, c): one shard per segment whose K/V rows still go
+// to the rank's global positions.
+int launch_proj_zz(const Sizes& zz, const Sizes& shards, int rank, const __half* xn, const void* const* fam[3],
+                   void* out[3], const int remap[3], int nseg, int epi, int F_cols, int* status, cudaStream_t st) {
+  static thread_local GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  const int shard_n = F_cols / shards.D;
+  int rc = make_map(&p.map_a, xn, zz.L, zz.h, zz.h, kGemmBM);
+  if (rc) return rc;
+  const int bn = pick_bn(shard_n);
+  for (int seg = 0; seg < nseg; ++seg)
+    for (int k = 0; k < shards.D; ++k) {
+      rc = make_map(&p.map_b[seg * shards.D + k], fam[seg][k], shard_n, zz.h, zz.h, b_box_rows(bn));
+      if (rc) return rc;
+    }
+  p.M = static_cast<int>(zz.L);
+  p.N = nseg * F_cols;
+  p.K = zz.h;
+  p.ksplit = 0;
+  p.shard_n = shard_n;
+  p.shard_k = zz.h;
+  p.seg_n = F_cols;
+  p.epi = epi;
+  for (int i = 0; i < nseg; ++i) {
+    p.out[i] = out[i];
+    p.remap[i] = remap[i];
+  }
+  p.ldo = F_cols;
+  gemm_common(p, zz, rank, status);
+  return launch_gemm(p, bn, st);
+}
+
 // K-split: out = resid + sum_k A[:, k-block] W_k^T, W_k [h, Kdim/D].
 int launch_ksplit(const Sizes& s, int rank, const __half* a, int Kdim, const void* const* fam, const void* resid,
                   int resid_f32, void* out, int out_f32, int* status, cudaStream_t st) {
@@ -1461,6 +1494,118 @@ int tsp_tp_all_reduce(const tsp_dims* dims, int n_parts, const void* const parts
   }
   TSP_CUDA(cudaGetLastError());
   return TSP_OK;
+}
+
+// ---------------------------------------------------------------- per-shard steps
+namespace {
+
+// Sizes of one head group (shard) of the attention: h/D columns, H/D heads.
+Sizes head_group(const Sizes& s) {
+  Sizes g = s;
+  g.h = s.hs;
+  g.H = s.H / s.D;
+  return g;
+}
+
+int shard_args(const tsp_dims* dims, int D, int rank, Sizes* s) {
+  int rc = check_dims(dims, D);
+  if (rc) return rc;
+  if (rank < 0 || rank >= D) return TSP_ERR_INVALID_ARG;
+  *s = sizes_of(dims, D);
+  return TSP_OK;
+}
+
+bool ok16(std::initializer_list<const void*> ps) {
+  for (const void* p : ps)
+    if (!p || !aligned16(p)) return false;
+  return true;
+}
+
+int* status_of(void* ws) { return static_cast<int*>(ws); }
+
+}  // namespace
+
+size_t tsp_shard_workspace_bytes(void) { return 2 * kAlign; }
+
+int tsp_layernorm(int64_t rows, int h, float eps, const void* x, int x_f32, void* y, cudaStream_t stream) {
+  if (rows < 0 || h <= 0 || h % 8 || h > 8192 || !(eps >= 0.f)) return TSP_ERR_INVALID_ARG;
+  if (rows == 0) return TSP_OK;
+  if (!ok16({x, y})) return TSP_ERR_INVALID_ARG;
+  if (x_f32) return launch_layernorm<float>(static_cast<const float*>(x), static_cast<__half*>(y), rows, h, eps, stream);
+  return launch_layernorm<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x), static_cast<__half*>(y), rows, h, eps,
+                                         stream);
+}
+
+int tsp_shard_qkv(const tsp_dims* dims, int D, int rank, const void* wq_k, const void* wk_k, const void* wv_k,
+                  const void* xn1, void* q_k, void* k_k, void* v_k, void* ws, cudaStream_t stream) {
+  Sizes s;
+  int rc = shard_args(dims, D, rank, &s);
+  if (rc) return rc;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return TSP_ERR_INVALID_ARG;
+  if (s.L == 0) return TSP_OK;
+  if (!ok16({wq_k, wk_k, wv_k, xn1, q_k, k_k, v_k})) return TSP_ERR_INVALID_ARG;
+  const void* wq[1] = {wq_k};
+  const void* wk[1] = {wk_k};
+  const void* wv[1] = {wv_k};
+  const void* const* fam[3] = {wq, wk, wv};
+  void* out[3] = {q_k, k_k, v_k};
+  const int remap[3] = {0, 1, 1};  // K, V rows to their global positions
+  Sizes one = s;
+  one.D = 1;  // one shard per segment; the zigzag rows still follow (rank, D)
+  return launch_proj_zz(s, one, rank, static_cast<const __half*>(xn1), fam, out, remap, 3, kEpiStoreBf16, s.hs,
+                        status_of(ws), stream);
+}
+
+int tsp_shard_attention(const tsp_dims* dims, int D, int rank, const void* q_k, const void* k_k, const void* v_k,
+                        void* a_k, void* ws, cudaStream_t stream) {
+  Sizes s;
+  int rc = shard_args(dims, D, rank, &s);
+  if (rc) return rc;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return TSP_ERR_INVALID_ARG;
+  if (s.L == 0) return TSP_OK;
+  if (!ok16({q_k, k_k, v_k, a_k})) return TSP_ERR_INVALID_ARG;
+  tsp_dims dg = *dims;
+  dg.h = s.hs;
+  dg.n_heads = s.H / D;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  return launch_attention(head_group(s), rank, &dg, static_cast<const __half*>(q_k), k_k, v_k,
+                          static_cast<__half*>(a_k), nullptr, reinterpret_cast<int*>(base + kAlign),
+                          status_of(ws), stream);
+}
+
+int tsp_shard_ffn_up(const tsp_dims* dims, int D, const void* w1_k, const void* xn2, void* h_k, void* ws,
+                     cudaStream_t stream) {
+  Sizes s;
+  int rc = shard_args(dims, D, 0, &s);
+  if (rc) return rc;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return TSP_ERR_INVALID_ARG;
+  if (s.L == 0) return TSP_OK;
+  if (!ok16({w1_k, xn2, h_k})) return TSP_ERR_INVALID_ARG;
+  const void* w1[1] = {w1_k};
+  const void* const* fam[3] = {w1, nullptr, nullptr};
+  void* out[3] = {h_k, nullptr, nullptr};
+  const int noremap[3] = {0, 0, 0};
+  Sizes one = s;
+  one.D = 1;
+  return launch_proj_zz(s, one, 0, static_cast<const __half*>(xn2), fam, out, noremap, 1, kEpiGeluBf16, s.Fs,
+                        status_of(ws), stream);
+}
+
+int tsp_shard_accumulate(const tsp_dims* dims, int D, const void* act, int k_dim, const void* w_k, void* y,
+                         void* ws, cudaStream_t stream) {
+  Sizes s;
+  int rc = shard_args(dims, D, 0, &s);
+  if (rc) return rc;
+  if (k_dim != s.hs && k_dim != s.Fs) return TSP_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return TSP_ERR_INVALID_ARG;
+  if (s.L == 0) return TSP_OK;
+  if (!ok16({act, w_k, y})) return TSP_ERR_INVALID_ARG;
+  // y += act [L, k_dim] w_k^T (w_k K-major [h, k_dim]); the residual epilogue
+  // reads each value of y before it writes it
+  const void* fam[1] = {w_k};
+  Sizes one = s;
+  one.D = 1;
+  return launch_ksplit(one, 0, static_cast<const __half*>(act), k_dim, fam, y, 1, y, 1, status_of(ws), stream);
 }
 
 int tsp_selftest_wait_timeout(void* ws, uint64_t timeout_ns, cudaStream_t stream) {

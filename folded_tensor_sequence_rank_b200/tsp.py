@@ -86,6 +86,12 @@ def lib() -> ctypes.CDLL:
                                      vp, vp, vp, sz, vp, ctypes.POINTER(vp)]),
         "tsp_kv_backward_workspace_bytes": (sz, [pd, i32]),
         "tsp_kv_backward": (i32, [pd, i32, ctypes.POINTER(vp), i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "tsp_shard_workspace_bytes": (sz, []),
+        "tsp_layernorm": (i32, [i64, i32, ctypes.c_float, vp, i32, vp, vp]),
+        "tsp_shard_qkv": (i32, [pd, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "tsp_shard_attention": (i32, [pd, i32, i32, vp, vp, vp, vp, vp, vp]),
+        "tsp_shard_ffn_up": (i32, [pd, i32, vp, vp, vp, vp, vp]),
+        "tsp_shard_accumulate": (i32, [pd, i32, vp, i32, vp, vp, vp, vp]),
         "tsp_tp_workspace_bytes": (sz, [pd, i32]),
         "tsp_tp_attention_partial": (i32, [pd, pw, i32, vp, vp, vp, sz, vp]),
         "tsp_tp_mlp_partial": (i32, [pd, pw, i32, vp, vp, vp, sz, vp]),

@@ -420,6 +420,52 @@ int tsp_tp_mlp_partial(const tsp_dims* dims, const tsp_weights* w, int k, const 
 int tsp_tp_all_reduce(const tsp_dims* dims, int n_parts, const void* const parts[], const void* resid,
                       int resid_f32, void* out, int out_dtype, cudaStream_t stream);
 
+/* ---- Per-shard steps --------------------------------------------------
+ * One rank's layer forward taken shard by shard, for running the TSP
+ * exchange across GPUs [zubnet.ai TSP item, paragraph 2: the attention
+ * shards are broadcast one after another and every rank applies each to its
+ * own tokens, K/V are all-gathered under the zigzag partition, and the MLP
+ * shards pass around a ring], where each weight shard and each head group's
+ * K/V arrive one at a time and the transfer of the next overlaps the
+ * compute of the current one.  Composed in order they compute what
+ * tsp_layer_forward computes (the shard sums accumulate in the fp32 output
+ * instead of inside one product):
+ *   xn1 = LN1(x);  y1 = x;
+ *   for each head group k: tsp_shard_qkv, all-gather K_k/V_k,
+ *       tsp_shard_attention, tsp_shard_accumulate(a_k, Wo_k, y1);
+ *   xn2 = LN2(y1);  y = y1;
+ *   for each FFN block k: tsp_shard_ffn_up, tsp_shard_accumulate(h_k, W2_k, y).
+ * Shard pointers are the packed fp16 shards of tsp_pack_shards.  ws:
+ * tsp_shard_workspace_bytes() bytes, 256-byte aligned, status section first
+ * (tsp_get_device_status). */
+size_t tsp_shard_workspace_bytes(void);
+
+/* y = LN(x) fp16 [rows, h] for x bf16 (x_f32 = 0) or fp32 (x_f32 = 1),
+ * biased variance, eps inside the square root, gamma = 1, beta = 0. */
+int tsp_layernorm(int64_t rows, int h, float eps, const void* x, int x_f32, void* y, cudaStream_t stream);
+
+/* Head group k of the rank's projections: q_k = xn1 Wq_k^T fp16 [T/D, h/D]
+ * (rank-local rows); K_k, V_k = xn1 Wk_k^T, xn1 Wv_k^T written at the rank's
+ * GLOBAL rows of k_k, v_k fp16 [T, h/D] (what the all-gather then fills in
+ * for the other ranks).  xn1: fp16 [T/D, h]. */
+int tsp_shard_qkv(const tsp_dims* dims, int D, int rank, const void* wq_k, const void* wk_k, const void* wv_k,
+                  const void* xn1, void* q_k, void* k_k, void* v_k, void* ws, cudaStream_t stream);
+
+/* Causal attention of head group k: a_k fp16 [T/D, h/D] from q_k [T/D, h/D]
+ * and the group's all-gathered k_k, v_k [T, h/D] (natural order). */
+int tsp_shard_attention(const tsp_dims* dims, int D, int rank, const void* q_k, const void* k_k, const void* v_k,
+                        void* a_k, void* ws, cudaStream_t stream);
+
+/* FFN block k: h_k = GELU(xn2 W1_k^T) fp16 [T/D, F/D], xn2 fp16 [T/D, h]. */
+int tsp_shard_ffn_up(const tsp_dims* dims, int D, const void* w1_k, const void* xn2, void* h_k, void* ws,
+                     cudaStream_t stream);
+
+/* y += act w_k^T for one shard: act fp16 [T/D, k_dim] with k_dim = h/D (the
+ * attention output a_k, w_k = Wo_k) or F/D (h_k, w_k = W2_k); y fp32
+ * [T/D, h], read and written in place. */
+int tsp_shard_accumulate(const tsp_dims* dims, int D, const void* act, int k_dim, const void* w_k, void* y,
+                         void* ws, cudaStream_t stream);
+
 /* Fault-detection self test: launches one block that waits on a barrier
  * nothing will ever complete, with a limit of `timeout_ns` nanoseconds
  * (at most 2e9).  The wait gives up, the kernel records TSP_ERR_TIMEOUT in
