@@ -290,17 +290,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
           const uint64_t dQ_k = dQ_k0 + static_cast<uint64_t>(qs * (S::kTileBytes >> 4));
           const uint64_t dQ_mn = dQ_mn0 + static_cast<uint64_t>(qs * (S::kTileBytes >> 4));
           if (!mbar_wait(&q_full[qs], qph[qs], ctl)) { ok = false; break; }
-          if (!mbar_wait(do_full, doph, ctl)) { ok = false; break; }
-          // the dP^T columns hold the previous tile's dQ until it is read out
-          if (tiles > 0 && !mbar_wait(dq_free, (tiles - 1) & 1, ctl)) { ok = false; break; }
           tc_fence_after();
-          // S^T = K Q^T and dP^T = V dO^T (K = head_dim)
+          // S^T = K Q^T (K = head_dim); the softmax warps read the previous
+          // tile's S^T before they signalled p_full
           if constexpr (HD == 128) {
             mma_ss_x8<0, 2, 4, 6, 1024, 1026, 1028, 1030>(t_s, dK_k, dQ_k, idesc_s, 0);
-            mma_ss_x8<0, 2, 4, 6, 1024, 1026, 1028, 1030>(t_dp, dV_k, dDO_k, idesc_s, 0);
           } else {
 #pragma unroll
             for (int kk = 0; kk < HD / 16; ++kk) mma_ss(t_s, dK_k + 2 * kk, dQ_k + 2 * kk, idesc_s, kk != 0);
+          }
+          if (!mbar_wait(do_full, doph, ctl)) { ok = false; break; }
+          // dP^T = V dO^T: the dP^T columns hold the previous tile's dQ until
+          // it is read out
+          if (tiles > 0 && !mbar_wait(dq_free, (tiles - 1) & 1, ctl)) { ok = false; break; }
+          tc_fence_after();
+          if constexpr (HD == 128) {
+            mma_ss_x8<0, 2, 4, 6, 1024, 1026, 1028, 1030>(t_dp, dV_k, dDO_k, idesc_s, 0);
+          } else {
 #pragma unroll
             for (int kk = 0; kk < HD / 16; ++kk) mma_ss(t_dp, dV_k + 2 * kk, dDO_k + 2 * kk, idesc_s, kk != 0);
           }
