@@ -39,7 +39,11 @@
 //   dV += P^T dO (TS, dO MN-major), dK += dS^T Q (SS, Q MN-major), and, once
 //   the dV MMA has completed (it reads P^T from the dP^T columns), dQ = dS K
 //   into the dP^T columns (SS, both MN-major); the softmax warps read dQ out
-//   and add it to global memory.
+//   of tensor memory (which frees the columns at once) and add it to global
+//   memory: each warp stages its 32 x 32 fp32 blocks in its 4 KiB of the dS^T
+//   buffer and one lane adds each block with a TMA bulk reduction (whole
+//   128-byte lines per L2 operation instead of 16-byte vector reductions);
+//   the next tile's dS^T waits until those reductions have read the staging.
 // Q, K, V, dO, P and dS are fp16 (the forward's operand format); scores,
 // statistics, accumulators and the outputs are fp32.
 #pragma once
@@ -57,6 +61,7 @@ struct __align__(64) AttnBwdParams {
   CUtensorMap map_do;  // dO [L, h] fp16, box {64, 128}
   CUtensorMap map_k;   // K [T, h] fp16, box {64, 128}
   CUtensorMap map_v;   // V [T, h] fp16, box {64, 128}
+  CUtensorMap map_dq;  // dQ [L, h] fp32, box {32, 32}, 128-byte swizzle (bulk reductions)
   const float* lse;    // [H][2][c_pad] log2-domain log-sum-exp (forward stash)
   const float* delta;  // [H][2][c_pad] scale * rowsum(dO * O) per head
   float* dq;           // [L, h] fp32, added to
@@ -143,8 +148,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
   uint64_t* p_full = s_full + 1;      // P^T (tensor memory) and dS^T (shared) written, 8 warps
   uint64_t* dv_done = p_full + 1;     // the dV MMA of the tile completed
   uint64_t* dq_full = dv_done + 1;    // dQ of the tile in tensor memory
-  uint64_t* dq_free = dq_full + 1;    // dQ read out, 8 warps
-  uint64_t* dkv_full = dq_free + 1;   // dK, dV of the item complete
+  uint64_t* dq_free = dq_full + 1;    // dQ read out of tensor memory, 8 warps
+  uint64_t* stg_free = dq_free + 1;   // the staged dQ blocks have been read by their bulk reductions, 8 warps
+  uint64_t* dkv_full = stg_free + 1;  // dK, dV of the item complete
   uint64_t* dkv_free = dkv_full + 1;  // dK, dV read out, 8 warps
   uint64_t* it_full = dkv_free + 1;   // [2]
   uint64_t* it_empty = it_full + 2;   // [2]
@@ -170,6 +176,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
     mbar_init(dv_done, 1);
     mbar_init(dq_full, 1);
     mbar_init(dq_free, 8);
+    mbar_init(stg_free, 8);
     mbar_init(dkv_full, 1);
     mbar_init(dkv_free, 8);
     for (int x = 0; x < 2; ++x) {
@@ -423,13 +430,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
             P[cc * 16 + i] = pack_half2(pr.x, pr.y);
             dsp[i] = pack_half2(dsv.x, dsv.y);
           }
-          // dS^T row kr, queries col0 .. col0+31: four 16-byte groups
+          // dS^T row kr, queries col0 .. col0+31: four 16-byte groups; the
+          // buffer held the previous tile's staged dQ until its bulk
+          // reductions had read it
+          if (cc == 0 && tiles > 0 && !warp_wait(stg_free, (tiles - 1) & 1, ctl)) { ok = false; break; }
           uint8_t* rowp = sDS;
 #pragma unroll
           for (int g = 0; g < 4; ++g)
             *reinterpret_cast<uint4*>(rowp + sw128_offset(kr, col0 / 8 + g)) =
                 make_uint4(dsp[4 * g], dsp[4 * g + 1], dsp[4 * g + 2], dsp[4 * g + 3]);
         }
+        if (!ok) break;
         // P^T over the dP^T columns this warp has read (queries 64*half ..)
         tmem_st32p(t_dp + lane_off + half * 64, P);
         tmem_st_wait();
@@ -441,27 +452,54 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
         if (!warp_wait(dq_full, tiles & 1, ctl)) { ok = false; break; }
         tc_fence_after();
         {
-          const int qrow = kr;  // lane = query row of the dQ tile
-          const bool qvalid = qrow < q.nvalid;
-          float* dst = p.dq + static_cast<int64_t>(q.m0 + qrow) * p.ld + head * HD + half * (HD / 2);
+          // the whole of this warp's dQ block into registers, then the tensor
+          // memory columns go back to the issuer
+          uint32_t r[HD / 2];
 #pragma unroll
-          for (int j = 0; j < HD / 64; ++j) {
-            uint32_t r[32];
-            tmem_ld32(t_dp + lane_off + half * (HD / 2) + 32 * j, r);
-            tmem_ld_wait();
-            reg_fence32(r);
-            if (qvalid) {
+          for (int j = 0; j < HD / 64; ++j) tmem_ld32p(t_dp + lane_off + half * (HD / 2) + 32 * j, &r[32 * j]);
+          tmem_ld_wait();
 #pragma unroll
-              for (int i = 0; i < 8; ++i)
-                atomicAdd(reinterpret_cast<float4*>(dst + 32 * j) + i,
+          for (int j = 0; j < HD / 64; ++j) reg_fence32(&r[32 * j]);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(dq_free);
+          if (q.nvalid == kBwdTile) {
+            // whole tile: stage each 32 x 32 block (128-byte swizzled) in this
+            // warp's 4 KiB of the dS^T buffer - free: the dQ MMA has read it -
+            // and add it with one bulk reduction
+            uint8_t* stg = sDS + (warp - 2) * 4096;
+#pragma unroll
+            for (int j = 0; j < HD / 64; ++j) {
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                    make_uint4(r[32 * j + 4 * c], r[32 * j + 4 * c + 1], r[32 * j + 4 * c + 2], r[32 * j + 4 * c + 3]);
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_reduce_add_2d(&p.map_dq, stg, head * HD + half * (HD / 2) + 32 * j, q.m0 + quarter * 32);
+                bulk_commit_group();
+                bulk_wait_group_read0();
+              }
+              __syncwarp();
+            }
+          } else {
+            // a ragged tile (the last of a chunk whose length is not a multiple
+            // of 128): rows past the chunk are skipped, one vector reduction
+            // per 16 bytes
+            const int qrow = kr;  // lane = query row of the dQ tile
+            if (qrow < q.nvalid) {
+              float* dst = p.dq + static_cast<int64_t>(q.m0 + qrow) * p.ld + head * HD + half * (HD / 2);
+#pragma unroll
+              for (int i = 0; i < HD / 8; ++i)
+                atomicAdd(reinterpret_cast<float4*>(dst) + i,
                           make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
                                       __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])));
             }
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(stg_free);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(dq_free);
         qph[qs] ^= 1;
         if (++qs == QST) qs = 0;
         ++tiles;

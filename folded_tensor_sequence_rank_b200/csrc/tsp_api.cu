@@ -85,6 +85,28 @@ int make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64
   return TSP_OK;
 }
 
+// 2-D fp32 row-major [rows, cols] with row stride ld elements; box = box_cols
+// (<= 32: at most 128 bytes, 128B swizzle) x box_rows rows.  Used as the
+// destination of bulk reductions.
+int make_map_f32(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int64_t ld, int box_rows, int box_cols) {
+  auto fn = encode_fn();
+  if (!fn) {
+    std::snprintf(g_cuda_err, sizeof(g_cuda_err), "cuTensorMapEncodeTiled unavailable");
+    return TSP_ERR_CUDA;
+  }
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 4};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_cuda_err, sizeof(g_cuda_err), "cuTensorMapEncodeTiled (fp32) failed (%d)", static_cast<int>(r));
+    return TSP_ERR_CUDA;
+  }
+  return TSP_OK;
+}
+
 int num_sms() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -548,6 +570,7 @@ int launch_attn_backward(const Sizes& s, int rank, const tsp_dims* dims, const _
   if ((rc = make_map(&p.map_do, d_o, s.L, s.h, s.h, kBwdTile))) return rc;
   if ((rc = make_map(&p.map_k, k_full, s.T, s.h, s.h, kBwdTile))) return rc;
   if ((rc = make_map(&p.map_v, v_full, s.T, s.h, s.h, kBwdTile))) return rc;
+  if ((rc = make_map_f32(&p.map_dq, dq, s.L, s.h, s.h, 32, 32))) return rc;
   p.lse = lse;
   p.delta = delta;
   p.dq = dq;
