@@ -17,6 +17,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "csrc", "tsp_api.cu")
 OUT = os.path.join(HERE, "libtsp_b200.so")
+# The same source with -DTSP_DEBUG: device index checks that record a status
+# (TSP_ERR_BOUNDS) and skip the access instead of faulting.
+OUT_DEBUG = os.path.join(HERE, "libtsp_b200_debug.so")
 HEADERS = [os.path.join(HERE, "csrc", f) for f in ("ptx.cuh", "gemm_sm100.cuh", "gemm_pair_sm100.cuh", "attn_sm100.cuh",
                                                    "attn_bwd_sm100.cuh", "misc_kernels.cuh")]
 HEADERS.append(os.path.join(ROOT, "include", "tsp.h"))
@@ -44,10 +47,13 @@ def up_to_date(out: str = OUT) -> bool:
     return all(os.path.getmtime(f) <= t for f in [SRC, *HEADERS])
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and not extra and up_to_date():
-        return OUT
-    cmd = command(extra=list(extra))
+def build(force: bool = False, verbose: bool = False, extra=(), debug: bool = False) -> str:
+    out = OUT_DEBUG if debug else OUT
+    if debug:
+        extra = ["-DTSP_DEBUG", *extra]
+    if not force and not (extra and not debug) and up_to_date(out):
+        return out
+    cmd = command(out=out, extra=list(extra))
     if verbose:
         print(" ".join(cmd), flush=True)
     res = subprocess.run(cmd, capture_output=True, text=True)
@@ -56,10 +62,10 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         sys.stderr.write(res.stderr)
     if res.returncode != 0:
         raise RuntimeError(f"nvcc failed with exit code {res.returncode}")
-    return OUT
+    return out
 
 
 if __name__ == "__main__":
     v = "--verbose" in sys.argv
     extra = ["-Xptxas", "-v"] if "--ptxas" in sys.argv else []
-    print(build(force=True, verbose=v, extra=extra))
+    print(build(force=True, verbose=v, extra=extra, debug="--debug" in sys.argv))

@@ -237,6 +237,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
           for (int b = 0; b < NB; ++b)
             tma_load_2d(sQ + qs * S::kTileBytes + b * 16384, &p.map_q, &q_full[qs], col0 + 64 * b, q.m0);
           const int64_t srow = static_cast<int64_t>(head * 2 + q.chunk) * p.c_pad + q.t * kBwdTile;
+          if (!dbg_ok(q.t * kBwdTile + kBwdTile <= p.c_pad && head < p.H, p.status)) { ok = false; break; }
           bulk_load(sStat + qs * 2 * kBwdTile, p.lse + srow, S::kStatBytes, &q_full[qs]);
           bulk_load(sStat + qs * 2 * kBwdTile + kBwdTile, p.delta + srow, S::kStatBytes, &q_full[qs]);
           q_used |= 1u << qs;
@@ -476,7 +477,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
                     make_uint4(r[32 * j + 4 * c], r[32 * j + 4 * c + 1], r[32 * j + 4 * c + 2], r[32 * j + 4 * c + 3]);
               fence_proxy_async_smem();
               __syncwarp();
-              if (lane == 0) {
+              if (lane == 0 && dbg_ok(q.m0 + quarter * 32 + 32 <= 2 * p.c && (head + 1) * HD <= p.ld, p.status)) {
                 tma_reduce_add_2d(&p.map_dq, stg, head * HD + half * (HD / 2) + 32 * j, q.m0 + quarter * 32);
                 bulk_commit_group();
                 bulk_wait_group_read0();
@@ -488,7 +489,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
             // of 128): rows past the chunk are skipped, one vector reduction
             // per 16 bytes
             const int qrow = kr;  // lane = query row of the dQ tile
-            if (qrow < q.nvalid) {
+            if (qrow < q.nvalid && dbg_ok(q.m0 + qrow < 2 * p.c, p.status)) {
               float* dst = p.dq + static_cast<int64_t>(q.m0 + qrow) * p.ld + head * HD + half * (HD / 2);
 #pragma unroll
               for (int i = 0; i < HD / 8; ++i)
@@ -523,7 +524,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
             tmem_ld32(src + 32 * j, r);
             tmem_ld_wait();
             reg_fence32(r);
-            if (kvalid) {
+            if (kvalid && dbg_ok((head + 1) * HD <= p.ld, p.status)) {
 #pragma unroll
               for (int i = 0; i < 8; ++i)
                 atomicAdd(reinterpret_cast<float4*>(dst + 32 * j) + i,
@@ -575,7 +576,8 @@ __global__ void __launch_bounds__(256) attn_bwd_delta_kernel(const __half* __res
     if (col < h && (threadIdx.x & (kLanesPerHead - 1)) == 0) {
       const int head = col / HD;
       const int chunk = row >= c ? 1 : 0;
-      delta[(static_cast<int64_t>(head) * 2 + chunk) * c_pad + (row - chunk * c)] = scale * sum;
+      if (dbg_ok(row - chunk * c < c, nullptr))
+        delta[(static_cast<int64_t>(head) * 2 + chunk) * c_pad + (row - chunk * c)] = scale * sum;
     }
   }
 }

@@ -489,7 +489,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
       const float inv = 1.0f / l;
       if (p.lse != nullptr && row_valid) {
         const int chunk = T.m0 >= p.c ? 1 : 0;
-        p.lse[(w.head * 2 + chunk) * p.c_pad + (T.m0 - chunk * p.c) + row] = m_used + lg2_approx(l);
+        const int li = (T.m0 - chunk * p.c) + row;
+        if (dbg_ok(w.head < p.H && li < p.c, p.status))
+          p.lse[(w.head * 2 + chunk) * p.c_pad + li] = m_used + lg2_approx(l);
       }
       __half* dst = p.out + static_cast<int64_t>(T.m0 + row) * p.ldo + w.head * HD;
 #pragma unroll
@@ -497,7 +499,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
         uint32_t r[32];
         tmem_ld32(t_o + j * 32, r);
         tmem_ld_wait();
-        if (row_valid) {
+        if (row_valid && dbg_ok(T.m0 + row < 2 * p.c && (w.head + 1) * HD <= p.ldo, p.status)) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + j * 32);
 #pragma unroll
           for (int i = 0; i < 4; ++i)

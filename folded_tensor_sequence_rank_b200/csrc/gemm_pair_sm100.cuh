@@ -180,12 +180,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_pair_f16_tcgen05(const _
       const bool valid = m < p.M;
       const int64_t grow = (m < p.c) ? (p.off0 + m) : (p.off1 + m);
       // Software-pipelined over the 32-column chunks: the next chunk's
-      // accumulators (and, for kEpiGeluBwd, its U values) are loaded while
-      // this chunk is processed.
+      // accumulators (and its U values or residual) are loaded while this
+      // chunk is processed.
       constexpr int kChunks = kPairBN / 32;
-      const bool aux_on = valid && p.epi == kEpiGeluBwd;
+      const bool aux_on = valid && epilogue_has_aux(p);
       uint32_t r[32], rn[32];
-      uint4 aux[4] = {}, auxn[4] = {};
+      uint4 aux[8] = {}, auxn[8] = {};
       __syncwarp();
       tmem_ld32(tmem_base + lane_off + buf * kPairBN, r);
       if (aux_on) load_epilogue_aux(p, m, nb * kPairBN, aux);
@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_pair_f16_tcgen05(const _
 #pragma unroll
           for (int i = 0; i < 32; ++i) r[i] = rn[i];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) aux[i] = auxn[i];
+          for (int i = 0; i < 8; ++i) aux[i] = auxn[i];
         }
       }
       tc_fence_before();

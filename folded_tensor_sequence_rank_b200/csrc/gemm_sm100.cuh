@@ -65,6 +65,7 @@ struct __align__(64) GemmParams {
   int out_f32;        // kEpiResidual: output fp32 (1) or bf16 (0)
   int c;              // zigzag: local rows [0,c) -> off0 + m, [c, 2c) -> off1 + m
   int64_t off0, off1;
+  int64_t remap_rows;  // rows of a remapped (global-row) output: index checks of the debug build
   int* status;        // status word; status[1] is the flags word
   uint64_t timeout_ns;
 };
@@ -154,19 +155,33 @@ __device__ __forceinline__ void store_transposed_bf16(const GemmParams& p, uint3
   for (int i = 0; i < 4; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
 }
 
-// kEpiGeluBwd's U values for row m, columns n .. n+31 (the epilogue loop
-// loads them one chunk ahead).
-__device__ __forceinline__ void load_epilogue_aux(const GemmParams& p, int m, int n, uint4 (&a)[4]) {
-  const uint4* us = reinterpret_cast<const uint4*>(static_cast<const __half*>(p.resid) + static_cast<int64_t>(m) * p.ldo + n);
+// The second operand an epilogue reads for row m, columns n .. n+31: U
+// (kEpiGeluBwd, fp16) or the residual (kEpiResidual, bf16 or fp32) - 64 or
+// 128 bytes, at the row stride ldo.  The epilogue loops load it one chunk
+// ahead, while the current chunk is processed.
+__device__ __forceinline__ bool epilogue_has_aux(const GemmParams& p) {
+  return p.epi == kEpiGeluBwd || p.epi == kEpiResidual;
+}
+
+__device__ __forceinline__ void load_epilogue_aux(const GemmParams& p, int m, int n, uint4 (&a)[8]) {
+  const int64_t off = static_cast<int64_t>(m) * p.ldo + n;
+  if (p.epi == kEpiResidual && p.resid_f32) {
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const float*>(p.resid) + off);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) a[i] = us[i];
+    for (int i = 0; i < 8; ++i) a[i] = src[i];
+  } else {
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.resid) + off);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] = src[i];
+  }
 }
 
 // One 32-column chunk of an output tile's epilogue: accumulator values r for
 // local row m (global zigzag row grow) and output columns n .. n+31.
 __device__ __forceinline__ void gemm_epilogue_chunk(const GemmParams& p, int m, int64_t grow, int n,
-                                                    const uint32_t (&r)[32], const uint4 (&aux)[4],
+                                                    const uint32_t (&r)[32], const uint4 (&aux)[8],
                                                     uint32_t* stage) {
+  if (!dbg_ok(m < p.M && n + 32 <= p.N, p.status)) return;
   if (p.epi == kEpiStoreF32) {
     float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out[0]) + static_cast<int64_t>(m) * p.ldo + n);
 #pragma unroll
@@ -203,17 +218,16 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const GemmParams& p, int m, 
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
     const int64_t off = static_cast<int64_t>(m) * p.ldo + n;
     if (p.resid_f32) {
-      const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.resid) + off);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float4 q = src[i];
-        v[4 * i] += q.x; v[4 * i + 1] += q.y; v[4 * i + 2] += q.z; v[4 * i + 3] += q.w;
+        const uint4 q = aux[i];
+        v[4 * i] += __uint_as_float(q.x); v[4 * i + 1] += __uint_as_float(q.y);
+        v[4 * i + 2] += __uint_as_float(q.z); v[4 * i + 3] += __uint_as_float(q.w);
       }
     } else {
-      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.resid) + off);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const uint4 q = src[i];
+        const uint4 q = aux[i];
         const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -239,6 +253,8 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const GemmParams& p, int m, 
     const int seg = n / p.seg_n;
     const int col = n - seg * p.seg_n;
     const int64_t orow = p.remap[seg] ? grow : m;
+    if (!dbg_ok(seg < 3 && col + 32 <= p.seg_n && (!p.remap[seg] || (orow >= 0 && orow < p.remap_rows)), p.status))
+      return;
     uint32_t packed[16];
     float mx = 0.f;  // largest magnitude converted: flags a saturation
     if (p.epi == kEpiGeluBf16) {
@@ -414,8 +430,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_f16_tcgen05(const __grid
         tmem_ld_wait();
         reg_fence32(r);
         const int n = nb * BN + ch * 32;
-        uint4 aux[4] = {};
-        if (valid && p.epi == kEpiGeluBwd) load_epilogue_aux(p, m, n, aux);
+        uint4 aux[8] = {};
+        if (valid && epilogue_has_aux(p)) load_epilogue_aux(p, m, n, aux);
         if (valid) gemm_epilogue_chunk(p, m, grow, n, r, aux, stage);
       }
       tc_fence_before();

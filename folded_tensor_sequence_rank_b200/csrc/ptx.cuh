@@ -12,6 +12,20 @@ namespace tsp {
 constexpr int kStatusTimeout = 4;
 // Bits of the flags word that follows the status word (status[1]).
 constexpr int kFlagFp16Saturated = 1;
+constexpr int kFlagBoundsCheck = 2;  // a debug-build index check failed (the access was skipped)
+
+// Index checks of the debug build (compiled with -DTSP_DEBUG): a failed check
+// records kFlagBoundsCheck and the caller skips the access, so a wrong index
+// shows up as a status, never as a memory fault.  In the normal build the
+// check is the constant true and costs nothing.
+#ifdef TSP_DEBUG
+__device__ __forceinline__ bool dbg_ok(bool cond, int* status) {
+  if (!cond && status) atomicOr(status + 1, kFlagBoundsCheck);
+  return cond;
+}
+#else
+__device__ __forceinline__ constexpr bool dbg_ok(bool, int*) { return true; }
+#endif
 
 // Records that a value outside fp16's finite range (|x| > 65504) was clamped
 // to +-65504 by a saturating conversion.  `status` is the status word; the

@@ -11,6 +11,8 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -28,6 +30,19 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[size_t(64) << 20];
 namespace {
 
 using namespace tsp;
+
+// NVTX range for the lifetime of a scope: every entry point and every launch
+// step is named in an Nsight timeline.  Without a tool attached, a push/pop
+// pair is a call through a no-op function pointer.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+#define TSP_CONCAT2(a, b) a##b
+#define TSP_CONCAT(a, b) TSP_CONCAT2(a, b)
+#define TSP_RANGE(name) NvtxRange TSP_CONCAT(tsp_nvtx_range_, __LINE__)(name)
 
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
 constexpr size_t kAlign = 1024;
@@ -207,6 +222,7 @@ int check_weights(const tsp_weights* w, int D) {
 // ---------------------------------------------------------------- launches
 template <typename Tin>
 int launch_layernorm(const Tin* x, __half* y, int64_t rows, int h, float eps, cudaStream_t st) {
+  TSP_RANGE("layernorm");
   if (rows == 0) return TSP_OK;
   if (h >= 1024 && h <= 8192) {  // one row per block
     const dim3 grid(static_cast<unsigned>(rows));
@@ -303,6 +319,7 @@ int pick_bn(int n_block) {
 int b_box_rows(int bn) { return bn == 256 ? 128 : bn; }
 
 int launch_gemm(GemmParams& p, int bn, cudaStream_t st) {
+  TSP_RANGE("gemm");
   if (p.M == 0) return TSP_OK;
   switch (bn) {
     case 256: return launch_gemm_pair(p, st);
@@ -315,6 +332,7 @@ void gemm_common(GemmParams& p, const Sizes& s, int rank, int* status) {
   p.c = static_cast<int>(s.c);
   p.off0 = static_cast<int64_t>(rank) * s.c;                 // chunk r
   p.off1 = static_cast<int64_t>(2 * s.D - 1 - rank) * s.c - s.c;  // chunk 2D-1-r
+  p.remap_rows = s.T;
   p.status = status;
   p.timeout_ns = kDefaultTimeoutNs;
 }
@@ -420,6 +438,7 @@ int launch_ksplit(const Sizes& s, int rank, const __half* a, int Kdim, const voi
 
 int launch_attention(const Sizes& s, int rank, const tsp_dims* dims, const __half* q, const void* k_full,
                      const void* v_full, __half* out, float* lse, int* counter, int* status, cudaStream_t st) {
+  TSP_RANGE("attention");
   if (s.L == 0) return TSP_OK;
   static thread_local AttnParams p;
   std::memset(&p, 0, sizeof(p));
@@ -553,6 +572,7 @@ int launch_attn_bwd_hd(AttnBwdParams& p, cudaStream_t st) {
 int launch_attn_backward(const Sizes& s, int rank, const tsp_dims* dims, const __half* q, const void* k_full,
                          const void* v_full, const __half* o, const float* lse, const __half* d_o, float* dq,
                          float* dk, float* dv, float* delta, int* counter, int* status, cudaStream_t st) {
+  TSP_RANGE("attention_backward");
   if (s.L == 0) return TSP_OK;
   TSP_CUDA(cudaMemsetAsync(dq, 0, static_cast<size_t>(s.L) * s.h * 4, st));
   const dim3 grid_rows(static_cast<unsigned>(s.L));
@@ -653,6 +673,7 @@ int launch_plain(const void* a, int M, int K, int64_t lda, const void* b, int N,
 
 template <typename Tin>
 int launch_transpose(const Tin* in, int64_t rows, int cols, __nv_bfloat16* out, cudaStream_t st) {
+  TSP_RANGE("transpose");
   if (rows == 0) return TSP_OK;
   if (rows % 8 || cols % 8) return TSP_ERR_UNSUPPORTED;
   const dim3 grid(static_cast<unsigned>((rows + 63) / 64), static_cast<unsigned>((cols + 63) / 64));
@@ -664,6 +685,7 @@ int launch_transpose(const Tin* in, int64_t rows, int cols, __nv_bfloat16* out, 
 template <typename Tx, typename Tr>
 int launch_ln_backward(const Tx* y1, const float* g, const Tr* dy, float* dy1, __nv_bfloat16* dy1_bf16, int64_t rows,
                        int h, float eps, cudaStream_t st) {
+  TSP_RANGE("layernorm_backward");
   if (rows == 0) return TSP_OK;
   const int groups = (h + 1023) / 1024;  // groups of 4 values per thread
   const dim3 grid(static_cast<unsigned>(rows));
@@ -936,10 +958,12 @@ int noalloc_scratch(void** out) {
 }
 
 // The status section's two words -> the status a caller sees: a timeout
-// first, then a saturation; anything else in the status word is unknown.
+// first, then a failed debug-build index check, then a saturation; anything
+// else in the status word is unknown.
 int status_of_words(const int (&h)[2]) {
   if (h[0] == TSP_ERR_TIMEOUT) return TSP_ERR_TIMEOUT;
   if (h[0] != 0) return TSP_ERR_CUDA;
+  if (h[1] & kFlagBoundsCheck) return TSP_ERR_BOUNDS;
   return (h[1] & kFlagFp16Saturated) ? TSP_ERR_SATURATED : TSP_OK;
 }
 
@@ -959,6 +983,7 @@ const char* tsp_status_string(int status) {
     case TSP_ERR_TIMEOUT: return "device wait timed out";
     case TSP_ERR_WORKSPACE: return "workspace too small";
     case TSP_ERR_SATURATED: return "fp16 conversion saturated";
+    case TSP_ERR_BOUNDS: return "device index check failed";
     default: return "unknown status";
   }
 }
@@ -968,6 +993,7 @@ const char* tsp_last_cuda_error(void) { return g_cuda_err; }
 int tsp_check_dims(const tsp_dims* dims, int D) { return check_dims(dims, D); }
 
 int tsp_zigzag_index(int64_t T, int D, int rank, int32_t* d_idx, cudaStream_t stream) {
+  TSP_RANGE("tsp_zigzag_index");
   if (D < 1 || D > TSP_MAX_D || rank < 0 || rank >= D || T < 0 || T % (2 * D) != 0) return TSP_ERR_INVALID_ARG;
   if (T >= (int64_t(1) << 31)) return TSP_ERR_UNSUPPORTED;
   const int64_t c = T / (2 * D);
@@ -990,6 +1016,7 @@ size_t tsp_shard_buffer_bytes(const tsp_dims* dims, int D) {
 
 int tsp_pack_shards(const tsp_dims* dims, int D, const void* const w_full[6], void* d_buf, size_t buf_bytes,
                     tsp_weights* out, cudaStream_t stream) {
+  TSP_RANGE("tsp_pack_shards");
   int rc = check_dims(dims, D);
   if (rc) return rc;
   if (!w_full || !d_buf || !out) return TSP_ERR_INVALID_ARG;
@@ -1050,6 +1077,7 @@ size_t tsp_attn_backward_workspace_bytes(const tsp_dims* dims, int D) {
 int tsp_attn_backward(const tsp_dims* dims, int D, int rank, const void* q, const void* k_full, const void* v_full,
                       const void* o, const void* lse, const void* d_o, void* dq, void* dk_full, void* dv_full,
                       void* ws, size_t ws_bytes, cudaStream_t stream) {
+  TSP_RANGE("tsp_attn_backward");
   int rc = check_dims(dims, D);
   if (rc) return rc;
   if (rank < 0 || rank >= D) return TSP_ERR_INVALID_ARG;
@@ -1086,6 +1114,7 @@ int tsp_get_device_status(const void* ws, cudaStream_t stream) {
 
 int tsp_kv_project(const tsp_dims* dims, const tsp_weights* w, int rank, const void* x_local, void* k_full,
                    void* v_full, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  TSP_RANGE("tsp_kv_project");
   Ctx c;
   int rc = make_ctx(c, dims, w, rank, ws, ws_bytes);
   if (rc) return rc;
@@ -1104,6 +1133,7 @@ int tsp_kv_project(const tsp_dims* dims, const tsp_weights* w, int rank, const v
 
 int tsp_kv_project_noalloc(const tsp_dims* dims, const tsp_weights* w, int rank, const void* x_local, void* k_full,
                            void* v_full, cudaStream_t stream) {
+  TSP_RANGE("tsp_kv_project_noalloc");
   const int D = w ? w->D : 0;
   int rc = check_dims(dims, D);
   if (rc) return rc;
@@ -1150,6 +1180,7 @@ int tsp_kv_project_noalloc_status(cudaStream_t stream) {
 int tsp_layer_forward(const tsp_dims* dims, const tsp_weights* w, int rank, const void* x_local, const void* k_full,
                       const void* v_full, void* y_local, int y_dtype, void* ws, size_t ws_bytes, cudaStream_t stream,
                       cudaEvent_t* step_events) {
+  TSP_RANGE("tsp_layer_forward");
   Ctx c;
   int rc = make_ctx(c, dims, w, rank, ws, ws_bytes);
   if (rc) return rc;
@@ -1175,6 +1206,7 @@ int tsp_layer_forward(const tsp_dims* dims, const tsp_weights* w, int rank, cons
 int tsp_rank_step(const tsp_dims* dims, const tsp_weights* w, int rank, const void* x_local, void* k_full,
                   void* v_full, void* y_local, int y_dtype, void* ws, size_t ws_bytes, cudaStream_t stream,
                   cudaEvent_t* step_events) {
+  TSP_RANGE("tsp_rank_step");
   Ctx c;
   int rc = make_ctx(c, dims, w, rank, ws, ws_bytes);
   if (rc) return rc;
@@ -1202,6 +1234,7 @@ int tsp_rank_step(const tsp_dims* dims, const tsp_weights* w, int rank, const vo
 int tsp_rank_step_host(const tsp_dims* dims, const tsp_weights* w, int rank, const void* h_x_local,
                        void* d_x_staging, void* k_full, void* v_full, void* d_y_staging, void* h_y_local, int y_dtype,
                        void* ws, size_t ws_bytes, cudaStream_t stream) {
+  TSP_RANGE("tsp_rank_step_host");
   Ctx c;
   int rc = make_ctx(c, dims, w, rank, ws, ws_bytes);
   if (rc) return rc;
@@ -1228,6 +1261,7 @@ size_t tsp_mlp_backward_workspace_bytes(const tsp_dims* dims, int D) {
 int tsp_mlp_backward(const tsp_dims* dims, const tsp_weights* w, const void* w1_full, const void* w2_full,
                      const void* y1, const void* dy, void* dy1, void* dw1, void* dw2, void* bws, size_t bws_bytes,
                      cudaStream_t stream, cudaEvent_t* ev) {
+  TSP_RANGE("tsp_mlp_backward");
   const int D = w ? w->D : 0;
   int rc = check_dims(dims, D);
   if (rc) return rc;
@@ -1263,6 +1297,7 @@ int tsp_layer_backward(const tsp_dims* dims, const tsp_weights* w, const void* c
                        const void* v_full, const void* dy, void* dx, void* dwq, void* dwo, void* dw1, void* dw2,
                        void* dk_full, void* dv_full, void* bws, size_t bws_bytes, cudaStream_t stream,
                        cudaEvent_t* ev) {
+  TSP_RANGE("tsp_layer_backward");
   const int D = w ? w->D : 0;
   int rc = check_dims(dims, D);
   if (rc) return rc;
@@ -1356,6 +1391,7 @@ int tsp_layer_backward(const tsp_dims* dims, const tsp_weights* w, const void* c
 int tsp_kv_backward(const tsp_dims* dims, int D, const void* const w_full[6], int rank, const void* x_local,
                     const void* dk_full, const void* dv_full, void* dx, void* dwk, void* dwv, void* kws,
                     size_t kws_bytes, cudaStream_t stream) {
+  TSP_RANGE("tsp_kv_backward");
   int rc = check_dims(dims, D);
   if (rc) return rc;
   if (rank < 0 || rank >= D || !w_full) return TSP_ERR_INVALID_ARG;
@@ -1417,6 +1453,7 @@ size_t tsp_tp_workspace_bytes(const tsp_dims* dims, int D) {
 
 int tsp_tp_attention_partial(const tsp_dims* dims, const tsp_weights* w, int k, const void* x, void* part, void* ws,
                              size_t ws_bytes, cudaStream_t stream) {
+  TSP_RANGE("tsp_tp_attention_partial");
   const int D = w ? w->D : 0;
   int rc = check_dims(dims, D);
   if (rc) return rc;
@@ -1464,6 +1501,7 @@ int tsp_tp_attention_partial(const tsp_dims* dims, const tsp_weights* w, int k, 
 
 int tsp_tp_mlp_partial(const tsp_dims* dims, const tsp_weights* w, int k, const void* y1, void* part, void* ws,
                        size_t ws_bytes, cudaStream_t stream) {
+  TSP_RANGE("tsp_tp_mlp_partial");
   const int D = w ? w->D : 0;
   int rc = check_dims(dims, D);
   if (rc) return rc;
@@ -1494,6 +1532,7 @@ int tsp_tp_mlp_partial(const tsp_dims* dims, const tsp_weights* w, int k, const 
 
 int tsp_tp_all_reduce(const tsp_dims* dims, int n_parts, const void* const parts[], const void* resid, int resid_f32,
                       void* out, int out_dtype, cudaStream_t stream) {
+  TSP_RANGE("tsp_tp_all_reduce");
   if (!dims || n_parts < 1 || n_parts > TSP_MAX_D || !parts) return TSP_ERR_INVALID_ARG;
   if (dims->T < 0 || dims->h <= 0 || dims->h % 4) return TSP_ERR_INVALID_ARG;
   if (out_dtype != TSP_OUT_BF16 && out_dtype != TSP_OUT_F32) return TSP_ERR_INVALID_ARG;
@@ -1551,6 +1590,7 @@ int* status_of(void* ws) { return static_cast<int*>(ws); }
 size_t tsp_shard_workspace_bytes(void) { return 2 * kAlign; }
 
 int tsp_layernorm(int64_t rows, int h, float eps, const void* x, int x_f32, void* y, cudaStream_t stream) {
+  TSP_RANGE("tsp_layernorm");
   if (rows < 0 || h <= 0 || h % 8 || h > 8192 || !(eps >= 0.f)) return TSP_ERR_INVALID_ARG;
   if (rows == 0) return TSP_OK;
   if (!ok16({x, y})) return TSP_ERR_INVALID_ARG;
@@ -1561,6 +1601,7 @@ int tsp_layernorm(int64_t rows, int h, float eps, const void* x, int x_f32, void
 
 int tsp_shard_qkv(const tsp_dims* dims, int D, int rank, const void* wq_k, const void* wk_k, const void* wv_k,
                   const void* xn1, void* q_k, void* k_k, void* v_k, void* ws, cudaStream_t stream) {
+  TSP_RANGE("tsp_shard_qkv");
   Sizes s;
   int rc = shard_args(dims, D, rank, &s);
   if (rc) return rc;
@@ -1581,6 +1622,7 @@ int tsp_shard_qkv(const tsp_dims* dims, int D, int rank, const void* wq_k, const
 
 int tsp_shard_attention(const tsp_dims* dims, int D, int rank, const void* q_k, const void* k_k, const void* v_k,
                         void* a_k, void* ws, cudaStream_t stream) {
+  TSP_RANGE("tsp_shard_attention");
   Sizes s;
   int rc = shard_args(dims, D, rank, &s);
   if (rc) return rc;
@@ -1598,6 +1640,7 @@ int tsp_shard_attention(const tsp_dims* dims, int D, int rank, const void* q_k, 
 
 int tsp_shard_ffn_up(const tsp_dims* dims, int D, const void* w1_k, const void* xn2, void* h_k, void* ws,
                      cudaStream_t stream) {
+  TSP_RANGE("tsp_shard_ffn_up");
   Sizes s;
   int rc = shard_args(dims, D, 0, &s);
   if (rc) return rc;
@@ -1616,6 +1659,7 @@ int tsp_shard_ffn_up(const tsp_dims* dims, int D, const void* w1_k, const void* 
 
 int tsp_shard_accumulate(const tsp_dims* dims, int D, const void* act, int k_dim, const void* w_k, void* y,
                          void* ws, cudaStream_t stream) {
+  TSP_RANGE("tsp_shard_accumulate");
   Sizes s;
   int rc = shard_args(dims, D, 0, &s);
   if (rc) return rc;

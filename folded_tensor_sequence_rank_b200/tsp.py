@@ -19,12 +19,14 @@ N_STEP_EVENTS = 8
 N_WS_OFFSETS = 9
 OUT_BF16, OUT_F32 = 0, 1
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "CUDA error",
-          4: "device wait timed out", 5: "workspace too small", 6: "fp16 conversion saturated"}
+          4: "device wait timed out", 5: "workspace too small", 6: "fp16 conversion saturated",
+          7: "device index check failed"}
 (TSP_OK, TSP_ERR_INVALID_ARG, TSP_ERR_UNSUPPORTED, TSP_ERR_CUDA, TSP_ERR_TIMEOUT, TSP_ERR_WORKSPACE,
- TSP_ERR_SATURATED) = range(7)
-DEVICE_STATUSES = (TSP_OK, TSP_ERR_TIMEOUT, TSP_ERR_SATURATED)
+ TSP_ERR_SATURATED, TSP_ERR_BOUNDS) = range(8)
+DEVICE_STATUSES = (TSP_OK, TSP_ERR_TIMEOUT, TSP_ERR_SATURATED, TSP_ERR_BOUNDS)
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtsp_b200.so")
+# TSP_LIBRARY selects another build of the library (the -DTSP_DEBUG one).
+LIB_PATH = os.environ.get("TSP_LIBRARY") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtsp_b200.so")
 WEIGHT_NAMES = ("wq", "wk", "wv", "wo", "w1", "w2")
 
 

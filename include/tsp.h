@@ -48,6 +48,8 @@
  *     device that loads it until exit), whose device address the library
  *     caches per device and CUDA context; that array keeps the last call's
  *     contents, and calls that overlap on the GPU race on it.
+ *   - Every entry point and launch step is an NVTX range (named after the
+ *     call) for Nsight timelines.
  *   - Host-detectable errors are returned synchronously and nothing is
  *     enqueued.  There is no fallback path: an unsupported shape is an
  *     error.  Device-side events are recorded in a status section (a status
@@ -82,9 +84,12 @@ typedef enum {
   TSP_ERR_CUDA = 3,        /* a CUDA runtime call failed; see tsp_last_cuda_error */
   TSP_ERR_TIMEOUT = 4,     /* a bounded wait inside a kernel ran out */
   TSP_ERR_WORKSPACE = 5,   /* workspace or buffer smaller than required */
-  TSP_ERR_SATURATED = 6    /* a value outside fp16's range (|x| > 65504) was
+  TSP_ERR_SATURATED = 6,   /* a value outside fp16's range (|x| > 65504) was
                               clamped to +-65504 on conversion: the results are
                               finite but may be wrong (device status only) */
+  TSP_ERR_BOUNDS = 7       /* an index check of the debug build (compiled with
+                              -DTSP_DEBUG) failed and the access was skipped
+                              (device status only; the normal build has none) */
 } tsp_status;
 
 /* Layer and sequence sizes. */
@@ -177,7 +182,8 @@ int tsp_reset_device_status(void* ws, cudaStream_t stream);
 
 /* Synchronises `stream`, then reads a status section (see
  * tsp_reset_device_status): TSP_ERR_TIMEOUT if a bounded wait ran out, else
- * TSP_ERR_SATURATED if an fp16 conversion saturated, else TSP_OK.  Both are
+ * TSP_ERR_BOUNDS if an index check of the debug build failed, else
+ * TSP_ERR_SATURATED if an fp16 conversion saturated, else TSP_OK.  All are
  * sticky until tsp_reset_device_status. */
 int tsp_get_device_status(const void* ws, cudaStream_t stream);
 

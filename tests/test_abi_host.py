@@ -45,7 +45,7 @@ def test_struct_layouts_match_header():
 
 
 def test_status_strings(L):
-    for code in range(7):
+    for code in range(8):
         assert L.tsp_status_string(code).decode() == tsp.STATUS[code]
 
 
@@ -253,3 +253,14 @@ def test_attn_backward_checks_arguments_first(L):
         assert call(ptrs=ok[:i] + [ok[i] + 8] + ok[i + 1:]) == tsp.TSP_ERR_INVALID_ARG, i
     e = dims(T=0)
     assert L.tsp_attn_backward(ctypes.byref(e), 2, 0, *ok, 256, 1 << 20, None) == tsp.TSP_OK  # no tokens
+
+
+def test_debug_build_exports_the_same_abi():
+    """The -DTSP_DEBUG build (device index checks that report TSP_ERR_BOUNDS)
+    exports every declared function too."""
+    lib = tsp_build.build(debug=True)
+    Ld = ctypes.CDLL(lib)
+    for name in declared_functions():
+        assert hasattr(Ld, name), name
+    Ld.tsp_status_string.restype = ctypes.c_char_p
+    assert Ld.tsp_status_string(tsp.TSP_ERR_BOUNDS).decode() == tsp.STATUS[tsp.TSP_ERR_BOUNDS]
