@@ -280,6 +280,47 @@ def run_reference(args, wl):
 
 # ---------------------------------------------------------------------------- GPU arm
 def run_tsp(args, wl):
+    import gc
+
+    import torch
+    line, world = measure_tsp(args, wl)
+    if line is None:
+        return
+    if world == 1 and not args.no_extras:
+        # the other configurations, measured in the same run on the same GPU
+        gc.collect()
+        torch.cuda.empty_cache()
+        line["other_configs"] = other_configs(args)
+    print(json.dumps(line), flush=True)
+
+
+def other_configs(args):
+    """Configurations 3 and 4, the layer's backward and the 32-layer stack,
+    each measured by its sweep (see run_sweep_*), kept in compact form."""
+    import gc
+
+    import torch
+    out = {}
+    keep = {"ranks": ("config3_all_8_ranks_128k", ["value", "unit", "layer_spread", "kv_project_ms",
+                                                   "layer_forward_ms", "clocks"]),
+            "shards": ("config4_shard_sweep_32k", ["by_D"]),
+            "layer_bwd": ("layer_backward_128k_rank0", ["value", "unit", "ms_per_step", "tflops", "roofline",
+                                                       "part_ms", "clocks"]),
+            "stack": ("stack_32_layers_128k", ["value", "unit", "ms_per_step", "ms_per_layer",
+                                               "peak_device_bytes_this_run", "per_gpu_bytes_on_8_gpus", "clocks"])}
+    fns = {"ranks": run_sweep_ranks, "shards": run_sweep_shards, "layer_bwd": run_sweep_layer_bwd,
+           "stack": run_sweep_stack}
+    for k, (name, fields) in keep.items():
+        sub = argparse.Namespace(**vars(args))
+        sub.workload = "7b-128k-d8"
+        r = fns[k](sub)
+        out[name] = {"metric": r["metric"], **{f: r[f] for f in fields if f in r}}
+        gc.collect()
+        torch.cuda.empty_cache()
+    return out
+
+
+def measure_tsp(args, wl):
     import torch
     import torch.distributed as dist
 
@@ -414,10 +455,12 @@ def run_tsp(args, wl):
         }
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(wl)
-        print(json.dumps(line), flush=True)
+    else:
+        line = None
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+    return line, world
 
 
 STEP_NAMES = ("ln1", "qkv", "attention", "o", "ln2", "w1", "w2")
@@ -499,7 +542,7 @@ def run_sweep_ranks(args):
                        "l2": "inputs larger than L2; no flush"},
             "kv_project_ms": [round(t, 4) for t in kv_ms], "layer_forward_ms": [round(t, 4) for t in fw_ms],
             "layer_spread": (max(fw_ms) - min(fw_ms)) / mean, "clocks": clk}
-    print(json.dumps(line), flush=True)
+    return line
 
 
 def run_sweep_shards(args):
@@ -547,7 +590,7 @@ def run_sweep_shards(args):
             "higher_is_better": True, "dtype": "fp16", "data": "synthetic",
             "config": {"workload": "7B dense layer, T=32768, rank 0, D in {1,2,4,8,16} (seed 4); value is D=8"},
             "by_D": out}
-    print(json.dumps(line), flush=True)
+    return line
 
 
 BWD_NAMES = ["ln2_u", "du", "dxn2", "ln2_bwd", "transposes", "dw1", "dw2"]
@@ -602,7 +645,7 @@ def run_sweep_mlp_bwd(args):
             "part_ms": {k: round(v, 4) for k, v in part.items()},
             "gemm_tflops": {k: round(v, 1) for k, v in rate.items()},
             "clocks": clk}
-    print(json.dumps(line), flush=True)
+    return line
 
 
 LBWD_NAMES = ["mlp_half", "d_a", "d_wo", "attention", "prep_dq_ln1", "d_wq", "d_x"]
@@ -687,7 +730,7 @@ def run_sweep_layer_bwd(args):
                          "peak_source": f"{src} bf16_tflops_sustained",
                          "algorithmic_per_launch": f"{attn_bwd_fl:.4e} FLOP = 10 h x causal pairs"},
             "part_ms": {k: round(v, 4) for k, v in part.items()}, "clocks": clk}
-    print(json.dumps(line), flush=True)
+    return line
 
 
 def run_sweep_tp(args):
@@ -769,7 +812,7 @@ def run_sweep_tp(args):
                                          "tp_with_estimated_comm": T / ((ms["tp_rank"] + comm_ms) * 1e-3)},
             "memory_per_gpu_bytes": {"tsp_one_layer": tsp_acc, "tp_one_layer": tp_acc},
             "clocks": clk}
-    print(json.dumps(line), flush=True)
+    return line
 
 
 def run_sweep_stack(args):
@@ -821,7 +864,7 @@ def run_sweep_stack(args):
             "config": {"workload": "32 x 7B dense layer (random weights per layer), T=131072, D=8, every rank in turn"},
             "peak_device_bytes_this_run": torch.cuda.max_memory_allocated(),
             "per_gpu_bytes_on_8_gpus": acc, "clocks": clk}
-    print(json.dumps(line), flush=True)
+    return line
 
 
 def main():
@@ -832,6 +875,9 @@ def main():
     ap.add_argument("--impl", default="tsp", choices=["tsp", "reference"])
     ap.add_argument("--workload", default="7b-128k-d8", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other configurations (all 8 ranks, the shard sweep, the backward, the stack) "
+                         "that a default 1-GPU run measures after its main line")
     ap.add_argument("--sweep", choices=["ranks", "shards", "stack", "mlp_bwd", "layer_bwd", "tp"], default=None,
                     help="ranks: all 8 ranks of the 128K layer in turn (per-rank spread, whole-layer tokens/s); "
                          "shards: rank 0 at T=32768 for D=1..16; stack: a 32-layer forward at 128K; "
@@ -842,18 +888,10 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
     wl = WORKLOADS[args.workload]
-    if args.sweep == "ranks":
-        run_sweep_ranks(args)
-    elif args.sweep == "shards":
-        run_sweep_shards(args)
-    elif args.sweep == "mlp_bwd":
-        run_sweep_mlp_bwd(args)
-    elif args.sweep == "layer_bwd":
-        run_sweep_layer_bwd(args)
-    elif args.sweep == "tp":
-        run_sweep_tp(args)
-    elif args.sweep == "stack":
-        run_sweep_stack(args)
+    sweeps = {"ranks": run_sweep_ranks, "shards": run_sweep_shards, "mlp_bwd": run_sweep_mlp_bwd,
+              "layer_bwd": run_sweep_layer_bwd, "tp": run_sweep_tp, "stack": run_sweep_stack}
+    if args.sweep is not None:
+        print(json.dumps(sweeps[args.sweep](args)), flush=True)
     elif args.impl == "reference":
         run_reference(args, wl)
     else:
