@@ -41,9 +41,10 @@
 //   into the dP^T columns (SS, both MN-major); the softmax warps read dQ out
 //   of tensor memory (which frees the columns at once) and add it to global
 //   memory: each warp stages its 32 x 32 fp32 blocks in its 4 KiB of the dS^T
-//   buffer and one lane adds each block with a TMA bulk reduction (whole
-//   128-byte lines per L2 operation instead of 16-byte vector reductions);
-//   the next tile's dS^T waits until those reductions have read the staging.
+//   buffer (and a second 4 KiB block at head_dim 128) and one lane adds each
+//   block with a TMA bulk reduction (whole 128-byte lines per L2 operation
+//   instead of 16-byte vector reductions); the next tile's dS^T stores wait
+//   until those reductions have read the staging.
 // Q, K, V, dO, P and dS are fp16 (the forward's operand format); scores,
 // statistics, accumulators and the outputs are fp32.
 #pragma once
@@ -86,10 +87,14 @@ struct AttnBwdShape {
   static constexpr int kStatBytes = kBwdTile * 4;       // lse2 or Delta of one query tile
   static constexpr int kQStages = 2;
   static constexpr int kBarBytes = 512;
-  // K, V, dO, dS^T (128 x 128 whatever the head size), then the Q ring with
-  // its statistics
+  // second staging block per softmax warp (head_dim 128: its 64 columns of a
+  // dQ row are two 32-column blocks; the first is staged in the dS^T buffer)
+  static constexpr int kStage2Bytes = HD == 128 ? 8 * 4096 : 0;
+  // K, V, dO, dS^T (128 x 128 whatever the head size), the Q ring, the second
+  // staging blocks, the Q ring's statistics.  The dynamic shared memory base
+  // is 1024-byte aligned (checked at run time), so no slack is added.
   static constexpr int kSmemBytes =
-      3 * kTileBytes + 32768 + kQStages * (kTileBytes + 2 * kStatBytes) + kBarBytes + 1024;
+      3 * kTileBytes + 32768 + kQStages * kTileBytes + kStage2Bytes + kQStages * 2 * kStatBytes + kBarBytes;
 };
 
 struct BwdQTile {
@@ -129,14 +134,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
   using S = AttnBwdShape<HD>;
   constexpr int NB = HD / 64;  // 64-column boxes per tile row
   constexpr int QST = S::kQStages;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // The 128-byte swizzle needs 1024-byte aligned tiles; the dynamic shared
+  // memory base is (0x400 on this GPU), and the size has no slack for a
+  // misaligned one: such a launch records the failed check and does nothing.
+  if (smem_u32(smem_raw) & 1023) {
+    if (threadIdx.x == 0) atomicOr(p.status + 1, kFlagBoundsCheck);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   uint8_t* sK = smem;
   uint8_t* sV = sK + S::kTileBytes;
   uint8_t* sDO = sV + S::kTileBytes;
   uint8_t* sDS = sDO + S::kTileBytes;  // dS^T [128 keys][128 queries] fp16: always 2 boxes of 64 queries
   uint8_t* sQ = sDS + 32768;           // [QST][kTileBytes]
-  float* sStat = reinterpret_cast<float*>(sQ + QST * S::kTileBytes);  // [QST][lse2 | Delta][128]
+  uint8_t* sStage2 = sQ + QST * S::kTileBytes;  // [8 warps][4 KiB] (head_dim 128)
+  float* sStat = reinterpret_cast<float*>(sStage2 + S::kStage2Bytes);  // [QST][lse2 | Delta][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sStat + QST * 2 * kBwdTile);
   uint64_t* kv_full = bars;           // K, V of the item landed
   uint64_t* kv_empty = kv_full + 1;   // the item's last MMA reading K, V done
@@ -149,7 +162,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
   uint64_t* dv_done = p_full + 1;     // the dV MMA of the tile completed
   uint64_t* dq_full = dv_done + 1;    // dQ of the tile in tensor memory
   uint64_t* dq_free = dq_full + 1;    // dQ read out of tensor memory, 8 warps
-  uint64_t* stg_free = dq_free + 1;   // the staged dQ blocks have been read by their bulk reductions, 8 warps
+  uint64_t* stg_free = dq_free + 1;   // every warp's staged dQ blocks have been read, 8 warps
   uint64_t* dkv_full = stg_free + 1;  // dK, dV of the item complete
   uint64_t* dkv_free = dkv_full + 1;  // dK, dV read out, 8 warps
   uint64_t* it_full = dkv_free + 1;   // [2]
@@ -431,10 +444,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
             P[cc * 16 + i] = pack_half2(pr.x, pr.y);
             dsp[i] = pack_half2(dsv.x, dsv.y);
           }
-          // dS^T row kr, queries col0 .. col0+31: four 16-byte groups; the
-          // buffer held the previous tile's staged dQ until its bulk
-          // reductions had read it
-          if (cc == 0 && tiles > 0 && !warp_wait(stg_free, (tiles - 1) & 1, ctl)) { ok = false; break; }
+          // dS^T row kr, queries col0 .. col0+31: four 16-byte groups.  The
+          // buffer held the previous tile's staged dQ blocks: each warp waits
+          // for its own bulk reductions to have read them, then for every
+          // warp's (deferred to here, so the wait overlaps this softmax)
+          if (cc == 0 && tiles > 0) {
+            if (lane == 0) bulk_wait_group_read0();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(stg_free);
+            if (!warp_wait(stg_free, (tiles - 1) & 1, ctl)) { ok = false; break; }
+          }
           uint8_t* rowp = sDS;
 #pragma unroll
           for (int g = 0; g < 4; ++g)
@@ -467,23 +486,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
           if (q.nvalid == kBwdTile) {
             // whole tile: stage each 32 x 32 block (128-byte swizzled) in this
             // warp's 4 KiB of the dS^T buffer - free: the dQ MMA has read it -
-            // and add it with one bulk reduction
-            uint8_t* stg = sDS + (warp - 2) * 4096;
+            // and, at head_dim 128, in its second block; one bulk reduction
+            // adds each.  The reads of the staging are waited for just before
+            // the next tile's dS^T stores.
 #pragma unroll
             for (int j = 0; j < HD / 64; ++j) {
+              uint8_t* stg = j == 0 ? sDS + (warp - 2) * 4096 : sStage2 + (warp - 2) * 4096;
 #pragma unroll
               for (int c = 0; c < 8; ++c)
                 *reinterpret_cast<uint4*>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
                     make_uint4(r[32 * j + 4 * c], r[32 * j + 4 * c + 1], r[32 * j + 4 * c + 2], r[32 * j + 4 * c + 3]);
-              fence_proxy_async_smem();
-              __syncwarp();
-              if (lane == 0 && dbg_ok(q.m0 + quarter * 32 + 32 <= 2 * p.c && (head + 1) * HD <= p.ld, p.status)) {
-                tma_reduce_add_2d(&p.map_dq, stg, head * HD + half * (HD / 2) + 32 * j, q.m0 + quarter * 32);
-                bulk_commit_group();
-                bulk_wait_group_read0();
-              }
-              __syncwarp();
             }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && dbg_ok(q.m0 + quarter * 32 + 32 <= 2 * p.c && (head + 1) * HD <= p.ld, p.status)) {
+#pragma unroll
+              for (int j = 0; j < HD / 64; ++j)
+                tma_reduce_add_2d(&p.map_dq, j == 0 ? sDS + (warp - 2) * 4096 : sStage2 + (warp - 2) * 4096,
+                                  head * HD + half * (HD / 2) + 32 * j, q.m0 + quarter * 32);
+              bulk_commit_group();
+            }
+            __syncwarp();
           } else {
             // a ragged tile (the last of a chunk whose length is not a multiple
             // of 128): rows past the chunk are skipped, one vector reduction
@@ -498,8 +521,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
                                       __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3])));
             }
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(stg_free);
         }
         qph[qs] ^= 1;
         if (++qs == QST) qs = 0;
@@ -541,6 +562,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
     }
   }
 
+  // the CTA outlives the reads of its last bulk reductions
+  if (warp >= 2 && lane == 0) bulk_wait_group_read0();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
