@@ -205,6 +205,43 @@ def test_attention_backward_128k_sampled():
     assert not dK[(2 * D) * c:].any() and not dV[(2 * D) * c:].any()
 
 
+def test_attention_backward_32k_d16_sampled():
+    """Rank 5 of 16 at T = 32768 (c = 1024; head groups of two heads): dQ on
+    sampled rows of both chunks, computed alone by the oracle."""
+    T, h, H, F, D, r, seed = 32768, 4096, 32, 16384, 16, 5, 13
+    L = T // D
+    c = L // 2
+    raw = inputs.rank_inputs(L, T, h, F, seed)
+    dev = {k: v.cuda() for k, v in raw.items()}
+    dims = tsp.make_dims(T, h, H, F)
+    sw = tsp.pack_shards(dims, D, dev)
+    ws = tsp.alloc_workspace(dims, D)
+    aws = tsp.alloc_attn_backward_workspace(dims, D)
+    y = torch.empty(L, h, dtype=torch.float32, device="cuda")
+    tsp.layer_forward(dims, sw, r, dev["x_local"], dev["k_full"], dev["v_full"], y, ws)
+    q = tsp.workspace_view(ws, dims, D, "q")
+    a = tsp.workspace_view(ws, dims, D, "a")
+    d_o = inputs.attention_grad_inputs(L, h, seed).cuda()
+    dq = torch.empty(L, h, dtype=torch.float32, device="cuda")
+    dK = torch.zeros(T, h, dtype=torch.float32, device="cuda")
+    dV = torch.zeros_like(dK)
+    tsp.attn_backward(dims, D, r, q, dev["k_full"], dev["v_full"], a, tsp.workspace_view(ws, dims, D, "lse"), d_o, dq,
+                      dK, dV, aws)
+    assert tsp.get_device_status(aws) == tsp.TSP_OK
+    s = dims.softmax_scale
+    rows = inputs.sample_rows(L, 12, seed, must=(0, c - 1, c, L - 1))
+    pos = O.zigzag_index(T, D, r)[rows]
+    Kf, Vf = raw["k_full"].double().numpy(), raw["v_full"].double().numpy()
+    qs, as_, dos = f64(q[rows]), f64(a[rows]), f64(d_o[rows])
+    dq_ref, _, _ = O.attention_backward_stored(qs, Kf, Vf, as_, pos, dos, H, s)
+    close("dq rows", f64(dq[rows]), dq_ref, 1e-3, 1e-2)
+    dq0, _, _ = O.causal_attention_backward(qs, Kf, Vf, pos, dos, H, s)
+    close("dq rows vs plain", f64(dq[rows]), dq0, 1e-2, 3e-2)
+    # keys past the rank's last position get nothing
+    last = (2 * D - r) * c
+    assert not dK[last:].any() and not dV[last:].any()
+
+
 def test_zero_gradient_gives_zeros():
     """dA = 0: dQ, dK and dV are exactly zero."""
     T, h, H, F, D = 512, 256, 4, 1024, 2

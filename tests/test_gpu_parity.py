@@ -337,6 +337,45 @@ def test_7b_layer_128k_middle_ranks_sampled():
     sampled_rank_check(131072, 8, [1, 2, 3, 4, 5, 6], 3, n_sample=16)
 
 
+def test_7b_layer_128k_kv_from_projection_sampled():
+    """The whole 128K layer as the all-ranks configuration runs it: every rank's
+    tsp_kv_project fills K and V over all 131072 tokens, then ranks 0 and 5 run
+    their layer forward on those K/V; sampled rows of both are checked against
+    the oracle, which projects K and V of the whole sequence itself (fp64,
+    ~9 TFLOP of CPU work, the slowest check here)."""
+    T, D, seed = 131072, 8, 3
+    L = T // D
+    c = L // 2
+    raw = inputs.layer_inputs(T, h7, F7, seed)
+    dev = to_cuda(raw)
+    dims = tsp.make_dims(T, h7, H7, F7)
+    sw = tsp.pack_shards(dims, D, dev)
+    ws = tsp.alloc_workspace(dims, D)
+    K = torch.zeros(T, h7, dtype=torch.float16, device="cuda")
+    V = torch.zeros_like(K)
+    xs = [dev["x"].index_select(0, tsp.zigzag_index(T, D, r).long()).contiguous() for r in range(D)]
+    for r in range(D):
+        tsp.kv_project(dims, sw, r, xs[r], K, V, ws)
+    got = {}
+    for r in (0, 5):
+        y = torch.empty(L, h7, dtype=torch.float32, device="cuda")
+        tsp.layer_forward(dims, sw, r, xs[r], K, V, y, ws)
+        rows = inputs.sample_rows(L, 12, seed + r, must=(0, c - 1, c, L - 1))
+        got[r] = (rows, f64(y[rows]))
+    assert tsp.get_device_status(ws) == tsp.TSP_OK
+    del K, V, dev, ws, sw, xs
+    torch.cuda.empty_cache()
+    x = f64(raw["x"])
+    for storage in ("fp16", None):
+        w = O.stored_weights(weights_f64(raw), storage)
+        Kr, Vr = O.kv_project(x, w, storage=storage)
+        for r, (rows, y_s) in got.items():
+            pos = O.zigzag_index(T, D, r)[rows]
+            ref = O.rank_rows_forward(x[pos], pos, Kr, Vr, w, H7, storage=storage)
+            assert_layer_close(y_s, ref["y"], f"128K rank {r}, K/V projected by every rank, oracle {storage}", x[pos])
+        del Kr, Vr
+
+
 @pytest.mark.parametrize("D", [1, 2, 4, 8, 16])
 def test_7b_layer_T32768_shard_sweep_sampled(D):
     sampled_rank_check(32768, D, [0], 4, n_sample=30)
