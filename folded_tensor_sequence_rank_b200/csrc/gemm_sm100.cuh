@@ -31,19 +31,19 @@ constexpr int kGemmThreads = 192;
 constexpr int kGemmMaxMaps = 48;  // 3 segments x 16 shards
 constexpr int kGemmGroupM = 16;   // M tiles per raster group (L2 reuse of A)
 
-// Epilogues.  kEpiStoreBf16 / kEpiGeluBf16 write fp16 operands for the next
-// matmul (the names keep the 16-bit operand role), saturating at +-65504 and
+// Epilogues.  kEpiStoreF16 / kEpiGeluF16 write fp16 operands for the next
+// matmul, saturating at +-65504 and
 // setting kFlagFp16Saturated in the flags word after `status` when a value
 // was out of range; kEpiResidual adds the
 // residual stream; kEpiGeluBwd writes the bf16 gradient acc * GELU'(U) with U
 // (fp16, [M, ldo]) at `resid`; kEpiStoreF32 writes acc as fp32.
-// kEpiStoreBf16 and kEpiGeluBwd can also write the tile transposed, as bf16,
-// to out_t [N, ld_t] (row n, column m): kEpiStoreBf16 writes GELU of the
+// kEpiStoreF16 and kEpiGeluBwd can also write the tile transposed, as bf16,
+// to out_t [N, ld_t] (row n, column m): kEpiStoreF16 writes GELU of the
 // fp16-rounded value there, kEpiGeluBwd the gradient itself.  A warp holds 32
 // consecutive rows; it transposes each 32 x 32 chunk through its own slice of
 // shared memory, so every lane writes one 64-byte output row segment.  The
 // transposed store needs every lane of the warp (M a multiple of 128).
-enum GemmEpi : int { kEpiStoreBf16 = 0, kEpiGeluBf16 = 1, kEpiResidual = 2, kEpiGeluBwd = 3, kEpiStoreF32 = 4 };
+enum GemmEpi : int { kEpiStoreF16 = 0, kEpiGeluF16 = 1, kEpiResidual = 2, kEpiGeluBwd = 3, kEpiStoreF32 = 4 };
 
 struct __align__(64) GemmParams {
   CUtensorMap map_a;
@@ -257,7 +257,7 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const GemmParams& p, int m, 
       return;
     uint32_t packed[16];
     float mx = 0.f;  // largest magnitude converted: flags a saturation
-    if (p.epi == kEpiGeluBf16) {
+    if (p.epi == kEpiGeluF16) {
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const float a = gelu_tanh_f(__uint_as_float(r[2 * i])), b = gelu_tanh_f(__uint_as_float(r[2 * i + 1]));

@@ -542,7 +542,7 @@ int layer_tail(Ctx& c, const tsp_dims* dims, const tsp_weights* w, int rank, con
   const void* const* w1fam[3] = {reinterpret_cast<const void* const*>(w->w1), nullptr, nullptr};
   void* hout[3] = {c.hbuf, nullptr, nullptr};
   const int noremap[3] = {0, 0, 0};
-  rc = launch_proj(s, rank, c.xn, w1fam, hout, noremap, 1, kEpiGeluBf16, s.F, c.status, st);
+  rc = launch_proj(s, rank, c.xn, w1fam, hout, noremap, 1, kEpiGeluF16, s.F, c.status, st);
   if (rc) return rc;
   if ((rc = record(ev, 6, st))) return rc;
   rc = launch_ksplit(s, rank, c.hbuf, s.F, reinterpret_cast<const void* const*>(w->w2), c.y1, 1, y_local,
@@ -744,7 +744,7 @@ int mlp_backward_core(const Sizes& s, const tsp_dims* dims, const tsp_weights* w
   const void* const* w1fam[3] = {reinterpret_cast<const void* const*>(w->w1), nullptr, nullptr};
   void* uout[3] = {u, nullptr, nullptr};
   const int noremap[3] = {0, 0, 0};
-  rc = launch_proj(s, 0, xn2, w1fam, uout, noremap, 1, kEpiStoreBf16, s.F, status, stream, ht);
+  rc = launch_proj(s, 0, xn2, w1fam, uout, noremap, 1, kEpiStoreF16, s.F, status, stream, ht);
   if (rc) return rc;
   if ((rc = record(ev, 1, stream))) return rc;
   // dU = (dY W2^T) * GELU'(U): B = W2 [F, h] is K-major over h; the
@@ -1128,7 +1128,7 @@ int tsp_kv_project(const tsp_dims* dims, const tsp_weights* w, int rank, const v
                                reinterpret_cast<const void* const*>(w->wv), nullptr};
   void* out[3] = {k_full, v_full, nullptr};
   const int remap[3] = {1, 1, 0};
-  return launch_proj(c.s, rank, c.xn, fam, out, remap, 2, kEpiStoreBf16, c.s.h, c.status, stream);
+  return launch_proj(c.s, rank, c.xn, fam, out, remap, 2, kEpiStoreF16, c.s.h, c.status, stream);
 }
 
 int tsp_kv_project_noalloc(const tsp_dims* dims, const tsp_weights* w, int rank, const void* x_local, void* k_full,
@@ -1164,7 +1164,7 @@ int tsp_kv_project_noalloc(const tsp_dims* dims, const tsp_weights* w, int rank,
                                reinterpret_cast<const void* const*>(w->wv), nullptr};
   void* out[3] = {k_full, v_full, nullptr};
   const int remap[3] = {1, 1, 0};
-  return launch_proj(sz, rank, xn, fam, out, remap, 2, kEpiStoreBf16, sz.h, status, stream);
+  return launch_proj(sz, rank, xn, fam, out, remap, 2, kEpiStoreF16, sz.h, status, stream);
 }
 
 int tsp_kv_project_noalloc_status(cudaStream_t stream) {
@@ -1197,7 +1197,7 @@ int tsp_layer_forward(const tsp_dims* dims, const tsp_weights* w, int rank, cons
   const void* const* fam[3] = {reinterpret_cast<const void* const*>(w->wq), nullptr, nullptr};
   void* out[3] = {c.q, nullptr, nullptr};
   const int remap[3] = {0, 0, 0};
-  rc = launch_proj(c.s, rank, c.xn, fam, out, remap, 1, kEpiStoreBf16, c.s.h, c.status, stream);
+  rc = launch_proj(c.s, rank, c.xn, fam, out, remap, 1, kEpiStoreF16, c.s.h, c.status, stream);
   if (rc) return rc;
   if ((rc = record(step_events, 2, stream))) return rc;
   return layer_tail(c, dims, w, rank, x_local, k_full, v_full, y_local, y_dtype, stream, step_events);
@@ -1225,7 +1225,7 @@ int tsp_rank_step(const tsp_dims* dims, const tsp_weights* w, int rank, const vo
                                reinterpret_cast<const void* const*>(w->wv)};
   void* out[3] = {c.q, k_full, v_full};
   const int remap[3] = {0, 1, 1};
-  rc = launch_proj(c.s, rank, c.xn, fam, out, remap, 3, kEpiStoreBf16, c.s.h, c.status, stream);
+  rc = launch_proj(c.s, rank, c.xn, fam, out, remap, 3, kEpiStoreF16, c.s.h, c.status, stream);
   if (rc) return rc;
   if ((rc = record(step_events, 2, stream))) return rc;
   return layer_tail(c, dims, w, rank, x_local, k_full, v_full, y_local, y_dtype, stream, step_events);
@@ -1353,7 +1353,7 @@ int tsp_layer_backward(const tsp_dims* dims, const tsp_weights* w, const void* c
   if ((rc = record(ev, 1, stream))) return rc;
   // dA = dY1 Wo^T (Wo [h_in, h_out] row-major is K-major over h_out), fp16 for
   // the attention backward's tensor cores
-  rc = launch_plain(dy1b, L, s.h, s.h, w_full[3], s.h, s.h, true, kEpiStoreBf16, d_o, s.h, nullptr, status, stream);
+  rc = launch_plain(dy1b, L, s.h, s.h, w_full[3], s.h, s.h, true, kEpiStoreF16, d_o, s.h, nullptr, status, stream);
   if (rc) return rc;
   if ((rc = record(ev, 2, stream))) return rc;
   // dWo = A^T dY1: both operands token-major
@@ -1482,7 +1482,7 @@ int tsp_tp_attention_partial(const tsp_dims* dims, const tsp_weights* w, int k, 
                                reinterpret_cast<const void* const*>(&w->wv[k])};
   void* out[3] = {q, kk, v};
   const int noremap[3] = {0, 0, 0};
-  rc = launch_proj(full, 0, xn, fam, out, noremap, 3, kEpiStoreBf16, s.hs, status, stream);
+  rc = launch_proj(full, 0, xn, fam, out, noremap, 3, kEpiStoreF16, s.hs, status, stream);
   if (rc) return rc;
   // causal attention of head group k over the whole sequence
   tsp_dims dk = *dims;
@@ -1524,7 +1524,7 @@ int tsp_tp_mlp_partial(const tsp_dims* dims, const tsp_weights* w, int k, const 
   const void* const* fam[3] = {reinterpret_cast<const void* const*>(&w->w1[k]), nullptr, nullptr};
   void* out[3] = {hb, nullptr, nullptr};
   const int noremap[3] = {0, 0, 0};
-  rc = launch_proj(full, 0, xn, fam, out, noremap, 1, kEpiGeluBf16, s.Fs, status, stream);
+  rc = launch_proj(full, 0, xn, fam, out, noremap, 1, kEpiGeluF16, s.Fs, status, stream);
   if (rc) return rc;
   return launch_plain(hb, static_cast<int>(s.T), s.Fs, s.Fs, w->w2[k], s.h, s.Fs, false, kEpiStoreF32, part, s.h,
                       nullptr, status, stream);
@@ -1616,7 +1616,7 @@ int tsp_shard_qkv(const tsp_dims* dims, int D, int rank, const void* wq_k, const
   const int remap[3] = {0, 1, 1};  // K, V rows to their global positions
   Sizes one = s;
   one.D = 1;  // one shard per segment; the zigzag rows still follow (rank, D)
-  return launch_proj_zz(s, one, rank, static_cast<const __half*>(xn1), fam, out, remap, 3, kEpiStoreBf16, s.hs,
+  return launch_proj_zz(s, one, rank, static_cast<const __half*>(xn1), fam, out, remap, 3, kEpiStoreF16, s.hs,
                         status_of(ws), stream);
 }
 
@@ -1653,7 +1653,7 @@ int tsp_shard_ffn_up(const tsp_dims* dims, int D, const void* w1_k, const void* 
   const int noremap[3] = {0, 0, 0};
   Sizes one = s;
   one.D = 1;
-  return launch_proj_zz(s, one, 0, static_cast<const __half*>(xn2), fam, out, noremap, 1, kEpiGeluBf16, s.Fs,
+  return launch_proj_zz(s, one, 0, static_cast<const __half*>(xn2), fam, out, noremap, 1, kEpiGeluF16, s.Fs,
                         status_of(ws), stream);
 }
 
