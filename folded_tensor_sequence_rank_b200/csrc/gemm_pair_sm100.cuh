@@ -22,6 +22,13 @@
 //   warp 0     TMA producer (this CTA's A rows and B half)
 //   warp 1     TMEM allocator (pair allocation); even CTA: MMA issuer
 //   warps 2-5  epilogue of this CTA's 128 rows (TMEM lane quarters 2,3,0,1)
+//
+// Residual epilogues (the K-split GEMMs' output plus the residual stream)
+// stage each warp's 32 x 32 output blocks in shared memory and write them with
+// tensor stores, whole 128- or 64-byte rows at a time, instead of a lane per
+// row storing 16 bytes to 32 different rows per instruction (which made the
+// O projection at 16384 x 4096 x 4096 about 7% slower).  A warp whose rows
+// run past M keeps the per-lane stores.
 #pragma once
 #include "gemm_sm100.cuh"
 #include "ptx.cuh"
@@ -37,7 +44,13 @@ struct GemmPairShape {
   static constexpr int kStages = 6;
   static constexpr int kTmemCols = 2 * kPairBN;  // two accumulators of 256 columns
   static constexpr int kBarBytes = 256;
-  static constexpr int kSmemBytes = kStages * (kABytes + kBBytes) + kBarBytes + kStageBytes + 1024;
+  // per epilogue warp 8 KiB: two 4 KiB staging buffers of the tensor-store
+  // epilogue, or the transpose buffer of the transposed bf16 stores
+  static constexpr int kEpiWarpBytes = 8192;
+  static constexpr int kEpiBytes = 4 * kEpiWarpBytes;
+  static constexpr int kSmemBytes = kStages * (kABytes + kBBytes) + kEpiBytes + kBarBytes + 1024;
+  static_assert(kStageWords * 4 <= kEpiWarpBytes, "transpose buffer fits the warp's staging");
+  static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
 };
 
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_pair_f16_tcgen05(const __grid_constant__ GemmParams p) {
@@ -47,7 +60,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_pair_f16_tcgen05(const _
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * S::kABytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * S::kBBytes);
+  uint8_t* sEpi = sB + STAGES * S::kBBytes;  // 1024-byte aligned
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + S::kEpiBytes);
   uint64_t* full = bars;               // [STAGES] even CTA: both CTAs' tiles landed
   uint64_t* empty = full + STAGES;     // [STAGES] both CTAs: MMAs done with the stage
   uint64_t* tfull = empty + STAGES;    // [2] both CTAs: accumulator holds a finished tile
@@ -164,9 +178,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_pair_f16_tcgen05(const _
   } else {
     // epilogue warps 2..5 -> TMEM lane quarters 2,3,0,1 of this CTA's 128 rows
     const int quarter = warp & 3;
-    uint32_t* stage = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(bars) + S::kBarBytes) +
-                      (warp - 2) * kStageWords;  // this warp's transpose buffer
+    uint8_t* wstage = sEpi + (warp - 2) * S::kEpiWarpBytes;  // this warp's staging
+    uint32_t* stage = reinterpret_cast<uint32_t*>(wstage);     // as the transpose buffer
     const int row = quarter * 32 + lane;
+    int staged = 0;  // tensor-store blocks this warp has issued: picks the buffer
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     int acc = 0;
     for (int tile = pair; tile < num_tiles; tile += npairs, ++acc) {
@@ -178,6 +193,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_pair_f16_tcgen05(const _
       tc_fence_after();
       const int m = mb * kPairBM + 128 * static_cast<int>(cta) + row;
       const bool valid = m < p.M;
+      // the warp's 32 rows go out by tensor stores when they all exist
+      const int m0w = m - lane;
+      const bool tma_rows = p.tma_out && m0w + 32 <= p.M;
       const int64_t grow = (m < p.c) ? (p.off0 + m) : (p.off1 + m);
       // Software-pipelined over the 32-column chunks: the next chunk's
       // accumulators (and its U values or residual) are loaded while this
@@ -198,7 +216,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_pair_f16_tcgen05(const _
           tmem_ld32(tmem_base + lane_off + buf * kPairBN + (ch + 1) * 32, rn);
           if (aux_on) load_epilogue_aux(p, m, nb * kPairBN + (ch + 1) * 32, auxn);
         }
-        if (valid) gemm_epilogue_chunk(p, m, grow, nb * kPairBN + ch * 32, r, aux, stage);
+        if (tma_rows)
+          residual_chunk_tma(p, m0w, nb * kPairBN + ch * 32, r, aux, wstage + (staged++ & 1) * 4096);
+        else if (valid)
+          gemm_epilogue_chunk(p, m, grow, nb * kPairBN + ch * 32, r, aux, stage);
         if (ch + 1 < kChunks) {
           tmem_ld_wait();
           reg_fence32(rn);  // no use of rn before the wait
@@ -212,6 +233,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_pair_f16_tcgen05(const _
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));
     }
+    // the tensor stores have read the staging and written the output before
+    // the CTA's shared memory is released
+    if (lane == 0 && staged) bulk_wait_group0();
   }
 
   // the MMA issuer may still write the odd CTA's tensor memory, and the odd

@@ -48,6 +48,8 @@ enum GemmEpi : int { kEpiStoreF16 = 0, kEpiGeluF16 = 1, kEpiResidual = 2, kEpiGe
 struct __align__(64) GemmParams {
   CUtensorMap map_a;
   CUtensorMap map_b[kGemmMaxMaps];
+  CUtensorMap map_out;  // pair kernel, kEpiResidual with tma_out: the output as a store destination
+  int tma_out;
   int M, N, K;
   int ksplit;     // 0: N-split, 1: K-split
   int shard_n;    // N-split: output columns per B map
@@ -176,6 +178,74 @@ __device__ __forceinline__ void load_epilogue_aux(const GemmParams& p, int m, in
   }
 }
 
+// kEpiResidual: accumulator values r plus the residual held in aux (fp32 or
+// bf16), for one row's 32-column chunk.
+__device__ __forceinline__ void residual_add(const GemmParams& p, const uint32_t (&r)[32], const uint4 (&aux)[8],
+                                             float (&v)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  if (p.resid_f32) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint4 q = aux[i];
+      v[4 * i] += __uint_as_float(q.x); v[4 * i + 1] += __uint_as_float(q.y);
+      v[4 * i + 2] += __uint_as_float(q.z); v[4 * i + 3] += __uint_as_float(q.w);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 q = aux[i];
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&w[j]);
+        const float2 f = __bfloat1622float2(b2);
+        v[8 * i + 2 * j] += f.x;
+        v[8 * i + 2 * j + 1] += f.y;
+      }
+    }
+  }
+}
+
+// One 32 x 32 block of a residual epilogue - a warp's rows m0 .. m0+31 (lane
+// = row), columns n .. n+31 - written by a tensor store.  Each lane puts its
+// row into `buf` (4 KiB, 1024-byte aligned) in the layout of p.map_out's
+// swizzle: 16-byte piece j of row i at piece j ^ (i & 7) of a 128-byte row
+// (fp32) or j ^ ((i >> 1) & 3) of a 64-byte row (bf16), so eight consecutive
+// lanes cover all 32 banks.  Lane 0 then stores the box.  The caller
+// alternates two buffers per warp: before refilling one, lane 0 waits until
+// at most its latest store (the other buffer's) is still reading.  The block
+// lies wholly inside the output.
+__device__ __forceinline__ void residual_chunk_tma(const GemmParams& p, int m0, int n, const uint32_t (&r)[32],
+                                                   const uint4 (&aux)[8], uint8_t* buf) {
+  const int lane = threadIdx.x & 31;
+  if (!dbg_ok(m0 >= 0 && m0 + 32 <= p.M && n + 32 <= p.N, p.status)) return;
+  float v[32];
+  residual_add(p, r, aux, v);
+  if (lane == 0) bulk_wait_group_read1();
+  __syncwarp();
+  if (p.out_f32) {
+    uint8_t* row = buf + lane * 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      *reinterpret_cast<float4*>(row + ((j ^ (lane & 7)) << 4)) =
+          make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  } else {
+    uint8_t* row = buf + lane * 64;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      *reinterpret_cast<uint4*>(row + ((j ^ ((lane >> 1) & 3)) << 4)) =
+          make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                     pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(&p.map_out, buf, n, m0);
+    bulk_commit_group();
+  }
+}
+
 // One 32-column chunk of an output tile's epilogue: accumulator values r for
 // local row m (global zigzag row grow) and output columns n .. n+31.
 __device__ __forceinline__ void gemm_epilogue_chunk(const GemmParams& p, int m, int64_t grow, int n,
@@ -214,30 +284,8 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const GemmParams& p, int m, 
   }
   if (p.epi == kEpiResidual) {
     float v[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+    residual_add(p, r, aux, v);
     const int64_t off = static_cast<int64_t>(m) * p.ldo + n;
-    if (p.resid_f32) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint4 q = aux[i];
-        v[4 * i] += __uint_as_float(q.x); v[4 * i + 1] += __uint_as_float(q.y);
-        v[4 * i + 2] += __uint_as_float(q.z); v[4 * i + 3] += __uint_as_float(q.w);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 q = aux[i];
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&w[j]);
-          const float2 f = __bfloat1622float2(b2);
-          v[8 * i + 2 * j] += f.x;
-          v[8 * i + 2 * j + 1] += f.y;
-        }
-      }
-    }
     if (p.out_f32) {
       float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out[0]) + off);
 #pragma unroll

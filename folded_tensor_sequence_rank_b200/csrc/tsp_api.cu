@@ -122,6 +122,30 @@ int make_map_f32(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int64_t
   return TSP_OK;
 }
 
+// The output of a residual epilogue as the destination of tensor stores:
+// [rows, cols] row-major with row stride ld elements, fp32 (32 x 32 boxes of
+// 128-byte rows, 128B swizzle) or bf16 (32 x 32 boxes of 64-byte rows, 64B
+// swizzle).
+int make_map_store(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int64_t ld, bool f32) {
+  auto fn = encode_fn();
+  if (!fn) {
+    std::snprintf(g_cuda_err, sizeof(g_cuda_err), "cuTensorMapEncodeTiled unavailable");
+    return TSP_ERR_CUDA;
+  }
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * (f32 ? 4 : 2)};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_cuda_err, sizeof(g_cuda_err), "cuTensorMapEncodeTiled (store) failed (%d)", static_cast<int>(r));
+    return TSP_ERR_CUDA;
+  }
+  return TSP_OK;
+}
+
 int num_sms() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -289,6 +313,13 @@ int launch_gemm_pair(GemmParams& p, cudaStream_t st) {
   if (max_clusters <= 0) {
     std::snprintf(g_cuda_err, sizeof(g_cuda_err), "no CTA pair of the GEMM kernel fits on this GPU");
     return TSP_ERR_CUDA;
+  }
+  // residual epilogues write through tensor stores when the output allows them
+  p.tma_out = 0;
+  if (p.epi == kEpiResidual && aligned16(p.out[0]) && (p.ldo * (p.out_f32 ? 4 : 2)) % 16 == 0 && p.N % 32 == 0) {
+    const int rc = make_map_store(&p.map_out, p.out[0], p.M, p.N, p.ldo, p.out_f32 != 0);
+    if (rc) return rc;
+    p.tma_out = 1;
   }
   const int tiles = ((p.M + kPairBM - 1) / kPairBM) * (p.N / kPairBN);
   const int pairs = tiles < max_clusters ? tiles : max_clusters;
