@@ -815,6 +815,212 @@ def run_sweep_tp(args):
     return line
 
 
+def _attn_lib_impls(q, a, d_o, K, V, c, kv_len, H, hd, scale, which):
+    """Library attention kernels on the rank's two requests (chunk r against
+    keys [0, c) and chunk 2D-1-r against keys [0, (2D-r) c), bottom-right
+    causal masks), as {name: (forward fn, backward fn or None, info)}.  A
+    library that is missing or refuses the shape is reported, not fatal."""
+    import torch
+    L, h = q.shape
+    out = {}
+
+    def bhsd(t, S):  # [S, h] row-major -> [1, H, S, hd]
+        return t.view(1, S, H, hd).permute(0, 2, 1, 3)
+
+    def new_bhsd(S):
+        return torch.empty(1, S, H, hd, dtype=torch.float16, device="cuda").permute(0, 2, 1, 3)
+
+    if "cudnn" in which:
+        try:
+            import cudnn
+            handle = cudnn.create_handle()
+            cudnn.set_stream(handle=handle, stream=torch.cuda.current_stream().cuda_stream)
+            DT = cudnn.data_type
+
+            def built(g):
+                g.validate()
+                g.build_operation_graph()
+                g.create_execution_plans([cudnn.heur_mode.A, cudnn.heur_mode.FALLBACK])
+                g.check_support()
+                g.build_plans()
+                return torch.empty(max(g.get_workspace_size(), 1), dtype=torch.uint8, device="cuda")
+
+            def graph():
+                return cudnn.pygraph(io_data_type=DT.HALF, intermediate_data_type=DT.FLOAT,
+                                     compute_data_type=DT.FLOAT, handle=handle)
+            fwd, bwd, outs = [], [], []
+            for q0, skv in ((0, kv_len[0]), (c, kv_len[1])):
+                qt, kt, vt = bhsd(q[q0:q0 + c], c), bhsd(K[:skv], skv), bhsd(V[:skv], skv)
+                ot, st = new_bhsd(c), torch.empty(1, H, c, 1, dtype=torch.float32, device="cuda")
+                g = graph()
+                tq, tk, tv = g.tensor_like(qt), g.tensor_like(kt), g.tensor_like(vt)
+                to, tst = g.sdpa(name="sdpa", q=tq, k=tk, v=tv, generate_stats=True, attn_scale=scale,
+                                 use_causal_mask_bottom_right=True)
+                to.set_output(True).set_dim(list(ot.shape)).set_stride(list(ot.stride()))
+                tst.set_output(True).set_data_type(DT.FLOAT).set_dim(list(st.shape)).set_stride(list(st.stride()))
+                fwd.append((g, {tq: qt, tk: kt, tv: vt, to: ot, tst: st}, built(g)))
+                outs.append(ot)
+                dot = bhsd(d_o[q0:q0 + c], c)
+                dqt, dkt, dvt = new_bhsd(c), new_bhsd(skv), new_bhsd(skv)
+                g = graph()
+                tq, tk, tv, to, tdo, tst = (g.tensor_like(x) for x in (qt, kt, vt, ot, dot, st))
+                tdq, tdk, tdv = g.sdpa_backward(name="sdpa_backward", q=tq, k=tk, v=tv, o=to, dO=tdo, stats=tst,
+                                                attn_scale=scale, use_causal_mask_bottom_right=True)
+                for t, x in ((tdq, dqt), (tdk, dkt), (tdv, dvt)):
+                    t.set_output(True).set_dim(list(x.shape)).set_stride(list(x.stride()))
+                bwd.append((g, {tq: qt, tk: kt, tv: vt, to: ot, tdo: dot, tst: st, tdq: dqt, tdk: dkt, tdv: dvt},
+                            built(g)))
+
+            def run(gs):
+                for g, m, w in gs:
+                    g.execute(m, w, handle=handle)
+            out["cudnn"] = (lambda: run(fwd), lambda: run(bwd),
+                            {"version": cudnn.backend_version(),
+                             "o": lambda: torch.cat([x.permute(0, 2, 1, 3).reshape(c, h) for x in outs])})
+        except Exception as ex:  # noqa: BLE001 - report any library refusal
+            out["cudnn"] = (None, None, {"error": repr(ex)[:300]})
+    kcat = vcat = None
+    if "fa2" in which or "flashinfer" in which:
+        kcat = torch.cat([K[:kv_len[0]], K[:kv_len[1]]]).view(-1, H, hd)
+        vcat = torch.cat([V[:kv_len[0]], V[:kv_len[1]]]).view(-1, H, hd)
+    if "fa2" in which:
+        try:
+            from flash_attn import flash_attn_varlen_func
+            cu_q = torch.tensor([0, c, 2 * c], dtype=torch.int32, device="cuda")
+            cu_k = torch.tensor([0, kv_len[0], kv_len[0] + kv_len[1]], dtype=torch.int32, device="cuda")
+
+            def fa(qq, kk, vv):
+                return flash_attn_varlen_func(qq, kk, vv, cu_q, cu_k, c, kv_len[1], softmax_scale=scale, causal=True)
+            qg, kg, vg = (x.detach().clone().requires_grad_() for x in (q.view(L, H, hd), kcat, vcat))
+            o_g = fa(qg, kg, vg)
+
+            def fb():
+                qg.grad = kg.grad = vg.grad = None
+                o_g.backward(d_o.view(L, H, hd), retain_graph=True)
+            out["fa2"] = (lambda: fa(q.view(L, H, hd), kcat, vcat), fb,
+                          {"o": lambda: fa(q.view(L, H, hd), kcat, vcat).reshape(L, h)})
+        except Exception as ex:  # noqa: BLE001
+            out["fa2"] = (None, None, {"error": repr(ex)[:300]})
+    if "flashinfer" in which:
+        try:
+            import flashinfer
+            qo = torch.tensor([0, c, 2 * c], dtype=torch.int32, device="cuda")
+            kvp = torch.tensor([0, kv_len[0], kv_len[0] + kv_len[1]], dtype=torch.int32, device="cuda")
+            wsb = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+            wr = flashinfer.BatchPrefillWithRaggedKVCacheWrapper(wsb, kv_layout="NHD", backend="cute-dsl")
+            wr.plan(qo, kvp, H, H, hd, causal=True, sm_scale=scale, q_data_type=torch.float16)
+            o_f = wr.run(q.view(L, H, hd), kcat, vcat)
+            out["flashinfer_cute_dsl"] = (lambda: wr.run(q.view(L, H, hd), kcat, vcat, out=o_f), None,
+                                          {"o": lambda: o_f.view(L, h)})
+        except Exception as ex:  # noqa: BLE001
+            out["flashinfer_cute_dsl"] = (None, None, {"error": repr(ex)[:300]})
+    return out
+
+
+def run_sweep_attn_lib(args):
+    """Context, not part of the product: rank 0's causal attention (forward
+    and backward) in this library beside the attention kernels of cuDNN
+    (Blackwell SDPA, forward and backward), flash-attn 2 (mma.sync, forward
+    and backward) and flashinfer (CuTe DSL Blackwell prefill, forward only),
+    all fed the same Q, K, V, dO (Q, O from this library's forward).  The
+    rank's work is two requests with bottom-right causal masks: chunk r
+    against keys [0, (r+1) c) and chunk 2D-1-r against keys [0, (2D-r) c).
+    Every round runs each implementation once, in rotating order, so drift of
+    the power-capped clock hits all alike; medians over the rounds."""
+    import torch
+    from folded_tensor_sequence_rank_b200 import tsp
+    wl = WORKLOADS[args.workload]
+    T, h, H, F, D, r = wl["T"], wl["h"], wl["H"], wl["F"], wl["D"], 0
+    L, hd = T // D, wl["h"] // wl["H"]
+    c = L // 2
+    torch.cuda.set_device(0)
+    dims = tsp.make_dims(T, h, H, F)
+    rnd, w_full = _synthetic(T, h, F, wl["seed"])
+    sw = tsp.pack_shards(dims, D, w_full)
+    del w_full
+    kv_std = 0.02 * math.sqrt(h)
+    K = rnd(T, h, std=kv_std, dtype=torch.float16)
+    V = rnd(T, h, std=kv_std, dtype=torch.float16)
+    x = rnd(L, h)
+    y = torch.empty(L, h, dtype=torch.float32, device="cuda")
+    ws = tsp.alloc_workspace(dims, D)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(8)]
+    tsp.layer_forward(dims, sw, r, x, K, V, y, ws)
+    torch.cuda.synchronize()
+    q = tsp.workspace_view(ws, dims, D, "q").clone()
+    a = tsp.workspace_view(ws, dims, D, "a").clone()
+    lse = tsp.workspace_view(ws, dims, D, "lse").clone()
+    d_o = rnd(L, h, std=kv_std, dtype=torch.float16)
+    aws = tsp.alloc_attn_backward_workspace(dims, D)
+    dq = torch.empty(L, h, dtype=torch.float32, device="cuda")
+    dK = torch.zeros(T, h, dtype=torch.float32, device="cuda")
+    dV = torch.zeros_like(dK)
+    kv_len = [(r + 1) * c, (2 * D - r) * c]
+    pairs = sum(float(sum(range(lo + 1, lo + c + 1))) for lo in (r * c, (2 * D - 1 - r) * c))
+    fl_f, fl_b = 4.0 * h * pairs, 10.0 * h * pairs
+
+    def ours_fwd():
+        tsp.layer_forward(dims, sw, r, x, K, V, y, ws, events=evs)
+    impls = {"tsp": (ours_fwd, lambda: tsp.attn_backward(dims, D, r, q, K, V, a, lse, d_o, dq, dK, dV, aws), {})}
+    impls.update(_attn_lib_impls(q, a, d_o, K, V, c, kv_len, H, hd, dims.softmax_scale,
+                                 ("cudnn", "fa2", "flashinfer")))
+
+    def timed(name, fn):
+        if name == "tsp" and fn is ours_fwd:
+            fn()
+            torch.cuda.synchronize()
+            return evs[2].elapsed_time(evs[3])  # the attention launch inside the layer forward
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+    live = [n for n, (f, _, _) in impls.items() if f is not None]
+    for n in live:
+        for _ in range(args.warmup):
+            impls[n][0]()
+            if impls[n][1] is not None:
+                impls[n][1]()
+    torch.cuda.synchronize()
+    rounds = max(3, min(args.steps, 8))
+    rec = {n: {"fwd": [], "bwd": []} for n in live}
+    clocks = ClockSampler(0)
+    time.sleep(0.3)
+    for i in range(rounds):
+        order = live[i % len(live):] + live[:i % len(live)]
+        for n in order:
+            rec[n]["fwd"].append(timed(n, impls[n][0]))
+        for n in order:
+            if impls[n][1] is not None:
+                rec[n]["bwd"].append(timed(n, impls[n][1]))
+    clk = clocks.stop()
+    assert tsp.get_device_status(ws) == tsp.TSP_OK and tsp.get_device_status(aws) == tsp.TSP_OK
+    res = {}
+    for n, (f, b, info) in impls.items():
+        if f is None:
+            res[n] = {"error": info.get("error")}
+            continue
+        d = {"fwd_ms": round(statistics.median(rec[n]["fwd"]), 3)}
+        d["fwd_tflops"] = round(fl_f / d["fwd_ms"] / 1e9, 1)
+        if rec[n]["bwd"]:
+            d["bwd_ms"] = round(statistics.median(rec[n]["bwd"]), 3)
+            d["bwd_tflops"] = round(fl_b / d["bwd_ms"] / 1e9, 1)
+        if "o" in info:
+            d["o_maxabs_vs_tsp"] = float((info["o"]().float() - a.float()).abs().max())
+        if "version" in info:
+            d["version"] = info["version"]
+        res[n] = d
+    line = {"metric": "causal attention of one TSP rank beside library kernels on the same work (context)",
+            "value": res["tsp"]["fwd_tflops"], "unit": "TFLOP/s (forward, this library)", "n_gpus": 1,
+            "steps": rounds, "warmup": args.warmup, "higher_is_better": True, "dtype": "fp16", "data": "synthetic",
+            "config": {"workload": f"rank 0 of T={T}, D={D}, {H} heads x {hd}: chunks 0 and {2 * D - 1} "
+                                   f"({c} rows each) against keys [0, {kv_len[0]}) and [0, {kv_len[1]})",
+                       "flops_fwd": fl_f, "flops_bwd": fl_b},
+            "impls": res, "clocks": clk}
+    return line
+
+
 def run_sweep_stack(args):
     """A 32-layer stack of the 7B layer at T = 131072 on one GPU, all D = 8
     ranks in turn per layer (K/V projections, then layer forwards), random
@@ -878,18 +1084,22 @@ def main():
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the other configurations (all 8 ranks, the shard sweep, the backward, the stack) "
                          "that a default 1-GPU run measures after its main line")
-    ap.add_argument("--sweep", choices=["ranks", "shards", "stack", "mlp_bwd", "layer_bwd", "tp"], default=None,
+    ap.add_argument("--sweep", choices=["ranks", "shards", "stack", "mlp_bwd", "layer_bwd", "tp", "attn_lib"],
+                    default=None,
                     help="ranks: all 8 ranks of the 128K layer in turn (per-rank spread, whole-layer tokens/s); "
                          "shards: rank 0 at T=32768 for D=1..16; stack: a 32-layer forward at 128K; "
                          "mlp_bwd: the MLP-half backward of rank 0 at 128K; "
                          "layer_bwd: the whole layer's backward of rank 0 at 128K; "
-                         "tp: the tensor-parallel baseline layer beside a TSP rank step at 128K")
+                         "tp: the tensor-parallel baseline layer beside a TSP rank step at 128K; "
+                         "attn_lib: the rank's attention beside cuDNN, flash-attn 2 and flashinfer kernels "
+                         "on the same work (--workload picks T)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     wl = WORKLOADS[args.workload]
     sweeps = {"ranks": run_sweep_ranks, "shards": run_sweep_shards, "mlp_bwd": run_sweep_mlp_bwd,
-              "layer_bwd": run_sweep_layer_bwd, "tp": run_sweep_tp, "stack": run_sweep_stack}
+              "layer_bwd": run_sweep_layer_bwd, "tp": run_sweep_tp, "stack": run_sweep_stack,
+              "attn_lib": run_sweep_attn_lib}
     if args.sweep is not None:
         print(json.dumps(sweeps[args.sweep](args)), flush=True)
     elif args.impl == "reference":
