@@ -391,7 +391,9 @@ def measure_tsp(args, wl):
     # Consecutive steps alternate between two streams ("lanes"), each with its
     # own staging buffers, workspace and K/V, so the copy engines move one
     # step's tokens while the SMs compute the other's; every step still does
-    # its own host->device and device->host copy.
+    # its own host->device and device->host copy.  Each step's kernels wait for
+    # the previous step's (the call's compute_after / compute_done events), so
+    # the two lanes' kernels never share the SMs.
     lanes = []
     for li in range(2):
         lanes.append(dict(stream=torch.cuda.Stream(), hx=x_local.cpu().pin_memory(),
@@ -401,10 +403,16 @@ def measure_tsp(args, wl):
                           K=K if li == 0 else K.clone(), V=V if li == 0 else V.clone()))
     torch.cuda.synchronize()
 
+    done = [torch.cuda.Event(), torch.cuda.Event()]
+    n_host = [0]
+
     def host_step(ln):
+        i = n_host[0]
+        n_host[0] += 1
         with torch.cuda.stream(ln["stream"]):
             tsp.rank_step_host(dims, sw, trank, ln["hx"], ln["xs"], ln["K"], ln["V"], ln["ys"], ln["hy"], ln["ws"],
-                               stream=ln["stream"])
+                               stream=ln["stream"], compute_after=done[(i - 1) % 2] if i > 0 else None,
+                               compute_done=done[i % 2])
     for i in range(4):
         host_step(lanes[i % 2])
     barrier()

@@ -1264,7 +1264,8 @@ int tsp_rank_step(const tsp_dims* dims, const tsp_weights* w, int rank, const vo
 
 int tsp_rank_step_host(const tsp_dims* dims, const tsp_weights* w, int rank, const void* h_x_local,
                        void* d_x_staging, void* k_full, void* v_full, void* d_y_staging, void* h_y_local, int y_dtype,
-                       void* ws, size_t ws_bytes, cudaStream_t stream) {
+                       void* ws, size_t ws_bytes, cudaStream_t stream, cudaEvent_t compute_after,
+                       cudaEvent_t compute_done) {
   TSP_RANGE("tsp_rank_step_host");
   Ctx c;
   int rc = make_ctx(c, dims, w, rank, ws, ws_bytes);
@@ -1278,8 +1279,10 @@ int tsp_rank_step_host(const tsp_dims* dims, const tsp_weights* w, int rank, con
   const size_t xb = static_cast<size_t>(c.s.L) * c.s.h * 2;
   const size_t yb = static_cast<size_t>(c.s.L) * c.s.h * (y_dtype == TSP_OUT_F32 ? 4 : 2);
   TSP_CUDA(cudaMemcpyAsync(d_x_staging, h_x_local, xb, cudaMemcpyHostToDevice, stream));
+  if (compute_after) TSP_CUDA(cudaStreamWaitEvent(stream, compute_after, 0));
   rc = tsp_rank_step(dims, w, rank, d_x_staging, k_full, v_full, d_y_staging, y_dtype, ws, ws_bytes, stream, nullptr);
   if (rc) return rc;
+  if (compute_done) TSP_CUDA(cudaEventRecord(compute_done, stream));
   TSP_CUDA(cudaMemcpyAsync(h_y_local, d_y_staging, yb, cudaMemcpyDeviceToHost, stream));
   return TSP_OK;
 }

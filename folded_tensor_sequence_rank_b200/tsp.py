@@ -79,7 +79,7 @@ def lib() -> ctypes.CDLL:
         "tsp_kv_project_noalloc_status": (i32, [vp]),
         "tsp_layer_forward": (i32, [pd, pw, i32, vp, vp, vp, vp, i32, vp, sz, vp, ctypes.POINTER(vp)]),
         "tsp_rank_step": (i32, [pd, pw, i32, vp, vp, vp, vp, i32, vp, sz, vp, ctypes.POINTER(vp)]),
-        "tsp_rank_step_host": (i32, [pd, pw, i32, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]),
+        "tsp_rank_step_host": (i32, [pd, pw, i32, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp, vp, vp]),
         "tsp_selftest_wait_timeout": (i32, [vp, ctypes.c_uint64, vp]),
         "tsp_attn_backward_workspace_bytes": (sz, [pd, i32]),
         "tsp_attn_backward": (i32, [pd, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
@@ -447,9 +447,21 @@ def mlp_backward(dims: Dims, w: ShardedWeights, w1_full, w2_full, y1, dy, dy1, d
                                   bws.numel(), _stream(stream), _events(events)), "tsp_mlp_backward")
 
 
+def _event(e):
+    """A torch.cuda.Event as a CUDA event handle (created on first use), or None."""
+    if e is None:
+        return None
+    if not e.cuda_event:
+        e.record()  # torch creates the CUDA event on its first record
+    return e.cuda_event
+
+
 def rank_step_host(dims: Dims, w: ShardedWeights, rank: int, h_x_local, x_staging, k_full, v_full,
-                   y_staging, h_y_local, ws, stream=None):
-    """rank_step with host (ideally pinned) token buffers; copies run on the stream."""
+                   y_staging, h_y_local, ws, stream=None, compute_after=None, compute_done=None):
+    """rank_step with host (ideally pinned) token buffers; copies run on the stream.
+    compute_after / compute_done: optional torch.cuda.Event objects that order
+    this step's kernels after another step's and mark their end (see the C
+    header)."""
     L, h = dims.T // w.D, dims.h
     if h_x_local.is_cuda or h_y_local.is_cuda:
         raise ValueError("h_x_local and h_y_local must be host tensors")
@@ -461,7 +473,8 @@ def rank_step_host(dims: Dims, w: ShardedWeights, rank: int, h_x_local, x_stagin
     pv = _ptr(v_full, "v_full", torch.float16, (dims.T, h))
     yd = OUT_F32 if y_staging.dtype == torch.float32 else OUT_BF16
     _check(lib().tsp_rank_step_host(ctypes.byref(dims), ctypes.byref(w.struct), rank, phx, pxs, pk, pv, pys, phy,
-                                    yd, _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream)),
+                                    yd, _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream),
+                                    _event(compute_after), _event(compute_done)),
            "tsp_rank_step_host")
 
 

@@ -263,12 +263,19 @@ int tsp_rank_step(const tsp_dims* dims, const tsp_weights* w, int rank,
 /* tsp_rank_step with the token buffers in HOST memory: copies h_x_local
  * ([T/D, h] bf16) to `d_x_staging` (device, T/D*h*2 bytes, caller-owned),
  * runs the step, copies the result back to h_y_local, all enqueued on
- * `stream`.  Pinned host memory makes the copies asynchronous. */
+ * `stream`.  Pinned host memory makes the copies asynchronous.
+ * compute_after (may be null): the step's kernels wait for this event, after
+ * the host-to-device copy has been enqueued; compute_done (may be null) is
+ * recorded when they end, before the device-to-host copy.  A caller that
+ * alternates steps between two streams chains each step's compute_after to
+ * the previous step's compute_done: the copies of one step then overlap the
+ * kernels of the other while the kernels of consecutive steps never share
+ * the GPU.  Both events are the caller's; neither is waited on by the host. */
 int tsp_rank_step_host(const tsp_dims* dims, const tsp_weights* w, int rank,
                        const void* h_x_local, void* d_x_staging,
                        void* k_full, void* v_full, void* d_y_staging,
                        void* h_y_local, int y_dtype, void* ws, size_t ws_bytes,
-                       cudaStream_t stream);
+                       cudaStream_t stream, cudaEvent_t compute_after, cudaEvent_t compute_done);
 
 /* Workspace bytes of tsp_attn_backward at this D (status section, work
  * queue counter, Delta); 0 on a bad argument. */

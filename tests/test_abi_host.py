@@ -137,7 +137,7 @@ def test_rank_step_host_checks_everything_before_its_first_copy(L):
     def call(y_dtype=0, **kw):
         a = dict(ok, **kw)
         return L.tsp_rank_step_host(ctypes.byref(d), ctypes.byref(w), 0, a["hx"], a["xs"], a["k"], a["v"], a["ys"],
-                                    a["hy"], y_dtype, ws, nws, None)
+                                    a["hy"], y_dtype, ws, nws, None, None, None)
     assert call(y_dtype=7) == tsp.TSP_ERR_INVALID_ARG      # output dtype
     assert call(k=None) == tsp.TSP_ERR_INVALID_ARG         # K
     assert call(v=0x4008) == tsp.TSP_ERR_INVALID_ARG       # V misaligned

@@ -244,6 +244,47 @@ def test_rank_step_host_buffers():
     assert torch.equal(hy, yd.cpu())
 
 
+def test_rank_step_host_two_lanes_chained():
+    """Steps alternating between two streams, each step's kernels ordered
+    after the previous step's by the call's events (as the end-to-end bench
+    runs them): every rank's host result equals its device rank step."""
+    T, h, H, F, D = 2048, 512, 4, 2048, 4
+    raw = to_cuda(inputs.layer_inputs(T, h, F, 17))
+    dims = tsp.make_dims(T, h, H, F)
+    sw = tsp.pack_shards(dims, D, raw)
+    L = T // D
+    K = torch.zeros(T, h, dtype=torch.float16, device="cuda")
+    V = torch.zeros_like(K)
+    ws0 = tsp.alloc_workspace(dims, D)
+    xs = [raw["x"].index_select(0, tsp.zigzag_index(T, D, r).long()).contiguous() for r in range(D)]
+    for r in range(D):
+        tsp.kv_project(dims, sw, r, xs[r], K, V, ws0)
+    want = []
+    for r in range(D):
+        y = torch.empty(L, h, dtype=torch.bfloat16, device="cuda")
+        tsp.rank_step(dims, sw, r, xs[r], K, V, y, ws0)
+        want.append(y.cpu())
+    torch.cuda.synchronize()
+    lanes = [dict(stream=torch.cuda.Stream(), ws=tsp.alloc_workspace(dims, D), K=K.clone(), V=V.clone(),
+                  xs=torch.empty(L, h, dtype=torch.bfloat16, device="cuda"),
+                  ys=torch.empty(L, h, dtype=torch.bfloat16, device="cuda")) for _ in range(2)]
+    done = [torch.cuda.Event(), torch.cuda.Event()]
+    hx = [xs[r].cpu().pin_memory() for r in range(D)]
+    hy = [torch.empty(L, h, dtype=torch.bfloat16).pin_memory() for _ in range(2 * D)]
+    torch.cuda.synchronize()
+    for i in range(2 * D):  # every rank twice
+        ln, r = lanes[i % 2], i % D
+        with torch.cuda.stream(ln["stream"]):
+            tsp.rank_step_host(dims, sw, r, hx[r], ln["xs"], ln["K"], ln["V"], ln["ys"], hy[i], ln["ws"],
+                               stream=ln["stream"], compute_after=done[(i - 1) % 2] if i > 0 else None,
+                               compute_done=done[i % 2])
+    torch.cuda.synchronize()
+    for ln in lanes:
+        assert tsp.get_device_status(ln["ws"]) == tsp.TSP_OK
+    for i in range(2 * D):
+        assert torch.equal(hy[i], want[i % D]), i
+
+
 # --------------------------------------------------------------------------
 # the 7B layer
 # --------------------------------------------------------------------------
