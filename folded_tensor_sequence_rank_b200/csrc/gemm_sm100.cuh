@@ -100,12 +100,16 @@ __device__ __forceinline__ void gemm_tile_coords(int tile, int num_m, int num_n,
 
 // GELU, tanh form, through the identity 0.5 (1 + tanh(u)) = 1 / (1 + e^(-2u)):
 //   GELU(x) = x / (1 + 2^(-2 u log2(e))),  u = sqrt(2/pi) (x + 0.044715 x^3).
-// ex2.approx has ~2^-22 relative error and the division is IEEE-rounded, so
-// the result is accurate to a few fp32 ulps before its bf16 rounding.
+// ex2.approx has ~2^-22 relative error and the fast division (__fdividef) at
+// most 2 ulps, so the result is accurate to a few fp32 ulps before its 16-bit
+// rounding.  An IEEE-rounded division cost the W1 GEMM 8% of its time.  The
+// fast division's limits are harmless here: a denominator beyond 2^126 (x <
+// about -44) gives 0, GELU's limit; an infinite x, for which it would give
+// NaN, cannot come out of a GEMM of finite fp16 operands.
 __device__ __forceinline__ float gelu_tanh_f(float x) {
   const float k = -2.0f * 0.7978845608028654f * 1.4426950408889634f;  // -2 sqrt(2/pi) log2(e)
   const float u = fmaf(0.044715f * x, x * x, x);
-  return x / (1.0f + ex2_approx(k * u));
+  return __fdividef(x, 1.0f + ex2_approx(k * u));
 }
 
 // d/dx GELU (tanh form).  With p = 1 / (1 + e^(-2u)) = 0.5 (1 + tanh(u)),
@@ -116,7 +120,7 @@ __device__ __forceinline__ float gelu_tanh_grad_f(float x) {
   const float k = -2.0f * 0.7978845608028654f * 1.4426950408889634f;  // -2 sqrt(2/pi) log2(e)
   const float x2 = x * x;
   const float u = fmaf(0.044715f * x, x2, x);
-  const float pr = __frcp_rn(1.0f + ex2_approx(k * u));
+  const float pr = __fdividef(1.0f, 1.0f + ex2_approx(k * u));  // as in gelu_tanh_f
   return fmaf(2.0f * x * pr * (1.0f - pr) * s, fmaf(3.0f * 0.044715f, x2, 1.0f), pr);
 }
 
