@@ -21,12 +21,18 @@
 // order makes the ~148 concurrent items stream the same head's K/V, so each
 // K/V tile is read from HBM about once and then served from L2.
 //
-// Roles (320 threads, one CTA per SM, persistent):
-//   warp 0     work queue + TMA producer (Q_A, Q_B, K ring, V ring)
-//   warp 1     TMEM allocator + single-thread tcgen05.mma issuer
-//   warps 2-5  softmax, correction and epilogue of query tile A (thread = row)
-//   warps 6-9  the same for query tile B
-// Each SM sub-partition runs one warp of each tile.
+// Roles (384 threads = three warpgroups, one CTA per SM, persistent):
+//   warp 0      work queue + TMA producer (Q_A, Q_B, K ring, V ring)
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
+//   warps 2-3   idle (they complete the first warpgroup)
+//   warps 4-7   softmax, correction and epilogue of query tile A (thread = row)
+//   warps 8-11  the same for query tile B
+// Each SM sub-partition runs one warp of each warpgroup.  The registers are
+// re-split at the start (setmaxnreg): the first warpgroup drops to
+// kAttnLowRegs per thread and the two softmax warpgroups rise to
+// kAttnHighRegs (128 x 56 + 256 x 224 = 384 x 168, the launch allocation,
+// which the launcher checks).  At the 168 of a uniform split the softmax
+// spilled, and reloading the spills cost 6% of the kernel's time.
 // Tensor memory (512 columns): [S | P_A | P_B | O_A | O_B] = 128 + 64 + 64 +
 // 128 + 128.  The score buffer S is shared by the two query tiles and used in
 // turn: S_A(j), S_B(j), S_A(j+1), ...  A softmax warp reads its whole score
@@ -49,7 +55,11 @@
 
 namespace tsp {
 
-constexpr int kAttnThreads = 320;
+constexpr int kAttnThreads = 384;
+constexpr int kAttnLaunchRegs = 168;  // per thread at launch: 65536 / 384, rounded down to 8
+constexpr int kAttnLowRegs = 56;      // warps 0-3 after the re-split
+constexpr int kAttnHighRegs = 224;    // the softmax warpgroups after the re-split
+static_assert(128 * kAttnLowRegs + 256 * kAttnHighRegs <= kAttnThreads * kAttnLaunchRegs, "register split");
 constexpr int kAttnBM = 128;
 constexpr int kAttnBN = 128;
 
@@ -122,7 +132,7 @@ __device__ __forceinline__ AttnItem attn_decode(const AttnParams& p, int it) {
 // (abort or timeout) the whole warp leaves together, so the .sync.aligned
 // tensor-memory instructions that follow are never reached by half a warp.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& ctl) {
-  const bool ok = mbar_wait(bar, parity, ctl);
+  const bool ok = mbar_wait_inl(bar, parity, ctl);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -192,6 +202,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
   const uint32_t tmem = *tmem_slot;
   const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
 
+  if (warp < 4) {
+    __syncwarp();
+    regs_dec<kAttnLowRegs>();
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
     if (elect_one()) {
@@ -204,7 +217,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
       bool ok = true;
       for (int n = 0; ok; ++n) {
         const int slot = n & 1;
-        if (!mbar_wait(&it_empty[slot], ((n >> 1) & 1) ^ 1, ctl)) break;
+        if (!mbar_wait_inl(&it_empty[slot], ((n >> 1) & 1) ^ 1, ctl)) break;
         int it = atomicAdd(p.counter, 1);
         if (it >= p.n_items) it = -1;
         it_slot[slot] = it;
@@ -214,7 +227,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
         const int col0 = w.head * HD;
         for (int x = 0; ok && x < 2; ++x) {
           if (w.t[x].nkv == 0) continue;
-          if (!mbar_wait(&q_empty[x], qph[x] ^ 1, ctl)) { ok = false; break; }
+          if (!mbar_wait_inl(&q_empty[x], qph[x] ^ 1, ctl)) { ok = false; break; }
           mbar_arrive_expect_tx(&q_full[x], S::kQBytes);
 #pragma unroll
           for (int b = 0; b < NB; ++b)
@@ -225,7 +238,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
         }
         const int nkv = max(w.t[0].nkv, w.t[1].nkv);
         for (int kt = 0; ok && kt < nkv; ++kt) {
-          if (!mbar_wait(&k_empty[ks], kph ^ 1, ctl)) { ok = false; break; }
+          if (!mbar_wait_inl(&k_empty[ks], kph ^ 1, ctl)) { ok = false; break; }
           mbar_arrive_expect_tx(&k_full[ks], S::kKVBytes);
 #pragma unroll
           for (int b = 0; b < NB; ++b)
@@ -233,7 +246,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
           kused |= 1u << ks;
           kpar = (kpar & ~(1u << ks)) | (kph << ks);
           if (++ks == KST) { ks = 0; kph ^= 1; }
-          if (!mbar_wait(&v_empty[vs], vph ^ 1, ctl)) { ok = false; break; }
+          if (!mbar_wait_inl(&v_empty[vs], vph ^ 1, ctl)) { ok = false; break; }
           mbar_arrive_expect_tx(&v_full[vs], S::kKVBytes);
 #pragma unroll
           for (int b = 0; b < NB; ++b)
@@ -272,7 +285,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
       // S_x = Q_x K^T for the K tile in slot ks (K = head_dim in 16-column steps:
       // +32 bytes inside a 128-byte swizzle row, +16 KiB to the next 64 columns)
       auto issue_s = [&](int x, bool last_s) -> bool {
-        if (scnt > 0 && !mbar_wait(s_free, (scnt - 1) & 1, ctl)) return false;
+        if (scnt > 0 && !mbar_wait_inl(s_free, (scnt - 1) & 1, ctl)) return false;
         ++scnt;
         tc_fence_after();
         if constexpr (HD == 128) {
@@ -291,8 +304,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
       // O_x += P_x V for the V tile in slot vs (K = 128 keys in 16-key steps:
       // P advances 8 TMEM columns, V 2 KiB = 128 units)
       auto issue_pv = [&](int x, bool first, bool last) -> bool {
-        if (first && !mbar_wait(&o_free[x], (icnt[x] & 1) ^ 1, ctl)) return false;
-        if (!mbar_wait(&p_full[x], pcnt[x] & 1, ctl)) return false;
+        if (first && !mbar_wait_inl(&o_free[x], (icnt[x] & 1) ^ 1, ctl)) return false;
+        if (!mbar_wait_inl(&p_full[x], pcnt[x] & 1, ctl)) return false;
         ++pcnt[x];
         tc_fence_after();
         mma_ts_x8<128>(tmem + 256 + x * 128, tmem + 128 + x * 64, vdesc(), idesc_o, first ? 0u : 1u);
@@ -300,7 +313,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
         return true;
       };
       auto wait_k = [&]() -> bool {
-        if (!mbar_wait(&k_full[ks], kph, ctl)) return false;
+        if (!mbar_wait_inl(&k_full[ks], kph, ctl)) return false;
         tc_fence_after();
         return true;
       };
@@ -310,7 +323,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
       };
       for (int n = 0; ok; ++n) {
         const int slot = n & 1;
-        if (!mbar_wait(&it_full[slot], (n >> 1) & 1, ctl)) break;
+        if (!mbar_wait_inl(&it_full[slot], (n >> 1) & 1, ctl)) break;
         const int it = it_slot[slot];
         mbar_arrive(&it_empty[slot]);
         if (it < 0) break;
@@ -319,7 +332,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
         const int nkv = max(na, nb);
         for (int x = 0; ok && x < 2; ++x) {
           if (w.t[x].nkv == 0) continue;
-          ok = mbar_wait(&q_full[x], qph[x], ctl);
+          ok = mbar_wait_inl(&q_full[x], qph[x], ctl);
           qph[x] ^= 1;
         }
         if (!ok) break;
@@ -331,7 +344,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
         release_k();
         // per key tile: S_A(kt+1) PV_A(kt) S_B(kt+1) PV_B(kt)
         for (int kt = 0; ok && kt < nkv; ++kt) {
-          if (!mbar_wait(&v_full[vs], vph, ctl)) { ok = false; break; }
+          if (!mbar_wait_inl(&v_full[vs], vph, ctl)) { ok = false; break; }
           bool k_waited = false;
           if (kt < na) {
             if (kt + 1 < na) {
@@ -362,9 +375,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
       mma_commit(drain);
       mbar_drain(drain, 0, p.timeout_ns);
     }
+  }
   } else {
     // ---------------------------------------------------------------- softmax
-    const int x = (warp - 2) >> 2;     // query tile of this warp group
+    __syncwarp();
+    regs_inc<kAttnHighRegs>();
+    const int x = (warp - 4) >> 2;     // query tile of this warp group
     const int quarter = warp & 3;      // TMEM lane quarter = rows 32*quarter ..
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;

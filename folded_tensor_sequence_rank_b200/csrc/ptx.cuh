@@ -187,6 +187,39 @@ __device__ __forceinline__ bool mbar_wait_cl(uint64_t* bar, uint32_t parity, con
   return mbar_wait_cl_slow(a, parity, ctl);
 }
 
+// The bounded wait with its slow path inlined, for kernels that re-split
+// registers between warpgroups (setmaxnreg): ptxas allocates each region for
+// its own register budget, and a function called from regions with different
+// budgets (mbar_wait_slow) cannot be allocated.
+__device__ __forceinline__ bool mbar_wait_inl(uint64_t* bar, uint32_t parity, const WaitCtl& ctl) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait_sleep(a, parity, 20000u)) return true;
+    if (*ctl.abort_flag) return false;
+    if (globaltimer_ns() - t0 > ctl.timeout_ns) {
+      *ctl.abort_flag = 1;
+      atomicExch(ctl.status, kStatusTimeout);
+      return false;
+    }
+  }
+}
+
+// Per-thread register budget of the executing warpgroup (setmaxnreg; each
+// of its four warps executes the same instruction, converged).  A CTA's
+// increases can only draw on registers its other warpgroups released, out of
+// what the CTA was launched with; an increase that cannot be met waits, so
+// the shares must add up to no more than the launch allocation.
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }

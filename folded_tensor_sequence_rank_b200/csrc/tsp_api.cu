@@ -467,6 +467,31 @@ int launch_ksplit(const Sizes& s, int rank, const __half* a, int Kdim, const voi
   return launch_gemm(p, bn, st);
 }
 
+template <int HD>
+cudaError_t prepare_attention() {
+  return cudaFuncSetAttribute(attn_fwd_tcgen05<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              AttnShape<HD>::kSmemBytes);
+}
+
+// The attention kernel re-splits its registers between warpgroups
+// (setmaxnreg): the split adds up only for the allocation it was built for;
+// with any other count an increase could wait forever, so refuse to launch.
+template <int HD>
+int check_attention_regs() {
+  static int regs = -1;
+  if (regs < 0) {
+    cudaFuncAttributes fa = {};
+    TSP_CUDA(cudaFuncGetAttributes(&fa, attn_fwd_tcgen05<HD>));
+    regs = fa.numRegs;
+  }
+  if (regs != kAttnLaunchRegs) {
+    std::snprintf(g_cuda_err, sizeof(g_cuda_err), "attention kernel built with %d registers per thread, not %d", regs,
+                  kAttnLaunchRegs);
+    return TSP_ERR_CUDA;
+  }
+  return TSP_OK;
+}
+
 int launch_attention(const Sizes& s, int rank, const tsp_dims* dims, const __half* q, const void* k_full,
                      const void* v_full, __half* out, float* lse, int* counter, int* status, cudaStream_t st) {
   TSP_RANGE("attention");
@@ -499,20 +524,16 @@ int launch_attention(const Sizes& s, int rank, const tsp_dims* dims, const __hal
   if (s.d == 128) {
     static std::once_flag once;
     static cudaError_t e = cudaSuccess;
-    std::call_once(once, [] {
-      e = cudaFuncSetAttribute(attn_fwd_tcgen05<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               AttnShape<128>::kSmemBytes);
-    });
+    std::call_once(once, [] { e = prepare_attention<128>(); });
     TSP_CUDA(e);
+    if ((rc = check_attention_regs<128>())) return rc;
     attn_fwd_tcgen05<128><<<grid, kAttnThreads, AttnShape<128>::kSmemBytes, st>>>(p);
   } else {
     static std::once_flag once;
     static cudaError_t e = cudaSuccess;
-    std::call_once(once, [] {
-      e = cudaFuncSetAttribute(attn_fwd_tcgen05<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               AttnShape<64>::kSmemBytes);
-    });
+    std::call_once(once, [] { e = prepare_attention<64>(); });
     TSP_CUDA(e);
+    if ((rc = check_attention_regs<64>())) return rc;
     attn_fwd_tcgen05<64><<<grid, kAttnThreads, AttnShape<64>::kSmemBytes, st>>>(p);
   }
   TSP_CUDA(cudaGetLastError());
