@@ -21,13 +21,17 @@
 // heaviest key tiles of a head first (key tile kt is reached by every query
 // tile that reaches kt + 1).
 //
-// Roles (320 threads, one CTA per SM, persistent):
-//   warp 0     work queue + TMA producer: K, V of the item; Q, lse2, Delta
-//              (2-stage ring) and dO (1 stage) of each query tile
-//   warp 1     TMEM allocator + single-thread tcgen05.mma issuer
-//   warps 2-9  elementwise softmax gradient, dQ read-out, dK/dV epilogue; a
-//              thread owns one key row (TMEM lane) and half of the columns,
-//              so two warps share each lane quarter
+// Roles (384 threads = three warpgroups, one CTA per SM, persistent):
+//   warp 0      work queue + TMA producer: K, V of the item; Q, lse2, Delta
+//               (2-stage ring) and dO (1 stage) of each query tile
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
+//   warps 2-3   idle (they complete the first warpgroup)
+//   warps 4-11  elementwise softmax gradient, dQ read-out, dK/dV epilogue; a
+//               thread owns one key row (TMEM lane) and half of the columns,
+//               so two warps share each lane quarter
+// As in the forward kernel the registers are re-split at the start
+// (setmaxnreg): kBwdLowRegs for the first warpgroup, kBwdHighRegs for the
+// two softmax warpgroups, within the 168 per thread of the launch.
 // Tensor memory (512 columns): [dK | dV | S^T | dP^T] = 128 each (dK, dV use
 // head_dim of their 128).  Per query tile:
 //   S^T = K Q^T  and  dP^T = V dO^T  (keys on the lanes; SS MMAs, K-major);
@@ -54,7 +58,11 @@
 
 namespace tsp {
 
-constexpr int kBwdThreads = 320;
+constexpr int kBwdThreads = 384;        // three warpgroups
+constexpr int kBwdLaunchRegs = 168;     // per thread at launch: 65536 / 384, rounded down to 8
+constexpr int kBwdLowRegs = 80;         // warps 0-3 after the re-split
+constexpr int kBwdHighRegs = 208;       // the softmax warpgroups after the re-split
+static_assert(128 * kBwdLowRegs + 256 * kBwdHighRegs <= kBwdThreads * kBwdLaunchRegs, "register split");
 constexpr int kBwdTile = 128;  // keys per item, queries per query tile
 
 struct __align__(64) AttnBwdParams {
@@ -209,6 +217,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
   const WaitCtl ctl{abort_flag, p.status, p.timeout_ns};
   const int nq_all = 2 * p.nqt;
 
+  if (warp < 4) {
+    __syncwarp();
+    regs_dec<kBwdLowRegs>();
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
     if (elect_one()) {
@@ -223,7 +234,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
       bool ok = true;
       for (int n = 0; ok; ++n) {
         const int slot = n & 1;
-        if (!mbar_wait(&it_empty[slot], ((n >> 1) & 1) ^ 1, ctl)) break;
+        if (!mbar_wait_inl(&it_empty[slot], ((n >> 1) & 1) ^ 1, ctl)) break;
         int it = atomicAdd(p.counter, 1);
         if (it >= p.n_items) it = -1;
         it_slot[slot] = it;
@@ -231,7 +242,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
         if (it < 0) break;
         const int head = it / p.nkt, kt = it % p.nkt;
         const int col0 = head * HD;
-        if (!mbar_wait(kv_empty, kvph ^ 1, ctl)) break;
+        if (!mbar_wait_inl(kv_empty, kvph ^ 1, ctl)) break;
         mbar_arrive_expect_tx(kv_full, 2 * S::kTileBytes);
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
@@ -244,7 +255,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
         for (int n2 = 0; ok && n2 < nq_all; ++n2) {
           const BwdQTile q = bwd_qtile(p, n2);
           if (!bwd_reaches(q, kt)) continue;
-          if (!mbar_wait(&q_empty[qs], qph[qs] ^ 1, ctl)) { ok = false; break; }
+          if (!mbar_wait_inl(&q_empty[qs], qph[qs] ^ 1, ctl)) { ok = false; break; }
           mbar_arrive_expect_tx(&q_full[qs], S::kTileBytes + 2 * S::kStatBytes);
 #pragma unroll
           for (int b = 0; b < NB; ++b)
@@ -257,7 +268,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
           q_par = (q_par & ~(1u << qs)) | (qph[qs] << qs);
           qph[qs] ^= 1;
           if (++qs == QST) qs = 0;
-          if (!mbar_wait(do_empty, doph ^ 1, ctl)) { ok = false; break; }
+          if (!mbar_wait_inl(do_empty, doph ^ 1, ctl)) { ok = false; break; }
           mbar_arrive_expect_tx(do_full, S::kTileBytes);
 #pragma unroll
           for (int b = 0; b < NB; ++b) tma_load_2d(sDO + b * 16384, &p.map_do, do_full, col0 + 64 * b, q.m0);
@@ -296,12 +307,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
       bool ok = true;
       for (int n = 0; ok; ++n) {
         const int slot = n & 1;
-        if (!mbar_wait(&it_full[slot], (n >> 1) & 1, ctl)) break;
+        if (!mbar_wait_inl(&it_full[slot], (n >> 1) & 1, ctl)) break;
         const int it = it_slot[slot];
         mbar_arrive(&it_empty[slot]);
         if (it < 0) break;
         const int kt = it % p.nkt;
-        if (!mbar_wait(kv_full, kvph, ctl)) break;
+        if (!mbar_wait_inl(kv_full, kvph, ctl)) break;
         kvph ^= 1;
         tc_fence_after();
         bool first = true;
@@ -310,7 +321,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
           if (!bwd_reaches(q, kt)) continue;
           const uint64_t dQ_k = dQ_k0 + static_cast<uint64_t>(qs * (S::kTileBytes >> 4));
           const uint64_t dQ_mn = dQ_mn0 + static_cast<uint64_t>(qs * (S::kTileBytes >> 4));
-          if (!mbar_wait(&q_full[qs], qph[qs], ctl)) { ok = false; break; }
+          if (!mbar_wait_inl(&q_full[qs], qph[qs], ctl)) { ok = false; break; }
           tc_fence_after();
           // S^T = K Q^T (K = head_dim); the softmax warps read the previous
           // tile's S^T before they signalled p_full
@@ -320,10 +331,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
 #pragma unroll
             for (int kk = 0; kk < HD / 16; ++kk) mma_ss(t_s, dK_k + 2 * kk, dQ_k + 2 * kk, idesc_s, kk != 0);
           }
-          if (!mbar_wait(do_full, doph, ctl)) { ok = false; break; }
+          if (!mbar_wait_inl(do_full, doph, ctl)) { ok = false; break; }
           // dP^T = V dO^T: the dP^T columns hold the previous tile's dQ until
           // it is read out
-          if (tiles > 0 && !mbar_wait(dq_free, (tiles - 1) & 1, ctl)) { ok = false; break; }
+          if (tiles > 0 && !mbar_wait_inl(dq_free, (tiles - 1) & 1, ctl)) { ok = false; break; }
           tc_fence_after();
           if constexpr (HD == 128) {
             mma_ss_x8<0, 2, 4, 6, 1024, 1026, 1028, 1030>(t_dp, dV_k, dDO_k, idesc_s, 0);
@@ -332,10 +343,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
             for (int kk = 0; kk < HD / 16; ++kk) mma_ss(t_dp, dV_k + 2 * kk, dDO_k + 2 * kk, idesc_s, kk != 0);
           }
           mma_commit(s_full);
-          if (!mbar_wait(p_full, tiles & 1, ctl)) { ok = false; break; }
+          if (!mbar_wait_inl(p_full, tiles & 1, ctl)) { ok = false; break; }
           // the first tile of an item overwrites dK, dV: the previous item's
           // epilogue must have read them
-          if (first && items > 0 && !mbar_wait(dkv_free, (items - 1) & 1, ctl)) { ok = false; break; }
+          if (first && items > 0 && !mbar_wait_inl(dkv_free, (items - 1) & 1, ctl)) { ok = false; break; }
           tc_fence_after();
           // dV += P^T dO: A = P^T from the dP^T columns (fp16 pairs; queries
           // 0-63 in columns 0-31, queries 64-127 in columns 64-95), B = dO
@@ -353,7 +364,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
             mma_ss(t_dk, dDS_k + ((kk >> 2) * 1024 + (kk & 3) * 2), dQ_mn + 128 * kk, idesc_kv,
                    (!first || kk != 0) ? 1u : 0u);
           // dQ = dS K into the dP^T columns, once the dV MMA has read P^T
-          if (!mbar_wait(dv_done, tiles & 1, ctl)) { ok = false; break; }
+          if (!mbar_wait_inl(dv_done, tiles & 1, ctl)) { ok = false; break; }
           tc_fence_after();
           mma_ss_x8<0, 128, 256, 384, 512, 640, 768, 896>(t_dp, dDS_mn, dK_mn, idesc_q, 0);
           mma_commit(dq_full);
@@ -372,10 +383,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
       mma_commit(drain);
       mbar_drain(drain, 0, p.timeout_ns);
     }
+  }
   } else {
     // ---------------------------------------------------------------- softmax gradient
+    __syncwarp();
+    regs_inc<kBwdHighRegs>();
     const int quarter = warp & 3;       // TMEM lane quarter: key rows 32*quarter ..
-    const int half = (warp - 2) >> 2;   // query columns 64*half .. 64*half+63
+    const int half = (warp - 4) >> 2;   // query columns 64*half .. 64*half+63
     const int kr = quarter * 32 + lane; // key row of this thread
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const float sl2 = p.scale_log2;
@@ -491,7 +505,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
             // the next tile's dS^T stores.
 #pragma unroll
             for (int j = 0; j < HD / 64; ++j) {
-              uint8_t* stg = j == 0 ? sDS + (warp - 2) * 4096 : sStage2 + (warp - 2) * 4096;
+              uint8_t* stg = j == 0 ? sDS + (warp - 4) * 4096 : sStage2 + (warp - 4) * 4096;
 #pragma unroll
               for (int c = 0; c < 8; ++c)
                 *reinterpret_cast<uint4*>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
@@ -502,7 +516,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
             if (lane == 0 && dbg_ok(q.m0 + quarter * 32 + 32 <= 2 * p.c && (head + 1) * HD <= p.ld, p.status)) {
 #pragma unroll
               for (int j = 0; j < HD / 64; ++j)
-                tma_reduce_add_2d(&p.map_dq, j == 0 ? sDS + (warp - 2) * 4096 : sStage2 + (warp - 2) * 4096,
+                tma_reduce_add_2d(&p.map_dq, j == 0 ? sDS + (warp - 4) * 4096 : sStage2 + (warp - 4) * 4096,
                                   head * HD + half * (HD / 2) + 32 * j, q.m0 + quarter * 32);
               bulk_commit_group();
             }
@@ -563,7 +577,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_tcgen05(const __grid_
   }
 
   // the CTA outlives the reads of its last bulk reductions
-  if (warp >= 2 && lane == 0) bulk_wait_group_read0();
+  if (warp >= 4 && lane == 0) bulk_wait_group_read0();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

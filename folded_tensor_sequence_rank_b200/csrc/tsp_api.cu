@@ -476,20 +476,24 @@ cudaError_t prepare_attention() {
 // The attention kernel re-splits its registers between warpgroups
 // (setmaxnreg): the split adds up only for the allocation it was built for;
 // with any other count an increase could wait forever, so refuse to launch.
-template <int HD>
-int check_attention_regs() {
-  static int regs = -1;
-  if (regs < 0) {
+template <typename Kernel>
+int check_launch_regs(Kernel kernel, int want, int& cached) {
+  if (cached < 0) {
     cudaFuncAttributes fa = {};
-    TSP_CUDA(cudaFuncGetAttributes(&fa, attn_fwd_tcgen05<HD>));
-    regs = fa.numRegs;
+    TSP_CUDA(cudaFuncGetAttributes(&fa, kernel));
+    cached = fa.numRegs;
   }
-  if (regs != kAttnLaunchRegs) {
-    std::snprintf(g_cuda_err, sizeof(g_cuda_err), "attention kernel built with %d registers per thread, not %d", regs,
-                  kAttnLaunchRegs);
+  if (cached != want) {
+    std::snprintf(g_cuda_err, sizeof(g_cuda_err), "kernel built with %d registers per thread, not %d", cached, want);
     return TSP_ERR_CUDA;
   }
   return TSP_OK;
+}
+
+template <int HD>
+int check_attention_regs() {
+  static int regs = -1;
+  return check_launch_regs(attn_fwd_tcgen05<HD>, kAttnLaunchRegs, regs);
 }
 
 int launch_attention(const Sizes& s, int rank, const tsp_dims* dims, const __half* q, const void* k_full,
@@ -613,6 +617,10 @@ int launch_attn_bwd_hd(AttnBwdParams& p, cudaStream_t st) {
     e = cudaFuncSetAttribute(attn_bwd_tcgen05<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes);
   });
   TSP_CUDA(e);
+  // the kernel re-splits its registers (setmaxnreg) for this launch allocation
+  static int regs = -1;
+  const int rc = check_launch_regs(attn_bwd_tcgen05<HD>, kBwdLaunchRegs, regs);
+  if (rc) return rc;
   const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
   attn_bwd_tcgen05<HD><<<grid, kBwdThreads, S::kSmemBytes, st>>>(p);
   TSP_CUDA(cudaGetLastError());
