@@ -43,10 +43,16 @@
 // never wait for its PV, and a softmax warp never waits for the tensor core
 // except for its next score tile.  P_x is rewritten only after the PV that
 // read it has finished (one commit per PV).
-// Online softmax in base 2 with a lazily updated row maximum: the tile's
-// maximum is found first; the running output is rescaled only when the
-// maximum grows by more than 2^8, which is exact (the final division by the
-// row sum cancels the common factor).
+// Online softmax in base 2 with a lazily moved offset: a row subtracts the
+// maximum of its first key tile from every later score, with no maximum pass
+// over the later tiles.  Any common offset is exact (the final division by
+// the row sum cancels it); the offset only has to keep every probability
+// inside fp16's range.  A tile's fp32 row sum bounds its largest probability,
+// and the largest input of the exp2 polynomial is tracked (the polynomial
+// holds below 2^126): a sum above 2^15 or a larger input sends that row's
+// tile down a rare path, which recomputes the row's 128 scores from Q and K
+// in global memory on the CUDA cores, moves the offset to their maximum,
+// redoes the probabilities and rescales O before the next PV.
 // Q, K, V, P and the output are fp16; scores, softmax statistics and O are
 // fp32.
 #pragma once
@@ -85,6 +91,11 @@ struct __align__(64) AttnParams {
   // multiple of 128, so every 128-row tile of a chunk starts 512-byte aligned).
   float* lse;
   int c_pad;
+  // Q and K again as plain row-major arrays (row stride ldqk elements), read
+  // only on the rare path that recomputes a score row on the CUDA cores.
+  const __half* q;
+  const __half* k;
+  int64_t ldqk;
 };
 
 template <int HD>
@@ -126,6 +137,73 @@ __device__ __forceinline__ AttnItem attn_decode(const AttnParams& p, int it) {
     }
   }
   return w;
+}
+
+// Maximum of a 128-entry row (three-input maxima in four chains).
+__device__ __forceinline__ float attn_row_max(const float* sv) {
+  float m4[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) m4[k] = fmaxf(sv[k], sv[k + 4]);
+#pragma unroll
+  for (int i = 8; i < 128; i += 8)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) m4[k] = fmax3(m4[k], sv[i + k], sv[i + k + 4]);
+  return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+}
+
+// P = 2^(s * sl2 - m) for a 128-entry score row as 64 fp16 pairs (one pair
+// in four by the polynomial on the FMA pipes, the rest on MUFU); returns the
+// row sum of the fp32 values and raises xpm to the largest polynomial input.
+__device__ __forceinline__ float attn_exp_pack(const float* sv, float sl2, float m, uint32_t* P, float& xpm) {
+  float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
+  const float2 sl2v = make_float2(sl2, sl2), negm = make_float2(-m, -m);
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    const float2 xv = ffma2(make_float2(sv[2 * i], sv[2 * i + 1]), sl2v, negm);
+    float2 pr;
+    if ((i & 3) == 3) {
+      xpm = fmax3(xpm, xv.x, xv.y);
+      pr = exp2_poly2(xv);
+    } else {
+      pr.x = ex2_approx(xv.x);
+      pr.y = ex2_approx(xv.y);
+    }
+    if (i & 1) lb = fadd2(lb, pr); else la = fadd2(la, pr);
+    P[i] = pack_half2(pr.x, pr.y);
+  }
+  const float2 lab = fadd2(la, lb);
+  return lab.x + lab.y;
+}
+
+// One query row's scores against keys kbase .. kbase+127 of one head, in
+// fp32 on the CUDA cores (keys past the row's position get -inf; a row past
+// the tile's valid rows gets zeros).  Only the rare path uses it.
+template <int HD>
+__device__ __forceinline__ void attn_scores_from_global(const AttnParams& p, int head, int qrow, int kbase, int qpos,
+                                                        bool row_valid, float* sv) {
+  const uint4* qr = reinterpret_cast<const uint4*>(p.q + static_cast<int64_t>(qrow) * p.ldqk + head * HD);
+#pragma unroll 1
+  for (int i = 0; i < 128; ++i) {
+    const int key = kbase + i;
+    float acc = row_valid ? -INFINITY : 0.f;
+    if (row_valid && key <= qpos) {
+      const uint4* kr = reinterpret_cast<const uint4*>(p.k + static_cast<int64_t>(key) * p.ldqk + head * HD);
+      acc = 0.f;
+#pragma unroll 1
+      for (int d = 0; d < HD / 8; ++d) {
+        const uint4 a = qr[d], b = kr[d];
+        const __half2* ah = reinterpret_cast<const __half2*>(&a);
+        const __half2* bh = reinterpret_cast<const __half2*>(&b);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 af = __half22float2(ah[e]), bf = __half22float2(bh[e]);
+          acc = fmaf(af.x, bf.x, acc);
+          acc = fmaf(af.y, bf.y, acc);
+        }
+      }
+    }
+    sv[i] = acc;
+  }
 }
 
 // Every lane of the warp waits, then the warp agrees: if any lane gave up
@@ -429,45 +507,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
           for (int i = 0; i < 128; ++i)
             if (kbase + i > qpos) sv[i] = -INFINITY;
         }
-        float m4[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) m4[k] = fmaxf(sv[k], sv[k + 4]);
-#pragma unroll
-        for (int i = 8; i < 128; i += 8)
-#pragma unroll
-          for (int k = 0; k < 4; ++k) m4[k] = fmax3(m4[k], sv[i + k], sv[i + k + 4]);
-        const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
-        // lazy maximum: move to the new one only if it grew by more than 2^8
+        // The row's first tile sets the offset m_used (its maximum); later
+        // tiles reuse it without a maximum pass, which is exact (the final
+        // division by the row sum cancels the common factor) while every
+        // probability fits fp16.  The fp32 row sum bounds the largest
+        // probability, and the largest polynomial input is tracked (the
+        // polynomial is only valid below 2^126): past either bound the tile
+        // takes the rare path, which recomputes the row's scores from Q and K
+        // in global memory and moves the offset to their maximum.
         float f = 1.0f;
         bool need = false;
-        if (kt == 0) {
-          m_used = mt;
-        } else {
-          need = mt > m_used + 8.0f;
-          if (need) {
-            f = ex2_approx(m_used - mt);
-            m_used = mt;
-          }
-        }
-        // P = 2^(s*scale*log2e - m) as fp16 pairs (one pair in four by the
-        // polynomial on the FMA pipes, the rest on MUFU), and its row sum
+        if (kt == 0) m_used = attn_row_max(sv) * sl2;
         uint32_t P[64];
-        float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
-        {
-          const float2 sl2v = make_float2(sl2, sl2), negm = make_float2(-m_used, -m_used);
-#pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            const float2 xv = ffma2(make_float2(sv[2 * i], sv[2 * i + 1]), sl2v, negm);
-            float2 pr;
-            if ((i & 3) == 3) {
-              pr = exp2_poly2(xv);
-            } else {
-              pr.x = ex2_approx(xv.x);
-              pr.y = ex2_approx(xv.y);
-            }
-            if (i & 1) lb = fadd2(lb, pr); else la = fadd2(la, pr);
-            P[i] = pack_half2(pr.x, pr.y);
-          }
+        float xpm = -INFINITY;
+        float lt = attn_exp_pack(sv, sl2, m_used, P, xpm);
+        if (kt > 0 && !(lt <= 32768.0f && xpm < 126.0f)) {
+          float srow[128];  // local memory: the registers of sv stay registers
+          attn_scores_from_global<HD>(p, w.head, T.m0 + row, kbase, qpos, row_valid, srow);
+          const float mt = fmaxf(attn_row_max(srow) * sl2, m_used);
+          f = ex2_approx(m_used - mt);
+          m_used = mt;
+          need = true;
+          lt = attn_exp_pack(srow, sl2, m_used, P, xpm);
         }
         // P_x and O_x are free once the previous PV of this tile has finished
         if (kt > 0) {
@@ -490,8 +551,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
         // keys 2c, 2c+1 -> column c of P
         tmem_st32p(t_p, &P[0]);
         tmem_st32p(t_p + 32, &P[32]);
-        const float2 lab = fadd2(la, lb);
-        l = l * f + (lab.x + lab.y);
+        l = l * f + lt;
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();

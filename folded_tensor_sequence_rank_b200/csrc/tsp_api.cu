@@ -523,6 +523,9 @@ int launch_attention(const Sizes& s, int rank, const tsp_dims* dims, const __hal
   p.timeout_ns = kDefaultTimeoutNs;
   p.lse = lse;
   p.c_pad = static_cast<int>(s.c_pad);
+  p.q = q;
+  p.k = static_cast<const __half*>(k_full);
+  p.ldqk = s.h;
   TSP_CUDA(cudaMemsetAsync(counter, 0, sizeof(int), st));
   const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
   if (s.d == 128) {

@@ -430,7 +430,8 @@ def test_growing_logits_force_rescales(T, h, H, F, D, ramp, n_sample):
     """K rows scaled by 1 + ramp * position / T: the logits grow along the
     sequence, so a row's running maximum grows by 17-25 in log2 units after
     its first key tile (about 0 at these sizes without the ramp), and the
-    attention kernel's lazy rescale of O (growth beyond 2^8), including a
+    attention kernel's move of its offset (a tile whose probabilities would
+    pass 2^15 is redone against the tile's maximum, O rescaled), including a
     growth of more than 2^16 inside one tile, runs many times.  The oracle
     takes the same fp16 K."""
     L = T // D
@@ -459,6 +460,50 @@ def test_growing_logits_force_rescales(T, h, H, F, D, ramp, n_sample):
                            x_all[rows])
         ref = O.rank_rows_forward(x_all[rows], pos[rows], Kf, Vf, w, H)
         assert_layer_close(f64(y)[rows], ref["y"], f"growing logits T={T} D={D} rank {r}", x_all[rows])
+
+
+@pytest.mark.parametrize("T,h,H,F,D,spike", [
+    (512, 256, 4, 1024, 2, 2000.0),     # head_dim 64, every row of both ranks
+    (2048, 512, 4, 2048, 2, 1500.0),    # head_dim 128
+])
+def test_score_jumps_beyond_fp32_range(T, h, H, F, D, spike):
+    """Every 97th K row from position 200 on scaled by `spike`: a query's
+    score against such a key exceeds the maximum of the query's first key
+    tile by hundreds of log2 units (2^x overflows fp32), or by 8 to 128 units
+    (2^x overflows fp16), or falls far below it, at random.  The offset the
+    attention kernel subtracts must follow the row's maximum in all three
+    cases.  The gate is the oracle that rounds Q, K, V and A to fp16 where
+    the kernels store them: with scores hundreds of units apart, Q's fp16
+    rounding alone (relative 2^-11) moves a score by a tenth of a unit, which
+    the softmax turns into output changes above the plain layer's max-abs
+    2e-2 in any fp16 implementation; the plain fp64 layer is checked at
+    rel-L2 5e-3 only."""
+    L = T // D
+    raw = inputs.rank_inputs(L, T, h, F, 9)
+    kf = raw["k_full"].float()
+    spikes = torch.arange(200, T, 97)
+    kf[spikes] *= spike
+    k_spiked = kf.to(torch.float16)
+    assert torch.isfinite(k_spiked).all()
+    dev = to_cuda({n: raw[n] for n in inputs.WEIGHT_NAMES})
+    dims = tsp.make_dims(T, h, H, F)
+    sw = tsp.pack_shards(dims, D, dev)
+    ws = tsp.alloc_workspace(dims, D)
+    Kd, Vd = k_spiked.cuda(), raw["v_full"].cuda()
+    Kf = k_spiked.double().numpy()
+    Vf = raw["v_full"].double().numpy()
+    x_all = f64(raw["x_local"])
+    for r in range(D):
+        y = torch.empty(L, h, dtype=torch.float32, device="cuda")
+        tsp.layer_forward(dims, sw, r, raw["x_local"].cuda(), Kd, Vd, y, ws)
+        assert tsp.get_device_status(ws) == tsp.TSP_OK
+        pos = O.zigzag_index(T, D, r)
+        w = O.stored_weights(weights_f64(raw))
+        ref = O.rank_rows_forward(x_all, pos, Kf, Vf, w, H)
+        assert_layer_close(f64(y), ref["y"], f"score jumps T={T} rank {r}", x_all)
+        plain = O.rank_rows_forward(x_all, pos, Kf, Vf, O.stored_weights(weights_f64(raw), None), H, storage=None)
+        rl = np.linalg.norm(f64(y) - plain["y"]) / np.linalg.norm(plain["y"])
+        assert rl <= 5e-3, f"score jumps T={T} rank {r} vs plain layer: rel-L2 {rl:.3e}"
 
 
 # --------------------------------------------------------------------------
