@@ -47,12 +47,12 @@
 // maximum of its first key tile from every later score, with no maximum pass
 // over the later tiles.  Any common offset is exact (the final division by
 // the row sum cancels it); the offset only has to keep every probability
-// inside fp16's range.  A tile's fp32 row sum bounds its largest probability,
-// and the largest input of the exp2 polynomial is tracked (the polynomial
-// holds below 2^126): a sum above 2^15 or a larger input sends that row's
-// tile down a rare path, which recomputes the row's 128 scores from Q and K
-// in global memory on the CUDA cores, moves the offset to their maximum,
-// redoes the probabilities and rescales O before the next PV.
+// inside fp16's range.  A tile's fp32 row sum bounds its largest probability
+// (every exponential is a MUFU ex2, which gives +inf past fp32's range): a
+// sum above 2^15 sends that row's tile down a rare path, which recomputes the
+// row's 128 scores from Q and K in global memory on the CUDA cores, moves the
+// offset to their maximum, redoes the probabilities and rescales O before the
+// next PV.
 // Q, K, V, P and the output are fp16; scores, softmax statistics and O are
 // fp32.
 #pragma once
@@ -151,23 +151,18 @@ __device__ __forceinline__ float attn_row_max(const float* sv) {
   return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
 }
 
-// P = 2^(s * sl2 - m) for a 128-entry score row as 64 fp16 pairs (one pair
-// in four by the polynomial on the FMA pipes, the rest on MUFU); returns the
-// row sum of the fp32 values and raises xpm to the largest polynomial input.
-__device__ __forceinline__ float attn_exp_pack(const float* sv, float sl2, float m, uint32_t* P, float& xpm) {
+// P = 2^(s * sl2 - m) for a 128-entry score row as 64 fp16 pairs (MUFU
+// ex2: +inf past fp32's range, +0 below it); returns the row sum of the fp32
+// values.
+__device__ __forceinline__ float attn_exp_pack(const float* sv, float sl2, float m, uint32_t* P) {
   float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
   const float2 sl2v = make_float2(sl2, sl2), negm = make_float2(-m, -m);
 #pragma unroll
   for (int i = 0; i < 64; ++i) {
     const float2 xv = ffma2(make_float2(sv[2 * i], sv[2 * i + 1]), sl2v, negm);
     float2 pr;
-    if ((i & 3) == 3) {
-      xpm = fmax3(xpm, xv.x, xv.y);
-      pr = exp2_poly2(xv);
-    } else {
-      pr.x = ex2_approx(xv.x);
-      pr.y = ex2_approx(xv.y);
-    }
+    pr.x = ex2_approx(xv.x);
+    pr.y = ex2_approx(xv.y);
     if (i & 1) lb = fadd2(lb, pr); else la = fadd2(la, pr);
     P[i] = pack_half2(pr.x, pr.y);
   }
@@ -511,24 +506,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
         // tiles reuse it without a maximum pass, which is exact (the final
         // division by the row sum cancels the common factor) while every
         // probability fits fp16.  The fp32 row sum bounds the largest
-        // probability, and the largest polynomial input is tracked (the
-        // polynomial is only valid below 2^126): past either bound the tile
-        // takes the rare path, which recomputes the row's scores from Q and K
-        // in global memory and moves the offset to their maximum.
+        // probability: past 2^15 the tile takes the rare path, which
+        // recomputes the row's scores from Q and K in global memory and moves
+        // the offset to their maximum.
         float f = 1.0f;
         bool need = false;
         if (kt == 0) m_used = attn_row_max(sv) * sl2;
         uint32_t P[64];
-        float xpm = -INFINITY;
-        float lt = attn_exp_pack(sv, sl2, m_used, P, xpm);
-        if (kt > 0 && !(lt <= 32768.0f && xpm < 126.0f)) {
+        float lt = attn_exp_pack(sv, sl2, m_used, P);
+        if (kt > 0 && !(lt <= 32768.0f)) {
           float srow[128];  // local memory: the registers of sv stay registers
           attn_scores_from_global<HD>(p, w.head, T.m0 + row, kbase, qpos, row_valid, srow);
           const float mt = fmaxf(attn_row_max(srow) * sl2, m_used);
           f = ex2_approx(m_used - mt);
           m_used = mt;
           need = true;
-          lt = attn_exp_pack(srow, sl2, m_used, P, xpm);
+          lt = attn_exp_pack(srow, sl2, m_used, P);
         }
         // P_x and O_x are free once the previous PV of this tile has finished
         if (kt > 0) {
