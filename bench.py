@@ -1029,6 +1029,77 @@ def run_sweep_attn_lib(args):
     return line
 
 
+def run_sweep_gemm_lib(args):
+    """Context, not part of the product: the rank step's four GEMMs in this
+    library (per-kernel CUDA events inside one rank step: the QKV product, O
+    with the shard sum and residual, W1 with GELU, W2 with the shard sum and
+    residual) beside cuBLAS (torch.matmul, fp16 operands, fp32 accumulation,
+    fp16 output, no epilogue) on the same M, K, N.  L2 is flushed before every
+    timed launch; each round runs cuBLAS on the four shapes, then one rank
+    step; medians over the rounds."""
+    import torch
+    from folded_tensor_sequence_rank_b200 import tsp
+    wl = WORKLOADS[args.workload]
+    T, h, H, F, D = wl["T"], wl["h"], wl["H"], wl["F"], wl["D"]
+    L = T // D
+    torch.cuda.set_device(0)
+    dims = tsp.make_dims(T, h, H, F)
+    rnd, w_full = _synthetic(T, h, F, wl["seed"])
+    sw = tsp.pack_shards(dims, D, w_full)
+    del w_full
+    kv_std = 0.02 * math.sqrt(h)
+    K = rnd(T, h, std=kv_std, dtype=torch.float16)
+    V = rnd(T, h, std=kv_std, dtype=torch.float16)
+    x = rnd(L, h)
+    y = torch.empty(L, h, dtype=torch.bfloat16, device="cuda")
+    ws = tsp.alloc_workspace(dims, D)
+    shapes = {"qkv": (L, h, 3 * h, 1), "o": (L, h, h, 3), "w1": (L, h, F, 5), "w2": (L, F, h, 6)}
+    mats = {n: (rnd(m, k, dtype=torch.float16), rnd(k, nn, std=0.02, dtype=torch.float16))
+            for n, (m, k, nn, _) in shapes.items()}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(8)]
+    rec = {n: {"cublas": [], "tsp": []} for n in shapes}
+    rounds = max(3, min(args.steps, 10))
+    clocks = None
+    for i in range(args.warmup + rounds):
+        if i == args.warmup:
+            clocks = ClockSampler(0)
+        for n, (a, b) in mats.items():
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch.matmul(a, b)
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                rec[n]["cublas"].append(e0.elapsed_time(e1))
+        flush.zero_()
+        tsp.rank_step(dims, sw, 0, x, K, V, y, ws, events=evs)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            for n, (_, _, _, j) in shapes.items():
+                rec[n]["tsp"].append(evs[j].elapsed_time(evs[j + 1]))
+    clk = clocks.stop()
+    assert tsp.get_device_status(ws) == tsp.TSP_OK
+    res = {}
+    for n, (m, k, nn, _) in shapes.items():
+        fl = 2.0 * m * k * nn
+        d = {"m_k_n": [m, k, nn]}
+        for impl in ("tsp", "cublas"):
+            ms = statistics.median(rec[n][impl])
+            d[f"{impl}_ms"] = round(ms, 4)
+            d[f"{impl}_tflops"] = round(fl / ms / 1e9, 1)
+        res[n] = d
+    tot_tsp = sum(r["tsp_ms"] for r in res.values())
+    tot_cb = sum(r["cublas_ms"] for r in res.values())
+    return {"metric": "the rank step's GEMMs in this library beside cuBLAS on the same shapes (context)",
+            "value": round(tot_cb / tot_tsp, 4), "unit": "cuBLAS time / this library's time, four GEMMs",
+            "n_gpus": 1, "steps": rounds, "warmup": args.warmup, "higher_is_better": True, "dtype": "fp16",
+            "data": "synthetic", "config": {"workload": f"rank 0 of T={T}, D={D}, h={h}, FFN {F}: M = {L} tokens",
+                                            "l2": "flushed (256 MiB write) before every timed launch"},
+            "gemms": res, "clocks": clk}
+
+
 def run_sweep_stack(args):
     """A 32-layer stack of the 7B layer at T = 131072 on one GPU, all D = 8
     ranks in turn per layer (K/V projections, then layer forwards), random
@@ -1092,7 +1163,7 @@ def main():
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the other configurations (all 8 ranks, the shard sweep, the backward, the stack) "
                          "that a default 1-GPU run measures after its main line")
-    ap.add_argument("--sweep", choices=["ranks", "shards", "stack", "mlp_bwd", "layer_bwd", "tp", "attn_lib"],
+    ap.add_argument("--sweep", choices=["ranks", "shards", "stack", "mlp_bwd", "layer_bwd", "tp", "attn_lib", "gemm_lib"],
                     default=None,
                     help="ranks: all 8 ranks of the 128K layer in turn (per-rank spread, whole-layer tokens/s); "
                          "shards: rank 0 at T=32768 for D=1..16; stack: a 32-layer forward at 128K; "
@@ -1100,14 +1171,15 @@ def main():
                          "layer_bwd: the whole layer's backward of rank 0 at 128K; "
                          "tp: the tensor-parallel baseline layer beside a TSP rank step at 128K; "
                          "attn_lib: the rank's attention beside cuDNN, flash-attn 2 and flashinfer kernels "
-                         "on the same work (--workload picks T)")
+                         "on the same work (--workload picks T); "
+                         "gemm_lib: the rank step's four GEMMs beside cuBLAS on the same shapes")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     wl = WORKLOADS[args.workload]
     sweeps = {"ranks": run_sweep_ranks, "shards": run_sweep_shards, "mlp_bwd": run_sweep_mlp_bwd,
               "layer_bwd": run_sweep_layer_bwd, "tp": run_sweep_tp, "stack": run_sweep_stack,
-              "attn_lib": run_sweep_attn_lib}
+              "attn_lib": run_sweep_attn_lib, "gemm_lib": run_sweep_gemm_lib}
     if args.sweep is not None:
         print(json.dumps(sweeps[args.sweep](args)), flush=True)
     elif args.impl == "reference":
