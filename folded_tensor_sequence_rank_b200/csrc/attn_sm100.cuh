@@ -176,12 +176,15 @@ __device__ __forceinline__ float attn_exp_pack(const float* sv, float sl2, float
 template <int HD>
 __device__ __forceinline__ void attn_scores_from_global(const AttnParams& p, int head, int qrow, int kbase, int qpos,
                                                         bool row_valid, float* sv) {
+  // (the debug build checks the row, the head and the row's position, which
+  // bounds every key read below it)
+  const bool ok = row_valid && dbg_ok(qrow < 2 * p.c && qpos < 2 * p.D * p.c && (head + 1) * HD <= p.ldqk, p.status);
   const uint4* qr = reinterpret_cast<const uint4*>(p.q + static_cast<int64_t>(qrow) * p.ldqk + head * HD);
 #pragma unroll 1
   for (int i = 0; i < 128; ++i) {
     const int key = kbase + i;
     float acc = row_valid ? -INFINITY : 0.f;
-    if (row_valid && key <= qpos) {
+    if (ok && key <= qpos) {
       const uint4* kr = reinterpret_cast<const uint4*>(p.k + static_cast<int64_t>(key) * p.ldqk + head * HD);
       acc = 0.f;
 #pragma unroll 1
