@@ -472,15 +472,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
       __syncwarp();
       if (lane == 0) mbar_arrive(&it_empty[slot]);
       if (it < 0) break;
-      const AttnItem w = attn_decode(p, it);
-      const AttnTile T = w.t[x];
-      if (T.nkv == 0) continue;
-      const int qpos = T.p0 + row;
-      const bool row_valid = row < T.nvalid;
+      // Only the key-loop's own values stay live across it (registers are
+      // tight here): the rare path and the epilogue decode the item again.
+      const int nkv_x = attn_decode(p, it).t[x].nkv;
+      if (nkv_x == 0) continue;
+      const int p0_x = attn_decode(p, it).t[x].p0;
+      const int qpos = p0_x + row;
       float m_used = -INFINITY;
       float l = 0.f;
       bool ok = true;
-      for (int kt = 0; kt < T.nkv; ++kt) {
+      for (int kt = 0; kt < nkv_x; ++kt) {
         if (!warp_wait(&s_full[x], scnt & 1, ctl)) { ok = false; break; }
         ++scnt;
         tc_fence_after();
@@ -500,7 +501,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
         if (lane == 0) mbar_arrive(s_free);
         float* sv = reinterpret_cast<float*>(sr);
         const int kbase = kt * kAttnBN;
-        if (kbase + kAttnBN - 1 > T.p0) {  // some key may lie past this row
+        if (kbase + kAttnBN - 1 > p0_x) {  // some key may lie past this row
 #pragma unroll
           for (int i = 0; i < 128; ++i)
             if (kbase + i > qpos) sv[i] = -INFINITY;
@@ -519,7 +520,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
         float lt = attn_exp_pack(sv, sl2, m_used, P);
         if (kt > 0 && !(lt <= 32768.0f)) {
           float srow[128];  // local memory: the registers of sv stay registers
-          attn_scores_from_global<HD>(p, w.head, T.m0 + row, kbase, qpos, row_valid, srow);
+          int it_r = it;
+          asm volatile("" : "+r"(it_r));  // decoded here, not kept live across the loop
+          const AttnItem wr = attn_decode(p, it_r);
+          attn_scores_from_global<HD>(p, wr.head, wr.t[x].m0 + row, kbase, qpos, row < wr.t[x].nvalid, srow);
           const float mt = fmaxf(attn_row_max(srow) * sl2, m_used);
           f = ex2_approx(m_used - mt);
           m_used = mt;
@@ -554,6 +558,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_tcgen05(const __grid
         if (lane == 0) mbar_arrive(&p_full[x]);
       }
       if (!ok) break;
+      int it_e = it;
+      asm volatile("" : "+r"(it_e));
+      const AttnItem w = attn_decode(p, it_e);
+      const AttnTile T = w.t[x];
+      const bool row_valid = row < T.nvalid;
       // epilogue: O / l -> fp16 -> A[m0 + row, head]
       if (!warp_wait(&o_full[x], icnt & 1, ctl)) break;
       ++icnt;
