@@ -470,9 +470,10 @@ def test_score_jumps_beyond_fp32_range(T, h, H, F, D, spike):
     """Every 97th K row from position 200 on scaled by `spike`: a query's
     score against such a key exceeds the maximum of the query's first key
     tile by hundreds of log2 units (2^x overflows fp32), or by 8 to 128 units
-    (2^x overflows fp16), or falls far below it, at random.  The offset the
-    attention kernel subtracts must follow the row's maximum in all three
-    cases.  The gate is the oracle that rounds Q, K, V and A to fp16 where
+    (2^x overflows fp16), or falls far below it, at random
+    (test_score_jump_inputs.py checks on the CPU that all three occur).  The
+    offset the attention kernel subtracts must follow the row's maximum in
+    all three cases.  The gate is the oracle that rounds Q, K, V and A to fp16 where
     the kernels store them: with scores hundreds of units apart, Q's fp16
     rounding alone (relative 2^-11) moves a score by a tenth of a unit, which
     the softmax turns into output changes above the plain layer's max-abs
